@@ -1,0 +1,118 @@
+"""Seeded synthetic inputs for the FP8 block-scaled MoE layer and the block-scale GEMM.
+
+This module only draws random numbers. It holds none of the method's arithmetic:
+no routing, no quantisation, no GEMM. Both the CUDA path (through the binding)
+and the CPU oracle consume what it produces, so the two sides see the same raw
+numbers and derive everything else on their own.
+
+Workloads (DeepSeek-V3-shaped, as in "Accelerate DeepSeek-R1 Inference:
+Integrate AITER into SGLang", section "Complete MoE Implementation"):
+
+  tiny      T=16,    H=256,  E=16,  G=4, TG=2, K=4, I=128
+  decode    T=64,    H=7168, E=256, G=8, TG=4, K=8, I=2048
+  prefill   T=4096,  same layer as decode
+  skewed    T=16384, same layer, correction bias +3.0 on 16 random experts
+  gemm      M=2048, N=4096, K=7168 (single-expert block-scale GEMM)
+
+Draw order for a MoE workload, from one CPU generator seeded with `seed`:
+router logits ~N(0,1) fp32 [T,E], correction bias ~N(0,0.1) fp32 [E], hidden
+states ~N(0,1) rounded to bf16 [T,H], then (skewed only) the 16 hot experts by
+a random permutation. Expert weights ~N(0,0.02) are drawn per expert and per
+matrix from their own generator, seeded from (seed, matrix, expert), on the
+device the caller asks for; a given device always yields the same numbers, so
+any single expert's raw weights can be drawn again later.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    name: str
+    T: int
+    H: int
+    E: int
+    G: int
+    TG: int
+    K: int
+    I: int
+    renorm: bool = True
+    scale: float = 2.5
+    hot_experts: int = 0        # experts that get +hot_bias on the correction bias
+    hot_bias: float = 3.0
+    logit_std: float = 1.0
+    bias_std: float = 0.1
+    x_std: float = 1.0
+    w_std: float = 0.02
+    seed: int = 0
+
+    @property
+    def P(self) -> int:
+        return self.T * self.K
+
+
+@dataclass(frozen=True)
+class GemmConfig:
+    name: str
+    M: int
+    N: int
+    K: int
+    a_std: float = 1.0
+    b_std: float = 0.02
+    seed: int = 0
+
+
+TINY = MoEConfig("tiny_t16_h256_e16", T=16, H=256, E=16, G=4, TG=2, K=4, I=128)
+DECODE = MoEConfig("decode_t64_h7168_e256", T=64, H=7168, E=256, G=8, TG=4, K=8, I=2048)
+PREFILL = MoEConfig("prefill_t4096_h7168_e256", T=4096, H=7168, E=256, G=8, TG=4, K=8, I=2048)
+SKEWED = MoEConfig("skewed_t16384_h7168_e256", T=16384, H=7168, E=256, G=8, TG=4, K=8, I=2048,
+                   hot_experts=16)
+GEMM = GemmConfig("gemm_m2048_n4096_k7168", M=2048, N=4096, K=7168)
+
+MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED)}
+
+
+@dataclass
+class MoEActivations:
+    logits: torch.Tensor      # fp32 [T, E]
+    bias: torch.Tensor        # fp32 [E]
+    x: torch.Tensor           # bf16 [T, H]
+    hot: torch.Tensor = field(default_factory=lambda: torch.empty(0, dtype=torch.int64))
+
+
+def moe_activations(cfg: MoEConfig) -> MoEActivations:
+    """Router logits, correction bias and hidden states on the CPU, in the stated draw order."""
+    g = torch.Generator(device="cpu").manual_seed(cfg.seed)
+    logits = torch.randn(cfg.T, cfg.E, generator=g, dtype=torch.float32) * cfg.logit_std
+    bias = torch.randn(cfg.E, generator=g, dtype=torch.float32) * cfg.bias_std
+    x = (torch.randn(cfg.T, cfg.H, generator=g, dtype=torch.float32) * cfg.x_std).to(torch.bfloat16)
+    hot = torch.empty(0, dtype=torch.int64)
+    if cfg.hot_experts:
+        hot = torch.randperm(cfg.E, generator=g)[: cfg.hot_experts]
+        bias[hot] += cfg.hot_bias
+    return MoEActivations(logits=logits.contiguous(), bias=bias.contiguous(), x=x.contiguous(), hot=hot)
+
+
+_MATRIX_TAG = {"w1": 1, "w2": 2}
+
+
+def _expert_seed(seed: int, which: str, e: int) -> int:
+    return (seed * 1_000_003 + _MATRIX_TAG[which] * 65_537 + e) & 0x7FFF_FFFF_FFFF
+
+
+def expert_weight_raw(cfg: MoEConfig, which: str, e: int, device="cpu") -> torch.Tensor:
+    """Raw fp32 weights of one expert: w1 [2I, H] (gate rows first, then up) or w2 [H, I]."""
+    rows, cols = (2 * cfg.I, cfg.H) if which == "w1" else (cfg.H, cfg.I)
+    g = torch.Generator(device=device).manual_seed(_expert_seed(cfg.seed, which, e))
+    return torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32) * cfg.w_std
+
+
+def gemm_inputs(cfg: GemmConfig, device="cpu"):
+    """A bf16 [M,K] ~N(0,a_std) and B fp32 [N,K] ~N(0,b_std), from one generator on `device`."""
+    g = torch.Generator(device=device).manual_seed(cfg.seed)
+    a = (torch.randn(cfg.M, cfg.K, generator=g, device=device) * cfg.a_std).to(torch.bfloat16)
+    b = torch.randn(cfg.N, cfg.K, generator=g, device=device) * cfg.b_std
+    return a, b
