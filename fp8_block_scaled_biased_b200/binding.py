@@ -1,0 +1,255 @@
+"""ctypes binding of libfp8moe.so: the C ABI in include/fp8moe.h, called with torch tensors.
+
+Argument marshalling only: every function checks dtypes/devices, passes raw
+device pointers and sizes to the library, and raises on a non-zero status.
+All arithmetic happens in the library's CUDA kernels. There is no fallback:
+if the library cannot be loaded, every call raises.
+
+PyTorch is used for device memory and streams only; each call runs on the
+current torch CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp8moe.so")
+
+_c_int, _c_float, _c_size, _p = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+
+_SIGNATURES = {
+    "fp8moe_last_error": (ctypes.c_char_p, []),
+    "fp8moe_device_status": (_c_int, [_p]),
+    "fp8moe_moe_block_m": (_c_int, []),
+    "moe_biased_grouped_topk": (_c_int, [_p, _c_int, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                         _c_int, _c_float, _p]),
+    "moe_align_sort_capacity": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "moe_align_sort_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "moe_align_sort": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_size, _p,
+                                _c_size, _p]),
+    "fp8_per_token_group_quant": (_c_int, [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_int, _p]),
+    "fp8_per_block_quant": (_c_int, [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _p]),
+    "fp8_blockscale_gemm": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _p]),
+    "fused_moe_fp8_blockscale_g1u1_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "fused_moe_fp8_blockscale_g1u1": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
+                                               _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int, _p, _p,
+                                               _c_size, _p]),
+}
+EXPORTED = tuple(_SIGNATURES)
+
+SCALE_ROW_MAJOR = 0
+SCALE_COL_MAJOR = 1
+FP8 = torch.float8_e4m3fn
+
+_lib = None
+
+
+class Fp8MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and type the library; raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} not found: build it with `python -m fp8_block_scaled_biased_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(name, rc):
+    if rc != 0:
+        raise Fp8MoeError(name, rc, load_library().fp8moe_last_error().decode())
+
+
+def _cuda(t, dtype, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _row_major(t, name):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def device_status() -> int:
+    """Synchronise the current stream; return and clear the device error word."""
+    rc = load_library().fp8moe_device_status(_stream())
+    if rc < 0:
+        raise Fp8MoeError("fp8moe_device_status", rc, load_library().fp8moe_last_error().decode())
+    return rc
+
+
+def moe_block_m() -> int:
+    return load_library().fp8moe_moe_block_m()
+
+
+def moe_biased_grouped_topk(gating_output, correction_bias, topk_weights, topk_ids, num_expert_group, topk_group,
+                            need_renorm, routed_scaling_factor=1.0):
+    """Writes topk_weights fp32 [T, topk] and topk_ids int32 [T, topk] (row stride may exceed topk)."""
+    _cuda(gating_output, torch.float32, "gating_output")
+    _cuda(correction_bias, torch.float32, "correction_bias")
+    _cuda(topk_weights, torch.float32, "topk_weights")
+    _cuda(topk_ids, torch.int32, "topk_ids")
+    T, E = gating_output.shape
+    topk = topk_weights.shape[1]
+    ld_out = _row_major(topk_weights, "topk_weights")
+    if _row_major(topk_ids, "topk_ids") != ld_out:
+        raise ValueError("topk_weights and topk_ids must share a row stride")
+    rc = load_library().moe_biased_grouped_topk(
+        _ptr(gating_output), _row_major(gating_output, "gating_output"), _ptr(correction_bias.contiguous()),
+        _ptr(topk_weights), _ptr(topk_ids), ld_out, T, E, topk, num_expert_group, topk_group, int(bool(need_renorm)),
+        float(routed_scaling_factor), _stream())
+    _check("moe_biased_grouped_topk", rc)
+
+
+def moe_align_sort_capacity(T, topk, E, block_m):
+    return load_library().moe_align_sort_capacity(T, topk, E, block_m)
+
+
+@dataclass
+class SortedPairs:
+    sorted_ids: torch.Tensor          # int32 [capacity]
+    sorted_weights: torch.Tensor      # fp32 [capacity]
+    sorted_expert_ids: torch.Tensor   # int32 [capacity // block_m + 1]
+    num_valid_ids: torch.Tensor       # int32 [1] (device)
+    block_m: int
+
+    @property
+    def capacity(self) -> int:
+        return self.sorted_ids.numel()
+
+
+def alloc_sorted(T, topk, E, block_m, device) -> SortedPairs:
+    cap = moe_align_sort_capacity(T, topk, E, block_m)
+    return SortedPairs(
+        sorted_ids=torch.empty(cap, dtype=torch.int32, device=device),
+        sorted_weights=torch.empty(cap, dtype=torch.float32, device=device),
+        sorted_expert_ids=torch.empty(cap // block_m + 1, dtype=torch.int32, device=device),
+        num_valid_ids=torch.empty(1, dtype=torch.int32, device=device),
+        block_m=block_m)
+
+
+def moe_align_sort(topk_ids, topk_weights, num_experts, block_m, out: SortedPairs | None = None) -> SortedPairs:
+    _cuda(topk_ids, torch.int32, "topk_ids")
+    _cuda(topk_weights, torch.float32, "topk_weights")
+    T, topk = topk_ids.shape
+    ld = _row_major(topk_ids, "topk_ids")
+    if _row_major(topk_weights, "topk_weights") != ld:
+        raise ValueError("topk_ids and topk_weights must share a row stride")
+    if out is None:
+        out = alloc_sorted(T, topk, num_experts, block_m, topk_ids.device)
+    lib = load_library()
+    ws_bytes = lib.moe_align_sort_workspace(T, topk, num_experts, block_m)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=topk_ids.device)
+    rc = lib.moe_align_sort(_ptr(topk_ids), _ptr(topk_weights), ld, T, topk, num_experts, block_m,
+                            _ptr(out.sorted_ids), _ptr(out.sorted_weights), _ptr(out.sorted_expert_ids),
+                            _ptr(out.num_valid_ids), out.capacity, _ptr(ws), ws_bytes, _stream())
+    _check("moe_align_sort", rc)
+    return out
+
+
+def fp8_per_token_group_quant(x, group=128, column_major_scales=False, q=None, scales=None):
+    """1 x group FP8 quantisation of bf16 x [M, K] -> (q fp8 [M, K], scales fp32)."""
+    _cuda(x, torch.bfloat16, "x")
+    M, K = x.shape
+    KB = (K + group - 1) // group
+    if q is None:
+        q = torch.empty(M, K, dtype=FP8, device=x.device)
+    if scales is None:
+        scales = torch.empty((KB, M) if column_major_scales else (M, KB), dtype=torch.float32, device=x.device)
+    rc = load_library().fp8_per_token_group_quant(
+        _ptr(x), _row_major(x, "x"), M, K, group, _ptr(q), _ptr(scales),
+        SCALE_COL_MAJOR if column_major_scales else SCALE_ROW_MAJOR, _stream())
+    _check("fp8_per_token_group_quant", rc)
+    return q, scales
+
+
+def fp8_per_block_quant(w, block=128, q=None, scales=None):
+    """128 x 128 FP8 quantisation of fp32 w [N, K] -> (q fp8 [N, K], scales fp32 [N/128, K/128])."""
+    _cuda(w, torch.float32, "w")
+    N, K = w.shape
+    if q is None:
+        q = torch.empty(N, K, dtype=FP8, device=w.device)
+    if scales is None:
+        scales = torch.empty((N + block - 1) // block, (K + block - 1) // block, dtype=torch.float32, device=w.device)
+    rc = load_library().fp8_per_block_quant(_ptr(w), _row_major(w, "w"), N, K, block, _ptr(q), _ptr(scales),
+                                            _stream())
+    _check("fp8_per_block_quant", rc)
+    return q, scales
+
+
+def fp8_blockscale_gemm(A, B, a_scale, b_scale, out=None):
+    """C bf16 [M, N] = block-scaled A fp8 [M, K] x B fp8 [N, K]^T."""
+    _cuda(A, FP8, "A")
+    _cuda(B, FP8, "B")
+    _cuda(a_scale, torch.float32, "a_scale")
+    _cuda(b_scale, torch.float32, "b_scale")
+    M, K = A.shape
+    N = B.shape[0]
+    if not (A.is_contiguous() and B.is_contiguous() and a_scale.is_contiguous() and b_scale.is_contiguous()):
+        raise ValueError("A, B and the scales must be contiguous")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
+    rc = load_library().fp8_blockscale_gemm(_ptr(A), _ptr(B), _ptr(a_scale), _ptr(b_scale), _ptr(out),
+                                            _row_major(out, "out"), M, N, K, _stream())
+    _check("fp8_blockscale_gemm", rc)
+    return out
+
+
+def fused_moe_workspace_bytes(T, topk, E, H, I, block_m):
+    return load_library().fused_moe_fp8_blockscale_g1u1_workspace(T, topk, E, H, I, block_m)
+
+
+def fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_pairs: SortedPairs, topk, a1_scale, fc1_scale, fc2_scale,
+                                  scale_blk_n=128, scale_blk_k=128, fc2_smooth_scale=None, workspace=None):
+    """out bf16 [T, H] = fused g1u1 MoE (GEMM1 + SiLU*up + requant + GEMM2 + weighted combine)."""
+    _cuda(out, torch.bfloat16, "out")
+    _cuda(a8, FP8, "a8")
+    _cuda(w1, FP8, "w1")
+    _cuda(w2, FP8, "w2")
+    T, H = a8.shape
+    E, twoI, _ = w1.shape
+    I = w2.shape[2]
+    if twoI != 2 * I:
+        raise ValueError("g1u1 requires w1.shape[1] == 2 * w2.shape[2]")
+    for name, t in (("out", out), ("a8", a8), ("w1", w1), ("w2", w2), ("a1_scale", a1_scale),
+                    ("fc1_scale", fc1_scale), ("fc2_scale", fc2_scale)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    sp = sorted_pairs
+    lib = load_library()
+    need = lib.fused_moe_fp8_blockscale_g1u1_workspace(T, topk, E, H, I, sp.block_m)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=a8.device)
+    rc = lib.fused_moe_fp8_blockscale_g1u1(
+        _ptr(out), _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights),
+        _ptr(sp.sorted_expert_ids), _ptr(sp.num_valid_ids), T, H, I, E, topk, sp.block_m, sp.capacity,
+        _ptr(a1_scale), _ptr(fc1_scale), _ptr(fc2_scale), scale_blk_n, scale_blk_k, _ptr(fc2_smooth_scale),
+        _ptr(workspace), workspace.numel(), _stream())
+    _check("fused_moe_fp8_blockscale_g1u1", rc)
+    return out

@@ -1,0 +1,401 @@
+// C ABI of the FP8 block-scaled biased MoE layer (declarations and contracts in
+// include/fp8moe.h). Host code: argument checks, TMA tensor maps, launches.
+// All kernels live in this one translation unit so they share the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "gemm_sm100.cuh"
+#include "quant.cuh"
+#include "route.cuh"
+#include "sort.cuh"
+
+using namespace fp8moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  g_last_error.clear();
+  return FP8MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- per-device state
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  std::once_flag once;
+  int sm_count = 0;
+  int err = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+template <int MODE>
+cudaError_t enable_gemm_smem() {
+  return cudaFuncSetAttribute(blockscale_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kGemmSmemBytes));
+}
+
+// Fetches the current device's SM count and opts every kernel into the shared
+// memory it needs, once per device.
+int device_setup(int* sm_count) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8MOE_ECUDA, "device ordinal %d unsupported", dev);
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&] {
+    cudaError_t r = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    int major = 0, minor = 0;
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (r == cudaSuccess && !(major == 10 && minor == 0)) {
+      d.err = -1;
+      return;
+    }
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeDense>();
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeUp>();
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown>();
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(align_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (2 + kSortWarps) * kSortMaxExperts * static_cast<int>(sizeof(int)));
+    d.err = static_cast<int>(r);
+  });
+  if (d.err == -1) return fail(FP8MOE_EUNSUPPORTED, "device %d is not sm_100 (B200)", dev);
+  if (d.err != 0)
+    return fail(FP8MOE_ECUDA, "device setup: %s", cudaGetErrorString(static_cast<cudaError_t>(d.err)));
+  *sm_count = d.sm_count;
+  return FP8MOE_OK;
+}
+
+// ---------------------------------------------------------------- TMA tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D map over a row-major byte matrix [rows, cols] (row stride `ld` bytes), box
+// {128 bytes, box_rows}, 128-byte swizzle, zero fill outside the matrix.
+int make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8MOE_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FP8MOE_ECUDA, "cuTensorMapEncodeTiled failed (%d) for [%llu x %llu]", static_cast<int>(r),
+                static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols));
+  return FP8MOE_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct MoeWorkspace {
+  size_t a2_off, s2_off, y_off, total;
+};
+
+MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I) {
+  MoeWorkspace w;
+  w.a2_off = 0;
+  w.s2_off = round_up(w.a2_off + capacity * static_cast<size_t>(I), 256);
+  w.y_off = round_up(w.s2_off + static_cast<size_t>(I / 128) * capacity * sizeof(float), 256);
+  w.total = round_up(w.y_off + static_cast<size_t>(T) * topk * H * sizeof(float), 256);
+  return w;
+}
+
+int choose_group_m(int n_tiles) {
+  // Visit a few consecutive row blocks per column tile so blocks of the same
+  // expert share each weight tile while it is in L2.
+  return n_tiles >= 8 ? 4 : 16;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fp8moe_last_error(void) { return g_last_error.c_str(); }
+
+int fp8moe_moe_block_m(void) { return kBM; }
+
+int fp8moe_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    fail(FP8MOE_ECUDA, "stream synchronize: %s", cudaGetErrorString(e));
+    return -1;
+  }
+  unsigned int word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) {
+    fail(FP8MOE_ECUDA, "device status: %s", cudaGetErrorString(e));
+    return -1;
+  }
+  return static_cast<int>(word);
+}
+
+// ------------------------------------------------------------------ S1 routing
+int moe_biased_grouped_topk(const float* gating_output, int ld_in, const float* correction_bias, float* topk_weights,
+                            int32_t* topk_ids, int ld_out, int T, int E, int topk, int num_expert_group,
+                            int topk_group, int need_renorm, float routed_scaling_factor, void* stream) {
+  if (T < 0) return fail(FP8MOE_EINVAL, "T must be >= 0 (got %d)", T);
+  if (E < 1 || E > 32 * kRouteMaxPerLane) return fail(FP8MOE_EUNSUPPORTED, "E must be in [1, 512] (got %d)", E);
+  if (num_expert_group < 1 || num_expert_group > 32 || E % num_expert_group != 0)
+    return fail(FP8MOE_EINVAL, "num_expert_group must divide E and be <= 32 (E=%d, groups=%d)", E,
+                num_expert_group);
+  if (topk_group < 1 || topk_group > num_expert_group)
+    return fail(FP8MOE_EINVAL, "topk_group must be in [1, num_expert_group] (got %d)", topk_group);
+  const int per_group = E / num_expert_group;
+  if (topk < 1 || topk > 32 || topk > topk_group * per_group)
+    return fail(FP8MOE_EINVAL, "topk must be in [1, min(32, topk_group*E/groups)] (got %d)", topk);
+  if (ld_in < E) return fail(FP8MOE_EINVAL, "ld_in (%d) < E (%d)", ld_in, E);
+  if (ld_out < topk) return fail(FP8MOE_EINVAL, "ld_out (%d) < topk (%d)", ld_out, topk);
+  if (T == 0) return FP8MOE_OK;
+  if (!gating_output || !correction_bias || !topk_weights || !topk_ids)
+    return fail(FP8MOE_EINVAL, "null pointer argument");
+  // experts per lane: the smallest divisor of the group size that covers E with 32 lanes
+  const int need = (E + 31) / 32;
+  int per_lane = 0;
+  for (int d = need; d <= per_group; ++d)
+    if (per_group % d == 0) {
+      per_lane = d;
+      break;
+    }
+  if (per_lane == 0 || per_lane > kRouteMaxPerLane)
+    return fail(FP8MOE_EUNSUPPORTED, "group size %d cannot be split over 32 lanes", per_group);
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const dim3 grid((T + kRouteWarps - 1) / kRouteWarps);
+  route_kernel<<<grid, 32 * kRouteWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+      gating_output, ld_in, correction_bias, topk_weights, topk_ids, ld_out, T, E, topk, num_expert_group,
+      topk_group, need_renorm ? 1 : 0, routed_scaling_factor, per_lane);
+  return check_launch("moe_biased_grouped_topk");
+}
+
+// ------------------------------------------------------------------ S2 align/sort
+size_t moe_align_sort_capacity(int T, int topk, int E, int block_m) {
+  if (T < 0 || topk < 1 || E < 1 || block_m < 1) return 0;
+  return static_cast<size_t>(T) * topk + static_cast<size_t>(E) * (block_m - 1);
+}
+
+size_t moe_align_sort_workspace(int, int, int, int) { return 0; }
+
+int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, int T, int topk, int E, int block_m,
+                   int32_t* sorted_ids, float* sorted_weights, int32_t* sorted_expert_ids, int32_t* num_valid_ids,
+                   size_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (T < 0 || topk < 1) return fail(FP8MOE_EINVAL, "T >= 0 and topk >= 1 required");
+  if (E < 1 || E > kSortMaxExperts) return fail(FP8MOE_EUNSUPPORTED, "E must be in [1, %d]", kSortMaxExperts);
+  if (block_m < 1 || block_m > 1024) return fail(FP8MOE_EINVAL, "block_m must be in [1, 1024]");
+  if (ld < topk) return fail(FP8MOE_EINVAL, "ld (%d) < topk (%d)", ld, topk);
+  if (static_cast<long long>(T) * topk >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "T*topk too large");
+  if (capacity < moe_align_sort_capacity(T, topk, E, block_m))
+    return fail(FP8MOE_EINVAL, "capacity %zu < required %zu", capacity, moe_align_sort_capacity(T, topk, E, block_m));
+  if (!sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids || (T > 0 && (!topk_ids || !topk_weights)))
+    return fail(FP8MOE_EINVAL, "null pointer argument");
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const size_t smem = static_cast<size_t>(2 + kSortWarps) * E * sizeof(int);
+  align_sort_kernel<<<1, kSortThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      topk_ids, topk_weights, ld, T, topk, E, block_m, sorted_ids, sorted_weights, sorted_expert_ids, num_valid_ids);
+  return check_launch("moe_align_sort");
+}
+
+// ------------------------------------------------------------------ S3 quant
+int fp8_per_token_group_quant(const uint16_t* x, int ld_x, int M, int K, int group, uint8_t* q, float* scales,
+                              int scale_layout, void* stream) {
+  if (group != 128) return fail(FP8MOE_EUNSUPPORTED, "only group == 128 is supported (got %d)", group);
+  if (M < 0 || K < 0) return fail(FP8MOE_EINVAL, "negative size");
+  if (K % 8 != 0) return fail(FP8MOE_EUNSUPPORTED, "K must be a multiple of 8 (got %d)", K);
+  if (ld_x < K || ld_x % 8 != 0) return fail(FP8MOE_EINVAL, "ld_x must be >= K and a multiple of 8");
+  if (scale_layout != FP8MOE_SCALE_ROW_MAJOR && scale_layout != FP8MOE_SCALE_COL_MAJOR)
+    return fail(FP8MOE_EINVAL, "unknown scale_layout %d", scale_layout);
+  if (M == 0 || K == 0) return FP8MOE_OK;
+  if (!x || !q || !scales) return fail(FP8MOE_EINVAL, "null pointer argument");
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7u)) return fail(FP8MOE_EINVAL, "x must be 16-byte and q 8-byte aligned");
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const dim3 grid((M + kQuantWarps - 1) / kQuantWarps);
+  quant_1x128_kernel<<<grid, 32 * kQuantWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(x), ld_x, M, K, q, scales, scale_layout == FP8MOE_SCALE_COL_MAJOR);
+  return check_launch("fp8_per_token_group_quant");
+}
+
+int fp8_per_block_quant(const float* w, int ld_w, int N, int K, int block, uint8_t* q, float* scales, void* stream) {
+  if (block != 128) return fail(FP8MOE_EUNSUPPORTED, "only block == 128 is supported (got %d)", block);
+  if (N < 0 || K < 0 || ld_w < K) return fail(FP8MOE_EINVAL, "bad size or stride");
+  if (N == 0 || K == 0) return FP8MOE_OK;
+  if (!w || !q || !scales) return fail(FP8MOE_EINVAL, "null pointer argument");
+  if ((N + 127) / 128 > 65535) return fail(FP8MOE_EUNSUPPORTED, "N too large");
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const dim3 grid((K + 127) / 128, (N + 127) / 128);
+  quant_128x128_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(w, ld_w, N, K, q, scales);
+  return check_launch("fp8_per_block_quant");
+}
+
+// ------------------------------------------------------------------ S0 GEMM
+int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale, const float* b_scale, uint16_t* C,
+                        int ldc, int M, int N, int K, void* stream) {
+  if (M < 1 || N < 1 || K < 1) return fail(FP8MOE_EINVAL, "M, N, K must be >= 1");
+  if (K % 16 != 0) return fail(FP8MOE_EUNSUPPORTED, "K must be a multiple of 16 (got %d)", K);
+  if (ldc < N) return fail(FP8MOE_EINVAL, "ldc (%d) < N (%d)", ldc, N);
+  if (!A || !B || !a_scale || !b_scale || !C) return fail(FP8MOE_EINVAL, "null pointer argument");
+  if (!aligned16(A) || !aligned16(B)) return fail(FP8MOE_EINVAL, "A and B must be 16-byte aligned");
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  CUtensorMap ma, mb;
+  if (int rc = make_map_u8(&ma, A, M, K, K, 128)) return rc;
+  if (int rc = make_map_u8(&mb, B, N, K, K, 128)) return rc;
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.num_kb = (K + 127) / 128;
+  a.n_tiles = (N + kBN - 1) / kBN;
+  a.group_m = choose_group_m(a.n_tiles);
+  a.a_scale = a_scale;
+  a.b_scale = b_scale;
+  a.nb_per_expert = (N + 127) / 128;
+  a.nb_valid = a.nb_per_expert;
+  a.C = reinterpret_cast<__nv_bfloat16*>(C);
+  a.ldc = ldc;
+  a.c_vec_ok = (ldc % 8 == 0) && aligned16(C);
+  a.b_rows_per_expert = 0;
+  const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * a.n_tiles;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  blockscale_gemm_kernel<kModeDense><<<grid, kGemmThreads, kGemmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      ma, mb, a);
+  return check_launch("fp8_blockscale_gemm");
+}
+
+// ------------------------------------------------------------------ S4-S7 fused MoE
+size_t fused_moe_fp8_blockscale_g1u1_workspace(int T, int topk, int E, int H, int I, int block_m) {
+  if (T < 0 || topk < 1 || E < 1 || H < 1 || I < 1 || block_m < 1) return 0;
+  return moe_workspace_layout(moe_align_sort_capacity(T, topk, E, block_m), T, topk, H, I).total;
+}
+
+int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_t* w1, const uint8_t* w2,
+                                  const int32_t* sorted_ids, const float* sorted_weights,
+                                  const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H, int I,
+                                  int E, int topk, int block_m, size_t capacity, const float* a1_scale,
+                                  const float* fc1_scale, const float* fc2_scale, int scale_blk_n, int scale_blk_k,
+                                  const float* fc2_smooth_scale, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (scale_blk_n != 128 || scale_blk_k != 128)
+    return fail(FP8MOE_EUNSUPPORTED, "only (128, 128) scale blocks are supported (got %d, %d)", scale_blk_n,
+                scale_blk_k);
+  if (fc2_smooth_scale) return fail(FP8MOE_EUNSUPPORTED, "fc2_smooth_scale must be NULL");
+  if (block_m != kBM) return fail(FP8MOE_EUNSUPPORTED, "block_m must be %d (got %d)", kBM, block_m);
+  if (T < 0 || E < 1 || topk < 1 || topk > E) return fail(FP8MOE_EINVAL, "bad T, E or topk");
+  if (H < 128 || I < 128 || H % 128 || I % 128)
+    return fail(FP8MOE_EUNSUPPORTED, "H and I must be positive multiples of 128 (H=%d, I=%d)", H, I);
+  if (static_cast<long long>(T) * topk >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "T*topk too large");
+  if (capacity < moe_align_sort_capacity(T, topk, E, block_m) || capacity >= (1ull << 31))
+    return fail(FP8MOE_EINVAL, "capacity %zu below the sort's bound %zu", capacity,
+                moe_align_sort_capacity(T, topk, E, block_m));
+  if (T == 0) return FP8MOE_OK;
+  if (!out || !a8 || !w1 || !w2 || !sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids ||
+      !a1_scale || !fc1_scale || !fc2_scale)
+    return fail(FP8MOE_EINVAL, "null pointer argument");
+  if (!aligned16(a8) || !aligned16(w1) || !aligned16(w2) || !aligned16(sorted_ids) || !aligned16(out))
+    return fail(FP8MOE_EINVAL, "a8, w1, w2, sorted_ids and out must be 16-byte aligned");
+  const MoeWorkspace lay = moe_workspace_layout(capacity, T, topk, H, I);
+  if (!workspace || workspace_bytes < lay.total)
+    return fail(FP8MOE_EWORKSPACE, "workspace of %zu bytes needed (got %zu)", lay.total, workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(FP8MOE_EINVAL, "workspace must be 256-byte aligned");
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* a2 = ws + lay.a2_off;
+  float* s2 = reinterpret_cast<float*>(ws + lay.s2_off);
+  float* ystage = reinterpret_cast<float*>(ws + lay.y_off);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap m_a8, m_w1, m_a2, m_w2;
+  if (int rc = make_map_u8(&m_a8, a8, T, H, H, 1)) return rc;
+  if (int rc = make_map_u8(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H, H, 128)) return rc;
+  if (int rc = make_map_u8(&m_a2, a2, capacity, I, I, 128)) return rc;
+  if (int rc = make_map_u8(&m_w2, w2, static_cast<uint64_t>(E) * H, I, I, 128)) return rc;
+
+  GemmArgs up{};
+  up.M = static_cast<int>(capacity);
+  up.N = I;
+  up.num_kb = H / 128;
+  up.n_tiles = I / 128;
+  up.group_m = choose_group_m(up.n_tiles);
+  up.a_scale = a1_scale;
+  up.b_scale = fc1_scale;
+  up.nb_per_expert = 2 * I / 128;
+  up.nb_valid = up.nb_per_expert;
+  up.sorted_ids = sorted_ids;
+  up.sorted_expert_ids = sorted_expert_ids;
+  up.num_valid_ids = num_valid_ids;
+  up.sorted_weights = sorted_weights;
+  up.T = T;
+  up.topk = topk;
+  up.E = E;
+  up.b_rows_per_expert = 2 * I;
+  up.a2 = a2;
+  up.s2 = s2;
+  blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8, m_w1, up);
+  if (int rc = check_launch("fused_moe (gate/up GEMM)")) return rc;
+
+  GemmArgs dn = up;
+  dn.N = H;
+  dn.num_kb = I / 128;
+  dn.n_tiles = (H + kBN - 1) / kBN;
+  dn.group_m = choose_group_m(dn.n_tiles);
+  dn.a_scale = s2;
+  dn.b_scale = fc2_scale;
+  dn.nb_per_expert = H / 128;
+  dn.nb_valid = H / 128;
+  dn.b_rows_per_expert = H;
+  dn.ystage = ystage;
+  blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
+  if (int rc = check_launch("fused_moe (down GEMM)")) return rc;
+
+  const size_t threads = static_cast<size_t>(T) * (H / 8);
+  moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(ystage, T, topk, H,
+                                                                                   reinterpret_cast<__nv_bfloat16*>(out));
+  return check_launch("fused_moe (combine)");
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+"""The FP8 block-scaled MoE layer as one object: weights resident on the device,
+buffers preallocated, forward = route -> align/sort -> 1x128 quant -> fused g1u1 MoE.
+
+This mirrors the composition the pages' asm_moe wrapper performs ("Accelerate
+DeepSeek-R1 Inference: Integrate AITER into SGLang", section "Blockscale FP8
+MoE Computation"): sorting, activation quantisation with transposed scales,
+then fmoe_fp8_blockscale_g1u1. Every step is a call into the CUDA library.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+from . import inputs as I
+
+
+class MoELayer:
+    def __init__(self, cfg: I.MoEConfig, device="cuda", max_tokens: int | None = None):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.max_tokens = max_tokens or cfg.T
+        E, H, Im = cfg.E, cfg.H, cfg.I
+        dev = self.device
+        self.w1 = torch.empty(E, 2 * Im, H, dtype=B.FP8, device=dev)
+        self.w1_scale = torch.empty(E, 2 * Im // 128, H // 128, dtype=torch.float32, device=dev)
+        self.w2 = torch.empty(E, H, Im, dtype=B.FP8, device=dev)
+        self.w2_scale = torch.empty(E, H // 128, Im // 128, dtype=torch.float32, device=dev)
+        self.block_m = B.moe_block_m()
+        self._alloc(self.max_tokens)
+
+    def _alloc(self, T):
+        cfg, dev = self.cfg, self.device
+        self.topk_w = torch.empty(T, cfg.K, dtype=torch.float32, device=dev)
+        self.topk_ids = torch.empty(T, cfg.K, dtype=torch.int32, device=dev)
+        self.sorted = B.alloc_sorted(T, cfg.K, cfg.E, self.block_m, dev)
+        self.a8 = torch.empty(T, cfg.H, dtype=B.FP8, device=dev)
+        self.a8_scale = torch.empty(cfg.H // 128, T, dtype=torch.float32, device=dev)
+        self.out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
+        ws = B.fused_moe_workspace_bytes(T, cfg.K, cfg.E, cfg.H, cfg.I, self.block_m)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+
+    def load_synthetic_weights(self):
+        """Draw each expert's raw fp32 weights on the device and quantise them in 128x128 blocks."""
+        for e in range(self.cfg.E):
+            raw1 = I.expert_weight_raw(self.cfg, "w1", e, self.device)
+            B.fp8_per_block_quant(raw1, q=self.w1[e], scales=self.w1_scale[e])
+            raw2 = I.expert_weight_raw(self.cfg, "w2", e, self.device)
+            B.fp8_per_block_quant(raw2, q=self.w2[e], scales=self.w2_scale[e])
+        return self
+
+    def forward(self, logits, bias, x):
+        """logits fp32 [T, E], bias fp32 [E], x bf16 [T, H] (all on the device) -> bf16 [T, H]."""
+        cfg = self.cfg
+        T = x.shape[0]
+        if T != self.max_tokens:
+            raise ValueError(f"layer buffers are sized for {self.max_tokens} tokens, got {T}")
+        B.moe_biased_grouped_topk(logits, bias, self.topk_w, self.topk_ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+        B.moe_align_sort(self.topk_ids, self.topk_w, cfg.E, self.block_m, out=self.sorted)
+        B.fp8_per_token_group_quant(x, 128, column_major_scales=True, q=self.a8, scales=self.a8_scale)
+        B.fused_moe_fp8_blockscale_g1u1(self.out, self.a8, self.w1, self.w2, self.sorted, cfg.K, self.a8_scale,
+                                        self.w1_scale, self.w2_scale, workspace=self.workspace)
+        return self.out
+
+    # kernels launched by one forward: route, sort, quant, gate/up GEMM, down GEMM, combine
+    LAUNCHES_PER_FORWARD = 6

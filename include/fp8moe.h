@@ -1,0 +1,217 @@
+/*
+ * fp8moe.h - C ABI of the B200 (sm_100a) FP8 block-scaled biased MoE layer.
+ *
+ * The operations, their argument order and their tensor layouts follow
+ * "Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang"
+ * (rocm.blogs.amd.com), section "Complete MoE Implementation" (Top-K routing,
+ * MoE Sorting, Blockscale FP8 MoE Computation) and section "General Linear
+ * Layer" (FP8 blockscale GEMM). FP8 is OCP E4M3 "fn" (largest finite 448), not
+ * the MI300X "fnuz" variant.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or keeps them. Scratch memory is passed in as
+ *     `workspace`, sized by the matching *_workspace query.
+ *   - Matrices are row-major; `ld*` arguments are row strides in elements.
+ *   - FP8 tensors are bytes (uint8_t) holding E4M3fn codes; bf16 tensors are
+ *     uint16_t holding bfloat16 bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
+ *     only enqueues work on it and returns without synchronising, so a chain of
+ *     calls can be captured in a CUDA graph. No value travels back to the host:
+ *     `num_valid_ids` stays on the device and the kernels read it there.
+ *   - Return value: FP8MOE_OK, or an error code with nothing launched (argument
+ *     errors) or a launch error (FP8MOE_ECUDA). fp8moe_last_error() returns a
+ *     message for the calling thread's last failure.
+ *   - Faults the kernels detect on the device (an expert id out of range, a
+ *     bounded wait that expired) set a device error word instead of trapping;
+ *     fp8moe_device_status() reports and clears it.
+ */
+#ifndef FP8MOE_H
+#define FP8MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum fp8moe_status {
+  FP8MOE_OK = 0,
+  FP8MOE_EINVAL = 1,        /* bad pointer, size, stride or argument combination */
+  FP8MOE_EUNSUPPORTED = 2,  /* a valid request this library does not implement   */
+  FP8MOE_EWORKSPACE = 3,    /* workspace missing or smaller than the query       */
+  FP8MOE_ECUDA = 4,         /* CUDA runtime/driver error (launch, device query)  */
+  FP8MOE_EDEVICE = 5        /* device-detected fault (fp8moe_device_status only) */
+};
+
+/* Device error word bits reported by fp8moe_device_status(). */
+enum fp8moe_device_error {
+  FP8MOE_DEVERR_TIMEOUT = 1u,     /* a bounded wait inside a GEMM kernel expired  */
+  FP8MOE_DEVERR_EXPERT_ID = 2u,   /* an expert id outside [0, E) was met          */
+  FP8MOE_DEVERR_PAIR_ID = 4u,     /* a sorted pair id outside [0, T*topk] was met */
+  FP8MOE_DEVERR_NUM_VALID = 8u    /* num_valid_ids above capacity or not a multiple of block_m */
+};
+
+/* Message describing the calling thread's most recent failure ("" if none). */
+const char* fp8moe_last_error(void);
+
+/* Synchronises `stream`, then returns and clears the device error word of the
+ * current device (0 = no fault seen). Returns -1 with a message if the
+ * synchronisation itself fails. */
+int fp8moe_device_status(void* stream);
+
+/* Block size of the M (token-expert pair) dimension that the fused MoE kernels
+ * tile by; moe_align_sort must be called with block_m equal to this. */
+int fp8moe_moe_block_m(void);
+
+/*
+ * S1 - biased grouped top-k routing.  (Top-K routing: biased_grouped_topk(
+ *      gating_output, correction_bias, topk_weights, topk_ids,
+ *      num_expert_group, topk_group, need_renorm, routed_scaling_factor).)
+ *
+ * gating_output   fp32 [T, E], row stride ld_in >= E
+ * correction_bias fp32 [E]
+ * topk_weights    fp32 [T, topk], row stride ld_out >= topk (gap columns are
+ *                 not written; the pages allocate these outputs strided)
+ * topk_ids        int32 [T, topk], same row stride ld_out
+ * Per token: s = sigmoid(logit), b = s + bias. Group score = sum of the two
+ * largest b of the group's E/num_expert_group experts. The topk_group best
+ * groups are kept (ties: lower group index), then the topk best experts by b
+ * among them (ties: lower expert index), written in that rank order. Weights
+ * are the unbiased s, divided by their sum if need_renorm, then multiplied by
+ * routed_scaling_factor. sigmoid uses a fixed fp32 operation sequence so the
+ * ids are reproducible bit for bit.
+ * Limits: 1 <= E <= 512, E % num_expert_group == 0, num_expert_group <= 32,
+ * 1 <= topk_group <= num_expert_group, 1 <= topk <= 32,
+ * topk <= topk_group * (E / num_expert_group). T == 0 is a no-op.
+ */
+int moe_biased_grouped_topk(const float* gating_output, int ld_in,
+                            const float* correction_bias,
+                            float* topk_weights, int32_t* topk_ids, int ld_out,
+                            int T, int E, int topk, int num_expert_group,
+                            int topk_group, int need_renorm,
+                            float routed_scaling_factor, void* stream);
+
+/*
+ * S2 - MoE align/sort.  (MoE Sorting: moe_sorting(topk_ids, topk_weights, E,
+ *      model_dim, dtype) -> sorted_token_ids, sorted_weight_buf,
+ *      sorted_expert_ids, num_valid_ids.)
+ *
+ * topk_ids int32 [T, topk] and topk_weights fp32 [T, topk], row stride ld.
+ * Pair (t, k) is named by its flat id p = t*topk + k. Experts are laid out in
+ * ascending id order, each expert's pairs in ascending p, each segment padded
+ * to a multiple of block_m with id T*topk and weight 0; experts without pairs
+ * get no block.
+ * Outputs (device): sorted_ids int32 [capacity], sorted_weights fp32
+ * [capacity], sorted_expert_ids int32 [capacity / block_m] (one expert per
+ * block), num_valid_ids int32 [1] (= padded length). Entries past the padded
+ * length are left untouched. capacity must be >= moe_align_sort_capacity().
+ * An id outside [0, E) is dropped and flagged (FP8MOE_DEVERR_EXPERT_ID).
+ * Limits: 1 <= E <= 1024, 1 <= block_m <= 1024, T*topk < 2^31.
+ */
+size_t moe_align_sort_capacity(int T, int topk, int E, int block_m);
+size_t moe_align_sort_workspace(int T, int topk, int E, int block_m);
+int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld,
+                   int T, int topk, int E, int block_m,
+                   int32_t* sorted_ids, float* sorted_weights,
+                   int32_t* sorted_expert_ids, int32_t* num_valid_ids,
+                   size_t capacity, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/*
+ * S3 - dynamic per-token-group FP8 quantisation (1 x group).
+ *      (dynamic_per_token_scaled_fp8_quant on hidden states viewed as
+ *      [M*H/128, 128]; per_token_group_quant_fp8(x, 128, column_major_scales).)
+ *
+ * x      bf16 [M, K], row stride ld_x (elements)
+ * q      fp8 [M, K], row stride K
+ * scales fp32 [M, ceil(K/group)] if scale_layout == FP8MOE_SCALE_ROW_MAJOR, or
+ *        [ceil(K/group), M] if FP8MOE_SCALE_COL_MAJOR (the transposed layout the
+ *        fused MoE call takes).
+ * scale = amax / 448 (fp32), q = E4M3fn(x / scale) rounded to nearest even and
+ * saturated; an all-zero group gives scale 0 and codes 0.
+ * Limits: group == 128; K % 8 == 0; ld_x % 8 == 0; x 16-byte aligned.
+ */
+enum { FP8MOE_SCALE_ROW_MAJOR = 0, FP8MOE_SCALE_COL_MAJOR = 1 };
+int fp8_per_token_group_quant(const uint16_t* x, int ld_x, int M, int K, int group,
+                              uint8_t* q, float* scales, int scale_layout,
+                              void* stream);
+
+/*
+ * Weight preparation - FP8 quantisation in 128 x 128 blocks (the recipe behind
+ * the "*_weight_scale_inv" tensors of the pages' MoE and linear layers).
+ *
+ * w      fp32 [N, K], row stride ld_w
+ * q      fp8 [N, K], row stride K
+ * scales fp32 [ceil(N/128), ceil(K/128)]; scale = amax / 448 over the block,
+ *        q = E4M3fn(w / scale); dequantised weight = q * scale.
+ * Limits: block == 128.
+ */
+int fp8_per_block_quant(const float* w, int ld_w, int N, int K, int block,
+                        uint8_t* q, float* scales, void* stream);
+
+/*
+ * S0 - FP8 block-scale GEMM.  (General Linear Layer:
+ *      gemm_a8w8_blockscale(XQ, WQ, x_scale, w_scale, dtype) -> Y.)
+ *
+ * A       fp8 [M, K] row-major (K contiguous)
+ * B       fp8 [N, K] row-major (the weight, K contiguous)
+ * a_scale fp32 [M, ceil(K/128)] row-major (one scale per 1x128 group of A)
+ * b_scale fp32 [ceil(N/128), ceil(K/128)] (one scale per 128x128 block of B)
+ * C       bf16 [M, N], row stride ldc >= N
+ * C[m,n] = bf16( sum_kb a_scale[m,kb] * b_scale[n/128,kb] *
+ *                sum_{k in kb} A[m,k] * B[n,k] ), fp32 accumulation.
+ * Limits: K % 16 == 0 (TMA row alignment); A, B 16-byte aligned; M, N >= 1.
+ */
+int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B,
+                        const float* a_scale, const float* b_scale,
+                        uint16_t* C, int ldc, int M, int N, int K, void* stream);
+
+/*
+ * S4-S7 - fused g1u1 MoE with 128x128 weight scales.
+ *      (Blockscale FP8 MoE Computation: fmoe_fp8_blockscale_g1u1(out, a8, w1,
+ *      w2, sorted_ids, sorted_weights, sorted_expert_ids, num_valid_ids, topk,
+ *      a1_scale, fc1_scale, fc2_scale, scale_blk_n, scale_blk_k,
+ *      fc2_smooth_scale).)
+ *
+ * out        bf16 [T, H] (every row written)
+ * a8         fp8 [T, H] quantised hidden states
+ * w1         fp8 [E, 2I, H]; rows [0, I) of each expert are the gate
+ *            projection, rows [I, 2I) the up projection
+ * w2         fp8 [E, H, I]
+ * sorted_*   the outputs of moe_align_sort with block_m == fp8moe_moe_block_m()
+ * a1_scale   fp32 [H/128, T] (transposed 1x128 scales of a8)
+ * fc1_scale  fp32 [E, 2I/128, H/128];  fc2_scale fp32 [E, H/128, I/128]
+ * For every pair p = (t, k) with expert e:
+ *   g = blockscale(a8[t], w1[e]) (fp32), h = silu(g[:I]) * g[I:],
+ *   a2 = 1x128 FP8 quantisation of h (as fp8_per_token_group_quant),
+ *   y_p = blockscale(a2, w2[e]),
+ *   out[t] = bf16( sum_{k=0..topk-1} w_{t,k} * y_{t,k} ) summed in slot order,
+ * which makes the output independent of scheduling (deterministic).
+ * Limits: scale_blk_n == scale_blk_k == 128; H % 128 == 0; I % 128 == 0;
+ * fc2_smooth_scale must be NULL (the pages do not define it); workspace >=
+ * fused_moe_fp8_blockscale_g1u1_workspace(); capacity >= the sort's padded
+ * length.
+ */
+size_t fused_moe_fp8_blockscale_g1u1_workspace(int T, int topk, int E, int H, int I,
+                                                int block_m);
+int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8,
+                                  const uint8_t* w1, const uint8_t* w2,
+                                  const int32_t* sorted_ids,
+                                  const float* sorted_weights,
+                                  const int32_t* sorted_expert_ids,
+                                  const int32_t* num_valid_ids,
+                                  int T, int H, int I, int E, int topk,
+                                  int block_m, size_t capacity,
+                                  const float* a1_scale, const float* fc1_scale,
+                                  const float* fc2_scale, int scale_blk_n,
+                                  int scale_blk_k, const float* fc2_smooth_scale,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8MOE_H */

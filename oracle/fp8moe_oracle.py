@@ -37,13 +37,9 @@ QUANT_GROUP = 128           # 1x128 activation groups and 128x128 weight blocks
 # OCP FP8 E4M3 ("fn") codec
 # ---------------------------------------------------------------------------
 
-def e4m3_decode(codes: torch.Tensor) -> torch.Tensor:
-    """Value of each FP8 E4M3fn code, in fp64.
-
-    OCP E4M3: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no
-    infinities; exponent field 0 holds subnormals m/8 * 2^-6; S.1111.111 is NaN.
-    """
-    c = codes.to(torch.int64) & 0xFF
+def _e4m3_value_of_code(c: torch.Tensor) -> torch.Tensor:
+    """OCP E4M3: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no
+    infinities; exponent field 0 holds subnormals m/8 * 2^-6; S.1111.111 is NaN."""
     sign = torch.where((c >> 7) == 1, -1.0, 1.0).to(F64)
     exp = (c >> 3) & 0xF
     man = (c & 0x7).to(F64)
@@ -53,24 +49,33 @@ def e4m3_decode(codes: torch.Tensor) -> torch.Tensor:
     return torch.where((exp == 0xF) & ((c & 7) == 7), torch.tensor(float("nan"), dtype=F64), val)
 
 
+_E4M3_TABLE = _e4m3_value_of_code(torch.arange(256, dtype=torch.int64))
+
+
+def e4m3_decode(codes: torch.Tensor) -> torch.Tensor:
+    """Value of each FP8 E4M3fn code, in fp64 (looked up in the 256-entry table above)."""
+    return _E4M3_TABLE[codes.to(torch.int64) & 0xFF]
+
+
 def e4m3_encode(x: torch.Tensor) -> torch.Tensor:
     """Round fp32 values to E4M3fn codes: round-to-nearest-even, saturating to +-448.
 
     Magnitudes above 448 (and +-inf) become +-448 (code 0x7E/0xFE), which is the
-    "satfinite" conversion; NaN becomes 0x7F. Below 2^-6 the grid is the
-    subnormal one, quantum 2^-9. All steps are exact in fp64 except the single
-    rounding to the grid (torch.round rounds half to even).
+    "satfinite" conversion; NaN becomes 0x7F. For |x| in [2^e, 2^(e+1)) with
+    e >= -6 the grid step is 2^(e-3); below 2^-6 it is the subnormal step 2^-9.
+    Each value is scaled by 1/step (a power of two: exact in fp32), rounded to an
+    integer half to even (the only rounding), and the code is assembled from
+    that integer and e.
     """
-    x = x.to(F32).to(F64)
-    sign = torch.signbit(x).to(torch.int64) << 7
+    x = x.to(F32)
+    sign = torch.signbit(x).to(torch.int32) << 7
     a = x.abs()
-    # exponent of the leading bit: a = f * 2^k, f in [0.5, 1)  ->  a in [2^(k-1), 2^k)
-    _, k = torch.frexp(torch.where(a > 0, a, torch.ones_like(a)))
-    e = (k - 1).to(torch.int64)
-    # normal numbers: quantum 2^(e-3); subnormals (a < 2^-6): quantum 2^-9
-    e_grid = torch.clamp(e, min=-6)
-    quantum = torch.pow(torch.tensor(2.0, dtype=F64), (e_grid - 3).to(F64))
-    n = torch.round(a / quantum).to(torch.int64)           # 0..16 (16 = carry into next binade)
+    # e = floor(log2(a)) read from the fp32 exponent field (subnormal fp32 inputs
+    # are far below the FP8 range and fall in the e < -6 branch either way)
+    e = ((a.view(torch.int32) >> 23) & 0xFF) - 127
+    e_grid = torch.clamp(e, min=-6, max=8)
+    inv_step = ((3 - e_grid + 127) << 23).view(F32)        # 2^(3 - e_grid), exact
+    n = torch.round(a * inv_step).to(torch.int32)          # 0..16 (16 = carry into next binade)
     carry = n == 16
     e_grid = torch.where(carry, e_grid + 1, e_grid)
     n = torch.where(carry, torch.full_like(n, 8), n)

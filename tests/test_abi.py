@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared entry
+point, sizes its buffers by the stated formulas and rejects bad arguments with a
+status code before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_block_scaled_biased_b200 import binding as B
+from fp8_block_scaled_biased_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return B.load_library()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "fp8moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", src, flags=re.M))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert names == set(B.EXPORTED)
+
+
+def test_capacity_and_workspace_formulas(lib):
+    assert lib.moe_align_sort_capacity(64, 8, 256, 128) == 64 * 8 + 256 * 127
+    assert lib.moe_align_sort_capacity(16, 4, 16, 1) == 64
+    cap = 64 * 8 + 256 * 127
+    need = lib.fused_moe_fp8_blockscale_g1u1_workspace(64, 8, 256, 7168, 2048, 128)
+    assert need >= cap * 2048 + 16 * cap * 4 + 64 * 8 * 7168 * 4
+    assert lib.fp8moe_moe_block_m() == 128
+
+
+def _rc(lib, name, *args):
+    return getattr(lib, name)(*args), lib.fp8moe_last_error().decode()
+
+
+# A non-null pointer that is never dereferenced: every call below fails validation
+# before any CUDA call, so nothing is launched (these tests must never reach a device).
+P = ctypes.c_void_p(16)
+
+
+def test_routing_rejects_bad_arguments(lib):
+    rc, msg = _rc(lib, "moe_biased_grouped_topk", P, 16, P, P, P, 3, 16, 16, 4, 4, 2, 1, 2.5, None)
+    assert rc == 1 and "ld_out" in msg                                    # strided outputs too narrow
+    rc, msg = _rc(lib, "moe_biased_grouped_topk", P, 16, P, P, P, 4, 16, 15, 4, 4, 2, 1, 2.5, None)
+    assert rc == 1                                                        # E % groups != 0
+    rc, _ = _rc(lib, "moe_biased_grouped_topk", P, 16, P, P, P, 4, 16, 16, 4, 4, 5, 1, 2.5, None)
+    assert rc == 1                                                        # topk_group > groups
+    rc, _ = _rc(lib, "moe_biased_grouped_topk", P, 16, P, P, P, 9, 16, 16, 9, 4, 2, 1, 2.5, None)
+    assert rc == 1                                                        # topk > candidates
+    rc, _ = _rc(lib, "moe_biased_grouped_topk", P, 1024, P, P, P, 8, 16, 1024, 8, 8, 4, 1, 2.5, None)
+    assert rc == 2                                                        # E above the kernel's limit
+    rc, _ = _rc(lib, "moe_biased_grouped_topk", P, 16, P, P, P, 4, 0, 16, 4, 4, 2, 1, 2.5, None)
+    assert rc == 0                                                        # T == 0: nothing to do
+
+
+def test_sort_rejects_bad_arguments(lib):
+    cap = lib.moe_align_sort_capacity(16, 4, 16, 4)
+    rc, msg = _rc(lib, "moe_align_sort", P, P, 4, 16, 4, 16, 4, P, P, P, P, cap - 1, None, 0, None)
+    assert rc == 1 and "capacity" in msg
+    rc, _ = _rc(lib, "moe_align_sort", P, P, 3, 16, 4, 16, 4, P, P, P, P, cap, None, 0, None)
+    assert rc == 1
+    rc, _ = _rc(lib, "moe_align_sort", P, P, 4, 16, 4, 2000, 4, P, P, P, P, 10 ** 6, None, 0, None)
+    assert rc == 2
+
+
+def test_quant_and_gemm_reject_bad_arguments(lib):
+    rc, _ = _rc(lib, "fp8_per_token_group_quant", P, 256, 4, 256, 64, P, P, 0, None)
+    assert rc == 2                                                        # group != 128
+    rc, _ = _rc(lib, "fp8_per_token_group_quant", P, 256, 4, 250, 128, P, P, 0, None)
+    assert rc == 2                                                        # K % 8 != 0
+    rc, _ = _rc(lib, "fp8_per_token_group_quant", P, 256, 4, 256, 128, P, P, 7, None)
+    assert rc == 1                                                        # unknown layout
+    rc, _ = _rc(lib, "fp8_per_block_quant", P, 256, 256, 256, 64, P, P, None)
+    assert rc == 2
+    rc, _ = _rc(lib, "fp8_blockscale_gemm", P, P, P, P, P, 64, 64, 64, 100, None)
+    assert rc == 2                                                        # K % 16 != 0
+    rc, _ = _rc(lib, "fp8_blockscale_gemm", P, P, P, P, P, 32, 64, 64, 128, None)
+    assert rc == 1                                                        # ldc < N
+    rc, _ = _rc(lib, "fp8_blockscale_gemm", None, P, P, P, P, 64, 64, 64, 128, None)
+    assert rc == 1
+
+
+def test_fused_moe_rejects_bad_arguments(lib):
+    T, K, E, H, I = 16, 4, 16, 256, 128
+    cap = lib.moe_align_sort_capacity(T, K, E, 128)
+    ws = lib.fused_moe_fp8_blockscale_g1u1_workspace(T, K, E, H, I, 128)
+    args = [P] * 8 + [T, H, I, E, K, 128, cap, P, P, P, 128, 128, None, ctypes.c_void_p(256), ws, None]
+
+    def call(**over):
+        a = list(args)
+        idx = {"scale_blk_n": 18, "scale_blk_k": 19, "smooth": 20, "ws_bytes": 22, "block_m": 13, "H": 9,
+               "cap": 14, "ws": 21}
+        for k, v in over.items():
+            a[idx[k]] = v
+        return _rc(lib, "fused_moe_fp8_blockscale_g1u1", *a)
+
+    assert call(scale_blk_n=64)[0] == 2
+    assert call(scale_blk_k=256)[0] == 2
+    assert call(smooth=P)[0] == 2
+    assert call(block_m=64)[0] == 2
+    assert call(H=200)[0] == 2
+    assert call(cap=cap - 1)[0] == 1
+    assert call(ws_bytes=ws - 1)[0] == 3
+    assert call(ws=None)[0] == 3
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = B._lib
+    B._lib = None
+    try:
+        with pytest.raises(RuntimeError):
+            B.load_library(str(tmp_path / "missing.so"))
+    finally:
+        B._lib = saved
