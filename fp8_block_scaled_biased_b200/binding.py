@@ -25,6 +25,8 @@ _SIGNATURES = {
     "fp8moe_last_error": (ctypes.c_char_p, []),
     "fp8moe_device_status": (_c_int, [_p]),
     "fp8moe_moe_block_m": (_c_int, []),
+    "fp8moe_timing_enable": (_c_int, [_c_int]),
+    "fp8moe_timing_last": (_c_int, [ctypes.POINTER(ctypes.c_float)]),
     "moe_biased_grouped_topk": (_c_int, [_p, _c_int, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                          _c_int, _c_float, _p]),
     "moe_align_sort_capacity": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
@@ -102,6 +104,18 @@ def device_status() -> int:
     if rc < 0:
         raise Fp8MoeError("fp8moe_device_status", rc, load_library().fp8moe_last_error().decode())
     return rc
+
+
+def timing_enable(on: bool = True):
+    """Record per-kernel events inside each fused MoE call (calling thread only)."""
+    _check("fp8moe_timing_enable", load_library().fp8moe_timing_enable(int(bool(on))))
+
+
+def timing_last():
+    """(gate/up GEMM ms, down GEMM ms, combine ms) of the most recent fused MoE call; waits for it."""
+    ms = (ctypes.c_float * 3)()
+    _check("fp8moe_timing_last", load_library().fp8moe_timing_last(ms))
+    return tuple(ms)
 
 
 def moe_block_m() -> int:

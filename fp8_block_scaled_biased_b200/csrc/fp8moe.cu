@@ -42,6 +42,24 @@ int check_launch(const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch check for the GEMM kernels: on failure the message carries the kernel's
+// resource attributes next to what the launch asked for.
+template <typename Kernel>
+int check_gemm_launch(const char* what, Kernel kernel, int threads, size_t smem) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    g_last_error.clear();
+    return FP8MOE_OK;
+  }
+  cudaFuncAttributes fa{};
+  cudaFuncGetAttributes(&fa, kernel);
+  return fail(FP8MOE_ECUDA,
+              "%s: launch failed: %s (kernel: %d regs, max %d threads, %zu B static smem, %d B max dynamic smem, "
+              "%zu B local; launch: %d threads, %zu B dynamic smem)",
+              what, cudaGetErrorString(e), fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+              fa.maxDynamicSharedSizeBytes, fa.localSizeBytes, threads, smem);
+}
+
 // ---------------------------------------------------------------- per-device state
 constexpr int kMaxDevices = 64;
 
@@ -140,6 +158,18 @@ MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I
   return w;
 }
 
+struct TimingState {
+  bool on = false;
+  int dev = -1;
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+};
+thread_local TimingState g_timing;
+
+void timing_record(int i, cudaStream_t st) {
+  // external record: inside a stream capture this becomes an event node of the graph
+  if (g_timing.on && g_timing.ev[i]) cudaEventRecordWithFlags(g_timing.ev[i], st, cudaEventRecordExternal);
+}
+
 int choose_group_m(int n_tiles) {
   // Visit a few consecutive row blocks per column tile so blocks of the same
   // expert share each weight tile while it is in L2.
@@ -153,6 +183,36 @@ extern "C" {
 const char* fp8moe_last_error(void) { return g_last_error.c_str(); }
 
 int fp8moe_moe_block_m(void) { return kBM; }
+
+int fp8moe_timing_enable(int on) {
+  if (!on) {
+    g_timing.on = false;
+    return FP8MOE_OK;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess && dev != g_timing.dev) {
+    for (auto& ev : g_timing.ev) {
+      if (ev) cudaEventDestroy(ev);
+      ev = nullptr;
+    }
+    for (auto& ev : g_timing.ev)
+      if (e == cudaSuccess) e = cudaEventCreate(&ev);
+    g_timing.dev = dev;
+  }
+  if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "timing events: %s", cudaGetErrorString(e));
+  g_timing.on = true;
+  return FP8MOE_OK;
+}
+
+int fp8moe_timing_last(float* ms) {
+  if (!ms) return fail(FP8MOE_EINVAL, "null pointer argument");
+  if (!g_timing.ev[3]) return fail(FP8MOE_EINVAL, "timing was never enabled");
+  cudaError_t e = cudaEventSynchronize(g_timing.ev[3]);
+  for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&ms[i], g_timing.ev[i], g_timing.ev[i + 1]);
+  if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "timing read: %s", cudaGetErrorString(e));
+  return FP8MOE_OK;
+}
 
 int fp8moe_device_status(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -303,7 +363,7 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   blockscale_gemm_kernel<kModeDense><<<grid, kGemmThreads, kGemmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       ma, mb, a);
-  return check_launch("fp8_blockscale_gemm");
+  return check_gemm_launch("fp8_blockscale_gemm", blockscale_gemm_kernel<kModeDense>, kGemmThreads, kGemmSmemBytes);
 }
 
 // ------------------------------------------------------------------ S4-S7 fused MoE
@@ -375,8 +435,12 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   up.b_rows_per_expert = 2 * I;
   up.a2 = a2;
   up.s2 = s2;
+  timing_record(0, st);
   blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8, m_w1, up);
-  if (int rc = check_launch("fused_moe (gate/up GEMM)")) return rc;
+  if (int rc = check_gemm_launch("fused_moe (gate/up GEMM)", blockscale_gemm_kernel<kModeMoeUp>, kGemmThreads,
+                                 kGemmSmemBytes))
+    return rc;
+  timing_record(1, st);
 
   GemmArgs dn = up;
   dn.N = H;
@@ -390,12 +454,17 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   dn.b_rows_per_expert = H;
   dn.ystage = ystage;
   blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
-  if (int rc = check_launch("fused_moe (down GEMM)")) return rc;
+  if (int rc = check_gemm_launch("fused_moe (down GEMM)", blockscale_gemm_kernel<kModeMoeDown>, kGemmThreads,
+                                 kGemmSmemBytes))
+    return rc;
+  timing_record(2, st);
 
   const size_t threads = static_cast<size_t>(T) * (H / 8);
   moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(ystage, T, topk, H,
                                                                                    reinterpret_cast<__nv_bfloat16*>(out));
-  return check_launch("fused_moe (combine)");
+  if (int rc = check_launch("fused_moe (combine)")) return rc;
+  timing_record(3, st);
+  return FP8MOE_OK;
 }
 
 }  // extern "C"

@@ -118,7 +118,7 @@ __device__ __forceinline__ void abort_all(GemmSmem* s) {
 }
 
 template <int MODE>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];

@@ -15,16 +15,23 @@ from . import inputs as I
 
 
 class MoELayer:
-    def __init__(self, cfg: I.MoEConfig, device="cuda", max_tokens: int | None = None):
+    def __init__(self, cfg: I.MoEConfig, device="cuda", max_tokens: int | None = None, weights_from=None):
+        """weights_from: another MoELayer of the same layer shape whose device weights are shared."""
         self.cfg = cfg
         self.device = torch.device(device)
         self.max_tokens = max_tokens or cfg.T
         E, H, Im = cfg.E, cfg.H, cfg.I
         dev = self.device
-        self.w1 = torch.empty(E, 2 * Im, H, dtype=B.FP8, device=dev)
-        self.w1_scale = torch.empty(E, 2 * Im // 128, H // 128, dtype=torch.float32, device=dev)
-        self.w2 = torch.empty(E, H, Im, dtype=B.FP8, device=dev)
-        self.w2_scale = torch.empty(E, H // 128, Im // 128, dtype=torch.float32, device=dev)
+        if weights_from is not None:
+            o = weights_from
+            if (o.cfg.E, o.cfg.H, o.cfg.I) != (E, H, Im):
+                raise ValueError("weights_from has a different layer shape")
+            self.w1, self.w1_scale, self.w2, self.w2_scale = o.w1, o.w1_scale, o.w2, o.w2_scale
+        else:
+            self.w1 = torch.empty(E, 2 * Im, H, dtype=B.FP8, device=dev)
+            self.w1_scale = torch.empty(E, 2 * Im // 128, H // 128, dtype=torch.float32, device=dev)
+            self.w2 = torch.empty(E, H, Im, dtype=B.FP8, device=dev)
+            self.w2_scale = torch.empty(E, H // 128, Im // 128, dtype=torch.float32, device=dev)
         self.block_m = B.moe_block_m()
         self._alloc(self.max_tokens)
 

@@ -61,6 +61,16 @@ const char* fp8moe_last_error(void);
  * synchronisation itself fails. */
 int fp8moe_device_status(void* stream);
 
+/* Measurement hook (not part of the pages' API). While enabled for the calling
+ * thread, each fused_moe_fp8_blockscale_g1u1 call records CUDA events on its
+ * stream before the gate/up GEMM, after it, after the down GEMM and after the
+ * combine. fp8moe_timing_last() waits for the last of those events and writes
+ * the three kernel durations of the most recent call in milliseconds
+ * (ms[0] gate/up GEMM, ms[1] down GEMM, ms[2] combine). Returns FP8MOE_OK or
+ * FP8MOE_ECUDA. Events are created on first use on the current device. */
+int fp8moe_timing_enable(int on);
+int fp8moe_timing_last(float* ms);
+
 /* Block size of the M (token-expert pair) dimension that the fused MoE kernels
  * tile by; moe_align_sort must be called with block_m equal to this. */
 int fp8moe_moe_block_m(void);

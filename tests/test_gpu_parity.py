@@ -1,0 +1,231 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against the oracle.
+
+Bit-exact for routing ids/weights, the sort, and FP8 codes and scales; the
+stated tolerance for the GEMM and the fused MoE output. Inputs come from the
+seeded generator; each side quantises raw numbers with its own code.
+"""
+import pytest
+import torch
+
+from oracle import fp8moe_oracle as O
+from fp8_block_scaled_biased_b200 import binding as B
+from fp8_block_scaled_biased_b200 import inputs as I
+from fp8_block_scaled_biased_b200.layer import MoELayer
+from tests.gpu_helpers import assert_moe_close, oracle_moe_rows
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device"),
+              pytest.mark.filterwarnings("ignore")]
+
+DEV = "cuda"
+MOE = [I.TINY, I.DECODE, I.PREFILL, I.SKEWED]
+
+
+def u8(t):
+    return t.view(torch.uint8).cpu() if t.dtype == B.FP8 else t.cpu()
+
+
+@pytest.fixture(autouse=True)
+def _device_status_clean():
+    yield
+    assert B.device_status() == 0
+
+
+# ---------------------------------------------------------------- FP8 conversion and sigmoid recipe
+def test_hardware_e4m3_conversion_matches_oracle_encoder():
+    g = torch.Generator().manual_seed(11)
+    vals = torch.cat([torch.randn(1 << 20, generator=g) * 40, torch.randn(1 << 18, generator=g) * 1e-2,
+                      (torch.rand(1 << 16, generator=g) - 0.5) * 2 ** -6,
+                      O.e4m3_decode(torch.arange(0, 0x7E, dtype=torch.int64)),        # grid points
+                      ]).float().clamp(-448, 448)
+    mids = O.e4m3_decode(torch.arange(0, 0x7E, dtype=torch.int64))
+    mids = ((mids[1:] + mids[:-1]) / 2).float()
+    vals = torch.cat([vals, mids, -mids])
+    n = (vals.numel() + 16383) // 16384 * 16384
+    w = torch.zeros(n, dtype=torch.float32)
+    w[: vals.numel()] = vals
+    w = w.view(-1, 128)
+    w[::128, 0] = 448.0            # every 128x128 block holds 448, so its scale is exactly 1
+    q, s = B.fp8_per_block_quant(w.to(DEV))
+    assert (s.cpu() == 1.0).all()
+    assert torch.equal(u8(q), O.e4m3_encode(w))
+
+
+def test_sigmoid_recipe_is_bit_identical():
+    # one group, all experts kept, no bias, no renorm: the weights are the sigmoid values
+    T, E = 1 << 15, 32
+    g = torch.Generator().manual_seed(12)
+    logits = torch.cat([torch.randn(T // 2, E, generator=g) * 4, (torch.rand(T // 2, E, generator=g) - 0.5) * 190])
+    bias = torch.zeros(E)
+    w = torch.empty(T, E, device=DEV)
+    ids = torch.empty(T, E, dtype=torch.int32, device=DEV)
+    B.moe_biased_grouped_topk(logits.to(DEV), bias.to(DEV), w, ids, 1, 1, False, 1.0)
+    w_ref, ids_ref = O.biased_grouped_topk(logits, bias, E, 1, 1, False, 1.0)
+    assert torch.equal(ids.cpu(), ids_ref)
+    assert torch.equal(w.cpu().view(torch.int32), w_ref.view(torch.int32))
+
+
+# ---------------------------------------------------------------- S1 routing
+@pytest.mark.parametrize("cfg", MOE, ids=lambda c: c.name)
+def test_routing_bit_exact_with_strided_outputs(cfg):
+    act = I.moe_activations(cfg)
+    ld = cfg.K + 10                                   # strided outputs, as the pages' test allocates them
+    wbuf = torch.full((cfg.T, ld), -7.0, device=DEV)
+    ibuf = torch.full((cfg.T, ld), -7, dtype=torch.int32, device=DEV)
+    w, ids = wbuf[:, : cfg.K], ibuf[:, : cfg.K]
+    B.moe_biased_grouped_topk(act.logits.to(DEV), act.bias.to(DEV), w, ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    w_ref, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    assert torch.equal(ids.cpu(), ids_ref)
+    assert torch.equal(w.cpu().view(torch.int32), w_ref.view(torch.int32))
+    assert (wbuf[:, cfg.K:] == -7.0).all() and (ibuf[:, cfg.K:] == -7).all()
+
+
+# ---------------------------------------------------------------- S2 align/sort
+@pytest.mark.parametrize("cfg,block_m", [(I.TINY, 4), (I.TINY, 128), (I.DECODE, 128), (I.DECODE, 16),
+                                         (I.PREFILL, 128), (I.PREFILL, 64), (I.SKEWED, 128)],
+                         ids=lambda v: getattr(v, "name", str(v)))
+def test_sort_bit_exact(cfg, block_m):
+    act = I.moe_activations(cfg)
+    w_ref, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    sp = B.alloc_sorted(cfg.T, cfg.K, cfg.E, block_m, DEV)
+    sp.sorted_ids.fill_(-5)
+    sp.sorted_weights.fill_(-5.0)
+    sp.sorted_expert_ids.fill_(-5)
+    B.moe_align_sort(ids_ref.to(DEV), w_ref.to(DEV), cfg.E, block_m, out=sp)
+    sid, sw, se, nv = O.align_sort(ids_ref, w_ref, cfg.E, block_m)
+    assert sp.num_valid_ids.item() == nv
+    assert torch.equal(sp.sorted_ids[:nv].cpu(), sid)
+    assert torch.equal(sp.sorted_weights[:nv].cpu().view(torch.int32), sw.view(torch.int32))
+    assert torch.equal(sp.sorted_expert_ids[: nv // block_m].cpu(), se)
+    assert (sp.sorted_ids[nv:] == -5).all() and (sp.sorted_expert_ids[nv // block_m:] == -5).all()
+
+
+def test_sort_empty_and_single_token():
+    for T in (0, 1):
+        ids = torch.arange(T * 4, dtype=torch.int32).view(T, 4) % 16
+        w = torch.ones(T, 4)
+        sp = B.moe_align_sort(ids.to(DEV), w.to(DEV), 16, 8)
+        sid, sw, se, nv = O.align_sort(ids, w, 16, 8)
+        assert sp.num_valid_ids.item() == nv
+        assert torch.equal(sp.sorted_ids[:nv].cpu(), sid)
+
+
+# ---------------------------------------------------------------- S3 quantisation
+@pytest.mark.parametrize("M,K", [(16, 256), (64, 7168), (2048, 7168), (37, 200), (5, 136), (1, 8)])
+@pytest.mark.parametrize("col_major", [False, True])
+def test_quant_1x128_bit_exact(M, K, col_major):
+    g = torch.Generator().manual_seed(M * 7 + K)
+    x = (torch.randn(M, K, generator=g) * torch.logspace(-4, 3, M)[:, None]).to(torch.bfloat16)
+    if M > 2:
+        x[1, : min(K, 128)] = 0                      # an all-zero group
+    q, s = B.fp8_per_token_group_quant(x.to(DEV), 128, column_major_scales=col_major)
+    q_ref, s_ref = O.quant_1x128(x)
+    assert torch.equal(u8(q), q_ref)
+    s_gpu = s.cpu().t() if col_major else s.cpu()
+    assert torch.equal(s_gpu.contiguous().view(torch.int32), s_ref.view(torch.int32))
+
+
+def test_quant_strided_rows():
+    x = torch.randn(40, 512).to(torch.bfloat16)
+    q, s = B.fp8_per_token_group_quant(x.to(DEV)[:, :384], 128)
+    q_ref, s_ref = O.quant_1x128(x[:, :384])
+    assert torch.equal(u8(q), q_ref) and torch.equal(s.cpu(), s_ref)
+
+
+@pytest.mark.parametrize("which", ["random_300x260", "w1_4096x7168", "w2_7168x2048"])
+def test_quant_128x128_bit_exact(which):
+    if which.startswith("random"):
+        w = (torch.randn(300, 260, generator=torch.Generator().manual_seed(3)) * 0.02).to(DEV)
+    else:
+        w = I.expert_weight_raw(I.DECODE, which[:2], 7, DEV)
+    q, s = B.fp8_per_block_quant(w)
+    q_ref, s_ref = O.quant_128x128(w.cpu())
+    assert torch.equal(u8(q), q_ref)
+    assert torch.equal(s.cpu().view(torch.int32), s_ref.view(torch.int32))
+
+
+# ---------------------------------------------------------------- S0 block-scale GEMM
+def _gemm_case(M, N, K, seed, sample_rows=None):
+    g = torch.Generator().manual_seed(seed)
+    a = (torch.randn(M, K, generator=g)).to(torch.bfloat16)
+    b = torch.randn(N, K, generator=g) * 0.02
+    qa, sa = B.fp8_per_token_group_quant(a.to(DEV), 128)
+    qb, sb = B.fp8_per_block_quant(b.to(DEV))
+    c = B.fp8_blockscale_gemm(qa, qb, sa, sb)
+    rows = torch.arange(M) if sample_rows is None else sample_rows
+    qa_ref, sa_ref = O.quant_1x128(a[rows])
+    qb_ref, sb_ref = O.quant_128x128(b)
+    ref = O.blockscale_gemm(qa_ref, sa_ref, qb_ref, sb_ref)
+    got = c.cpu()[rows].double()
+    return got, ref
+
+
+def _assert_gemm_close(got, ref):
+    d = (got - ref).abs()
+    # bf16 output rounding (2^-9 relative) plus fp32 accumulation
+    assert (d <= ref.abs() * 2.0 ** -8 + 1e-5 * ref.abs().max()).all(), d.max()
+    assert d.max() <= 2e-2 * ref.abs().max() + 1e-3
+    assert d.sum() / ref.abs().sum() <= 5e-3
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (200, 300, 400), (1, 8, 16), (257, 1000, 1024), (130, 520, 272)])
+def test_gemm_small_and_ragged(M, N, K):
+    got, ref = _gemm_case(M, N, K, seed=M + N + K)
+    _assert_gemm_close(got, ref)
+
+
+def test_gemm_2048x4096x7168_sampled_rows():
+    rows = torch.cat([torch.arange(0, 2048, 61), torch.tensor([127, 128, 2047])])
+    got, ref = _gemm_case(2048, 4096, 7168, seed=0, sample_rows=rows)
+    _assert_gemm_close(got, ref)
+
+
+def test_gemm_is_deterministic():
+    g = torch.Generator().manual_seed(5)
+    a = torch.randn(512, 1024, generator=g).to(torch.bfloat16).to(DEV)
+    b = (torch.randn(768, 1024, generator=g) * 0.02).to(DEV)
+    qa, sa = B.fp8_per_token_group_quant(a, 128)
+    qb, sb = B.fp8_per_block_quant(b)
+    c1 = B.fp8_blockscale_gemm(qa, qb, sa, sb).clone()
+    c2 = B.fp8_blockscale_gemm(qa, qb, sa, sb)
+    assert torch.equal(c1, c2)
+
+
+# ---------------------------------------------------------------- S4-S7 fused MoE
+MID = I.MoEConfig("mid_t256_h1024_e32", T=256, H=1024, E=32, G=4, TG=2, K=4, I=512, seed=1)
+SKEW_SMALL = I.MoEConfig("skew_t512_h512_e64", T=512, H=512, E=64, G=8, TG=4, K=8, I=256, hot_experts=4, seed=2)
+
+
+@pytest.mark.parametrize("cfg", [I.TINY, MID, SKEW_SMALL], ids=lambda c: c.name)
+def test_fused_moe_full_small_layers(cfg):
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    act = I.moe_activations(cfg)
+    out = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV)).clone()
+    ref, w_ref, ids_ref = oracle_moe_rows(cfg, act, None)
+    assert torch.equal(layer.topk_ids.cpu(), ids_ref)
+    assert_moe_close(out, ref)
+    out2 = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    assert torch.equal(out, out2)                      # deterministic combine
+
+
+@pytest.fixture(scope="module")
+def big_layer():
+    layer = MoELayer(I.DECODE, DEV).load_synthetic_weights()
+    yield layer
+    del layer
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg,n_sample", [(I.DECODE, 6), (I.PREFILL, 4), (I.SKEWED, 8)], ids=lambda v: getattr(v, "name", str(v)))
+def test_fused_moe_full_size_sampled_tokens(big_layer, cfg, n_sample):
+    layer = MoELayer(cfg, DEV, weights_from=big_layer)
+    act = I.moe_activations(cfg)
+    out = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV)).clone()
+    g = torch.Generator().manual_seed(99)
+    tokens = torch.sort(torch.cat([torch.randperm(cfg.T, generator=g)[: n_sample - 1],
+                                   torch.tensor([cfg.T - 1])]).unique()).values
+    ref, w_ref, ids_ref = oracle_moe_rows(cfg, act, tokens)
+    assert torch.equal(layer.topk_ids.cpu(), ids_ref)
+    assert_moe_close(out.cpu()[tokens], ref)
+    out2 = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    assert torch.equal(out, out2)
