@@ -125,36 +125,63 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major byte matrix [rows, cols] (row stride `ld` bytes), box
-// {128 bytes, box_rows}, 128-byte swizzle, zero fill outside the matrix.
-int make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+// 2-D map over a row-major matrix [rows, cols] of `elem_bytes`-byte elements
+// (row stride `ld_bytes`), box {box_cols, box_rows}, zero fill outside the matrix.
+int make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t rows,
+                uint64_t cols, uint64_t ld_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FP8MOE_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  (void)elem_bytes;
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {ld};
-  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint64_t strides[1] = {ld_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(FP8MOE_ECUDA, "cuTensorMapEncodeTiled failed (%d) for [%llu x %llu]", static_cast<int>(r),
                 static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols));
   return FP8MOE_OK;
 }
 
+// Operand tile map: FP8 bytes, box {128 bytes of K, 128 rows}, 128-byte swizzle.
+int make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, cols, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Epilogue store map: boxes of 32 rows x 64 bytes, 64-byte swizzle (the staging layout).
+int make_store_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t rows,
+                   uint64_t cols, uint64_t ld_bytes) {
+  return make_map_2d(map, dtype, elem_bytes, base, rows, cols, ld_bytes, 64 / elem_bytes, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Scratch of the fused MoE call, all slot-ordered (capacity rows): the gathered
+// FP8 activations and their scales, pair -> slot, the re-quantised intermediate
+// and its scales, and the weighted down-projection rows.
 struct MoeWorkspace {
-  size_t a2_off, s2_off, y_off, total;
+  size_t a8s_off, s1s_off, inv_off, a2_off, s2_off, y_off, total;
 };
 
 MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I) {
   MoeWorkspace w;
-  w.a2_off = 0;
-  w.s2_off = round_up(w.a2_off + capacity * static_cast<size_t>(I), 256);
-  w.y_off = round_up(w.s2_off + static_cast<size_t>(I / 128) * capacity * sizeof(float), 256);
-  w.total = round_up(w.y_off + static_cast<size_t>(T) * topk * H * sizeof(float), 256);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = round_up(off + bytes, 256);
+    return at;
+  };
+  w.a8s_off = take(capacity * static_cast<size_t>(H));
+  w.s1s_off = take(static_cast<size_t>(H / 128) * capacity * sizeof(float));
+  w.inv_off = take(static_cast<size_t>(T) * topk * sizeof(int32_t));
+  w.a2_off = take(capacity * static_cast<size_t>(I));
+  w.s2_off = take(static_cast<size_t>(I / 128) * capacity * sizeof(float));
+  w.y_off = take(capacity * static_cast<size_t>(H) * sizeof(float));
+  w.total = off;
   return w;
 }
 
@@ -342,9 +369,16 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   if (!aligned16(A) || !aligned16(B)) return fail(FP8MOE_EINVAL, "A and B must be 16-byte aligned");
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
-  CUtensorMap ma, mb;
-  if (int rc = make_map_u8(&ma, A, M, K, K, 128)) return rc;
-  if (int rc = make_map_u8(&mb, B, N, K, K, 128)) return rc;
+  CUtensorMap ma, mb, mc;
+  if (int rc = make_operand_map(&ma, A, M, K)) return rc;
+  if (int rc = make_operand_map(&mb, B, N, K)) return rc;
+  const bool c_tma = (ldc % 8 == 0) && aligned16(C);
+  if (c_tma) {
+    if (int rc = make_store_map(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, M, N, static_cast<uint64_t>(ldc) * 2))
+      return rc;
+  } else {
+    mc = ma;   // unused: the kernel stores C directly
+  }
   GemmArgs a{};
   a.M = M;
   a.N = N;
@@ -357,12 +391,12 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   a.nb_valid = a.nb_per_expert;
   a.C = reinterpret_cast<__nv_bfloat16*>(C);
   a.ldc = ldc;
-  a.c_vec_ok = (ldc % 8 == 0) && aligned16(C);
+  a.c_tma = c_tma ? 1 : 0;
   a.b_rows_per_expert = 0;
   const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * a.n_tiles;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   blockscale_gemm_kernel<kModeDense><<<grid, kGemmThreads, kGemmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      ma, mb, a);
+      ma, mb, mc, a);
   return check_gemm_launch("fp8_blockscale_gemm", blockscale_gemm_kernel<kModeDense>, kGemmThreads, kGemmSmemBytes);
 }
 
@@ -404,16 +438,28 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* a8s = ws + lay.a8s_off;
+  float* s1s = reinterpret_cast<float*>(ws + lay.s1s_off);
+  int32_t* slot_of_pair = reinterpret_cast<int32_t*>(ws + lay.inv_off);
   uint8_t* a2 = ws + lay.a2_off;
   float* s2 = reinterpret_cast<float*>(ws + lay.s2_off);
   float* ystage = reinterpret_cast<float*>(ws + lay.y_off);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  CUtensorMap m_a8, m_w1, m_a2, m_w2;
-  if (int rc = make_map_u8(&m_a8, a8, T, H, H, 1)) return rc;
-  if (int rc = make_map_u8(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H, H, 128)) return rc;
-  if (int rc = make_map_u8(&m_a2, a2, capacity, I, I, 128)) return rc;
-  if (int rc = make_map_u8(&m_w2, w2, static_cast<uint64_t>(E) * H, I, I, 128)) return rc;
+  CUtensorMap m_a8s, m_w1, m_a2_ld, m_a2_st, m_w2, m_y;
+  if (int rc = make_operand_map(&m_a8s, a8s, capacity, H)) return rc;
+  if (int rc = make_operand_map(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H)) return rc;
+  if (int rc = make_operand_map(&m_a2_ld, a2, capacity, I)) return rc;
+  if (int rc = make_operand_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
+  if (int rc = make_store_map(&m_a2_st, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a2, capacity, I, I)) return rc;
+  if (int rc = make_store_map(&m_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ystage, capacity, H,
+                              static_cast<uint64_t>(H) * 4))
+    return rc;
+
+  timing_record(0, st);
+  moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, num_valid_ids, T, topk, H,
+                                                            static_cast<int>(capacity), a8s, s1s, slot_of_pair);
+  if (int rc = check_launch("fused_moe (gather)")) return rc;
 
   GemmArgs up{};
   up.M = static_cast<int>(capacity);
@@ -421,7 +467,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   up.num_kb = H / 128;
   up.n_tiles = I / 128;
   up.group_m = choose_group_m(up.n_tiles);
-  up.a_scale = a1_scale;
+  up.a_scale = s1s;
   up.b_scale = fc1_scale;
   up.nb_per_expert = 2 * I / 128;
   up.nb_valid = up.nb_per_expert;
@@ -433,10 +479,8 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   up.topk = topk;
   up.E = E;
   up.b_rows_per_expert = 2 * I;
-  up.a2 = a2;
   up.s2 = s2;
-  timing_record(0, st);
-  blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8, m_w1, up);
+  blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, m_a2_st, up);
   if (int rc = check_gemm_launch("fused_moe (gate/up GEMM)", blockscale_gemm_kernel<kModeMoeUp>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
@@ -452,16 +496,16 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   dn.nb_per_expert = H / 128;
   dn.nb_valid = H / 128;
   dn.b_rows_per_expert = H;
-  dn.ystage = ystage;
-  blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
+  dn.s2 = nullptr;
+  blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2_ld, m_w2, m_y, dn);
   if (int rc = check_gemm_launch("fused_moe (down GEMM)", blockscale_gemm_kernel<kModeMoeDown>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
   timing_record(2, st);
 
   const size_t threads = static_cast<size_t>(T) * (H / 8);
-  moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(ystage, T, topk, H,
-                                                                                   reinterpret_cast<__nv_bfloat16*>(out));
+  moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
+      ystage, slot_of_pair, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
   if (int rc = check_launch("fused_moe (combine)")) return rc;
   timing_record(3, st);
   return FP8MOE_OK;

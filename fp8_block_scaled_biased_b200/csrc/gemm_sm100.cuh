@@ -8,16 +8,24 @@
 //     GEMM2 over w2, weighted by the routing weights.
 //
 // One kernel, three epilogues (Mode). Tile: 128 rows x 256 MMA columns x 128 K
-// per pipeline stage (one scale block). Warp roles in a persistent CTA:
-//   warp 0      producer: TMA loads of A (tiled, or gathered rows via
-//               tile::gather4) and B into a 4-stage shared-memory ring, plus
-//               the stage's scales into a separate 8-slot ring (cp.async);
+// per pipeline stage (one scale block). Warp roles in a persistent CTA of three
+// warpgroups; warpgroup 0 gives registers to the two epilogue warpgroups
+// (setmaxnreg: 56 / 224 / 224 per thread, the launch's 3 x 168 in total):
+//   warp 0      producer: TMA loads of the A and B tiles into a 4-stage
+//               shared-memory ring;
 //   warp 1      MMA issuer: per K block, 4 x tcgen05.mma (K=32 each) into one
 //               of two 256-column TMEM buffers, fresh (not accumulated) so the
 //               buffer holds that block's partial sums;
-//   warps 2..9  epilogue: tcgen05.ld the partials, multiply by
+//   warp 2      scale loader: each K block's row and column scales into an
+//               8-slot ring (cp.async); warp 3 idles;
+//   warps 4..11 epilogue: tcgen05.ld the partials, multiply by
 //               a_scale[row, kb] * b_scale[col/128, kb] and add into fp32
-//               registers (the per-128-K promotion), then the mode's output.
+//               registers (the per-128-K promotion), then the mode's output,
+//               staged through a 64-byte-swizzled shared buffer per warp and
+//               written with TMA bulk stores.
+// In the MoE modes the rows are the sorted token-expert slots: A is the
+// slot-ordered activation matrix (gathered by moe_gather_kernel for GEMM1, the
+// re-quantised intermediate for GEMM2), one expert per 128-row block.
 // All waits are bounded; on expiry the CTA flags FP8MOE_DEVERR_TIMEOUT, sets a
 // shared abort flag so the other roles stop, frees TMEM and exits.
 #pragma once
@@ -30,16 +38,19 @@ namespace fp8moe {
 
 enum GemmMode : int { kModeDense = 0, kModeMoeUp = 1, kModeMoeDown = 2 };
 
-constexpr int kBM = 128;                      // rows (tokens / token-expert pairs) per tile
+constexpr int kBM = 128;                      // rows (tokens / token-expert slots) per tile
 constexpr int kBN = 256;                      // MMA columns per tile
 constexpr int kBK = 128;                      // K per stage = one scale block
 constexpr int kUmmaK = 32;                    // K of one tcgen05.mma kind::f8f6f4
 constexpr int kStages = 4;
 constexpr int kScaleSlots = 8;
 constexpr int kEpiWarps = 8;
-constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kGemmThreads = 128 + 32 * kEpiWarps;   // warpgroup 0 + two epilogue warpgroups
+constexpr uint32_t kRegsWg0 = 56;                     // producer / MMA / scale-loader warpgroup
+constexpr uint32_t kRegsEpilogue = 224;               // 56 + 2 x 224 == 3 x 168 (launch budget)
 constexpr int kStageA = kBM * kBK;            // bytes
 constexpr int kStageB = kBN * kBK;
+constexpr int kStagingBytes = 32 * 64;        // per epilogue warp: 32 rows x 64 bytes
 constexpr uint32_t kTmemCols = 512;           // two 256-column partial buffers
 constexpr uint32_t kIdesc = umma_idesc_e4m3_f32(kBM, kBN);
 
@@ -49,22 +60,20 @@ struct GemmArgs {
   int num_kb;             // ceil(K / 128)
   int n_tiles;            // tiles along N
   int group_m;            // M blocks visited together for each N tile (L2 reuse)
-  const float* a_scale;   // dense: [M, num_kb]; up: a1_scale [H/128, T]; down: s2 [I/128, M]
+  const float* a_scale;   // dense: [M, num_kb]; MoE: slot-ordered [num_kb, M]
   const float* b_scale;   // [E][nb_per_expert][num_kb] (dense: E = 1)
   int nb_per_expert;      // 128-row scale blocks per expert matrix
   int nb_valid;           // dense: ceil(N/128) (clamp for the last tile)
-  __nv_bfloat16* C;       // dense output
+  int c_tma;              // dense: C can be written by TMA (else direct stores)
+  __nv_bfloat16* C;       // dense output (direct-store path)
   int ldc;
-  int c_vec_ok;           // dense: 16-byte stores allowed
   const int32_t* sorted_ids;
   const int32_t* sorted_expert_ids;
   const int32_t* num_valid_ids;
   const float* sorted_weights;
   int T, topk, E;
   int b_rows_per_expert;  // up: 2I; down: H
-  uint8_t* a2;            // up output [M, I]
   float* s2;              // up output [I/128, M]
-  float* ystage;          // down output [T*topk, N]
 };
 
 struct GemmSmem {
@@ -82,7 +91,8 @@ struct GemmSmem {
   float amax_x[2][2][kBM];
 };
 
-constexpr size_t kGemmSmemBytes = 1024 /*alignment slack*/ + kStages * (kStageA + kStageB) + sizeof(GemmSmem);
+constexpr size_t kGemmSmemBytes =
+    1024 /*alignment slack*/ + kStages * (kStageA + kStageB) + kEpiWarps * kStagingBytes + sizeof(GemmSmem);
 
 __device__ __forceinline__ void tile_coords(int tile, int m_blocks, int n_tiles, int group_m, int& mb, int& nt) {
   const int per_group = n_tiles * group_m;
@@ -117,172 +127,40 @@ __device__ __forceinline__ void abort_all(GemmSmem* s) {
   s->abort = 1;
 }
 
+// Writes 64 bytes of row `lane` into the warp's 32 x 64 B staging buffer in the
+// 64-byte-swizzled order a SWIZZLE_64B tensor map reads (16-byte chunk c of row
+// r lives at chunk c ^ ((r >> 1) & 3)), then stores the box with TMA.
+__device__ __forceinline__ void stage_and_store(uint8_t* staging, int lane, const uint4 (&d)[4],
+                                                const CUtensorMap* map, int x, int y, bool any_valid) {
+  if (lane == 0) bulk_wait_read_all();   // previous store from this buffer has read it
+  __syncwarp();
+  uint8_t* row = staging + lane * 64;
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) = d[c];
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && any_valid) {
+    tma_store_2d(map, staging, x, y);
+    bulk_commit();
+  }
+}
+
+// The epilogue warpgroups: promotion of each K block's partial sums into fp32
+// registers, then the mode's output through the per-warp staging buffer.
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const GemmArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* tiles = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint8_t* tiles_a = tiles;                                  // kStages x 16 KB
-  uint8_t* tiles_b = tiles + kStages * kStageA;              // kStages x 32 KB
-  GemmSmem* s = reinterpret_cast<GemmSmem*>(tiles + kStages * (kStageA + kStageB));
+__device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s, uint8_t* staging,
+                                              const CUtensorMap* tmC_ptr, uint32_t tmem_base, int warp, int lane,
+                                              int m_blocks, int total_tiles, int num_kb, int P) {
   volatile int* abort_flag = &s->abort;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (warp == 0 && lane == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s->full[i], 1);
-      mbar_init(&s->empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s->tfull[i], 1);
-      mbar_init(&s->tempty[i], kEpiWarps);
-      mbar_init(&s->xbar[i], kEpiWarps);
-    }
-    for (int i = 0; i < kScaleSlots; ++i) {
-      mbar_init(&s->sfull[i], 32);
-      mbar_init(&s->sempty[i], kEpiWarps);
-    }
-    s->abort = 0;
-    fence_mbar_init();
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(&s->tmem_base, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = s->tmem_base;
-
-  const int m_blocks = (MODE == kModeDense) ? (args.M + kBM - 1) / kBM : moe_m_blocks(args);
-  const int total_tiles = m_blocks * args.n_tiles;
-  const int num_kb = args.num_kb;
-  const int P = args.T * args.topk;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int stage = 0, sslot = 0;
-    uint32_t sphase = 0, scphase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      int mb, nt;
-      tile_coords(tile, m_blocks, args.n_tiles, args.group_m, mb, nt);
-      const int e = (MODE == kModeDense) ? 0 : moe_expert(args, mb);
-      // this lane's four rows of the tile: 4*lane .. 4*lane+3
-      int tok[4];
-      const float* sa_src[4];
-      if (MODE == kModeMoeUp) {
-        const int4 sid4 = *reinterpret_cast<const int4*>(args.sorted_ids + mb * kBM + 4 * lane);
-        const int sid[4] = {sid4.x, sid4.y, sid4.z, sid4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int t = 0;                                         // padding slots read token 0 (discarded)
-          if (sid[i] >= 0 && sid[i] < P)
-            t = sid[i] / args.topk;
-          else if (sid[i] != P)
-            raise_device_error(FP8MOE_DEVERR_PAIR_ID);
-          tok[i] = t;
-          sa_src[i] = args.a_scale + t;                      // + kb * T
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = mb * kBM + 4 * lane + i;
-          tok[i] = r;
-          sa_src[i] = (MODE == kModeDense) ? args.a_scale + static_cast<size_t>(min(r, args.M - 1)) * num_kb
-                                           : args.a_scale + r;   // + kb * M
-        }
-      }
-      int nb0, nb1, brow0, brow1;
-      if (MODE == kModeMoeUp) {
-        nb0 = nt;
-        nb1 = args.N / 128 + nt;
-        brow0 = e * args.b_rows_per_expert + nt * 128;
-        brow1 = brow0 + args.N;
-      } else {
-        nb0 = min(2 * nt, args.nb_valid - 1);
-        nb1 = min(2 * nt + 1, args.nb_valid - 1);
-        brow0 = e * args.b_rows_per_expert + nt * kBN;
-        brow1 = brow0 + 128;
-      }
-      const float* sw_src0 = args.b_scale + (static_cast<size_t>(e) * args.nb_per_expert + nb0) * num_kb;
-      const float* sw_src1 = args.b_scale + (static_cast<size_t>(e) * args.nb_per_expert + nb1) * num_kb;
-
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&s->empty[stage], sphase ^ 1u, abort_flag)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(&s->full[stage], kStageA + kStageB);
-        __syncwarp();
-        uint8_t* sa_tile = tiles_a + stage * kStageA;
-        uint8_t* sb_tile = tiles_b + stage * kStageB;
-        if (MODE == kModeMoeUp) {
-          tma_gather4(sa_tile + lane * 512, &tmA, &s->full[stage], kb * kBK, tok[0], tok[1], tok[2], tok[3]);
-        } else if (lane == 0) {
-          tma_load_2d(sa_tile, &tmA, &s->full[stage], kb * kBK, mb * kBM);
-        }
-        if (lane == 0) {
-          tma_load_2d(sb_tile, &tmB, &s->full[stage], kb * kBK, brow0);
-          tma_load_2d(sb_tile + kStageB / 2, &tmB, &s->full[stage], kb * kBK, brow1);
-        }
-        // scales of this K block
-        if (!mbar_wait(&s->sempty[sslot], scphase ^ 1u, abort_flag)) { ok = false; break; }
-        const size_t kstride = (MODE == kModeDense) ? 1 : (MODE == kModeMoeUp ? args.T : args.M);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) cp_async_4(&s->sa[sslot][4 * lane + i], sa_src[i] + kb * kstride);
-        if (lane == 0) {
-          cp_async_4(&s->sw[sslot][0], sw_src0 + kb);
-          cp_async_4(&s->sw[sslot][1], sw_src1 + kb);
-        }
-        cp_async_mbar_arrive(&s->sfull[sslot]);
-        if (++stage == kStages) { stage = 0; sphase ^= 1u; }
-        if (++sslot == kScaleSlots) { sslot = 0; scphase ^= 1u; }
-      }
-      if (!ok) break;
-    }
-    if (!ok) {
-      abort_all(s);
-      // let copies already in flight land before the CTA's shared memory goes away
-      const unsigned long long t0 = global_timer_ns();
-      while (global_timer_ns() - t0 < 10000000ull) {}
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0, buf = 0;
-      uint32_t sphase = 0, tphase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&s->full[stage], sphase, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&s->tempty[buf], tphase ^ 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles_a + stage * kStageA);
-          const uint32_t b_addr = smem_u32(tiles_b + stage * kStageB);
-          const uint32_t d_tmem = tmem_base + buf * kBN;
-#pragma unroll
-          for (int k = 0; k < kBK / kUmmaK; ++k)
-            umma_f8(d_tmem, umma_desc_sw128(a_addr + k * kUmmaK), umma_desc_sw128(b_addr + k * kUmmaK), kIdesc,
-                    k > 0 ? 1u : 0u);
-          umma_commit(&s->empty[stage]);
-          umma_commit(&s->tfull[buf]);
-          if (++stage == kStages) { stage = 0; sphase ^= 1u; }
-          if (++buf == 2) { buf = 0; tphase ^= 1u; }
-        }
-      }
-      if (!ok) abort_all(s);
-    }
-    __syncwarp();
-  } else {
+  const CUtensorMap& tmC = *tmC_ptr;
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
+    const int ew = warp - 4;
     const int half = ew >> 2;                  // which 128 of the 256 MMA columns (up: which 64 of I)
     const int quarter = warp & 3;              // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;       // tile row = TMEM lane
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint8_t* my_staging = staging + ew * kStagingBytes;
     // TMEM columns of this thread's two 64-column segments
     const int col0 = (MODE == kModeMoeUp) ? half * 64 : half * 128;
     const int col1 = (MODE == kModeMoeUp) ? kBN / 2 + half * 64 : half * 128 + 64;
@@ -295,9 +173,9 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const int slot = mb * kBM + row;
       int pair = 0;
       float wroute = 0.0f;
-      if (MODE == kModeMoeDown) {               // needed only at the end: load early
+      if (MODE != kModeDense) {                 // needed only at the end: load early
         pair = args.sorted_ids[slot];
-        wroute = args.sorted_weights[slot];
+        if (MODE == kModeMoeDown) wroute = args.sorted_weights[slot];
       }
       float acc[128];
 #pragma unroll
@@ -321,15 +199,21 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         if (!mbar_wait(&s->tfull[buf], tphase, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tb = lane_base + buf * kBN;
+        // four 32-column chunks; the load of chunk c+1 overlaps the FMAs of chunk c
+        float v[2][32];
+        tmem_ld_32x32b_x32(tb + col0, v[0]);
+        tmem_wait_ld();
+        reg_fence_32(v[0]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float v[32];
-          const int col = (c < 2 ? col0 : col1) + (c & 1) * 32;
-          tmem_ld_32x32b_x32(tb + col, v);
-          tmem_wait_ld();
+          if (c + 1 < 4) tmem_ld_32x32b_x32(tb + ((c + 1) < 2 ? col0 : col1) + ((c + 1) & 1) * 32, v[(c + 1) & 1]);
           const float f = (c < 2) ? f0 : f1;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(f, v[j], acc[c * 32 + j]);
+          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(f, v[c & 1][j], acc[c * 32 + j]);
+          if (c + 1 < 4) {
+            tmem_wait_ld();
+            reg_fence_32(v[(c + 1) & 1]);
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -338,28 +222,29 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       }
       if (!ok) break;
 
+      const int y0 = mb * kBM + quarter * 32;   // first row of this warp's 32-row slice
       if (MODE == kModeDense) {
         const int grow = mb * kBM + row;
-        if (grow < args.M) {
+        if (args.c_tma) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
+            const int x = nt * kBN + half * 128 + ch * 32;
+            const bool any = y0 < args.M && x < args.N;
+            uint4 d[4];
+            uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const __nv_bfloat162 p = __floats2bfloat162_rn(acc[ch * 32 + 2 * u], acc[ch * 32 + 2 * u + 1]);
+              w32[u] = *reinterpret_cast<const uint32_t*>(&p);
+            }
+            stage_and_store(my_staging, lane, d, &tmC, x, y0, any);
+          }
+        } else if (grow < args.M) {
           __nv_bfloat16* crow = args.C + static_cast<size_t>(grow) * args.ldc;
 #pragma unroll
-          for (int sgm = 0; sgm < 2; ++sgm) {
-            const int cbase = nt * kBN + half * 128 + sgm * 64;
-#pragma unroll
-            for (int j = 0; j < 64; j += 8) {
-              const int col = cbase + j;
-              if (args.c_vec_ok && col + 8 <= args.N) {
-                __align__(16) __nv_bfloat162 pk[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  pk[u] = __floats2bfloat162_rn(acc[sgm * 64 + j + 2 * u], acc[sgm * 64 + j + 2 * u + 1]);
-                *reinterpret_cast<uint4*>(crow + col) = *reinterpret_cast<const uint4*>(pk);
-              } else {
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                  if (col + u < args.N) crow[col + u] = __float2bfloat16_rn(acc[sgm * 64 + j + u]);
-              }
-            }
+          for (int j = 0; j < 128; ++j) {
+            const int col = nt * kBN + half * 128 + j;
+            if (col < args.N) crow[col] = __float2bfloat16_rn(acc[j]);
           }
         }
       } else if (MODE == kModeMoeUp) {
@@ -380,40 +265,199 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         if (!mbar_wait(&s->xbar[xb], (tcount >> 1) & 1, abort_flag)) { ok = false; break; }
         amax = fmaxf(amax, s->amax_x[xb][half ^ 1][row]);
         const float scale = __fdiv_rn(amax, 448.0f);
-        uint8_t* dst = args.a2 + static_cast<size_t>(slot) * args.N + nt * 128 + half * 64;
+        uint4 d[4];
+        uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
 #pragma unroll
-        for (int j = 0; j < 64; j += 16) {
-          uint4 pk;
-          uint32_t* w32 = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (scale != 0.0f) {
-              w32[u] = static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(acc[j + 4 * u], scale),
-                                                        __fdiv_rn(acc[j + 4 * u + 1], scale))) |
-                       (static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(acc[j + 4 * u + 2], scale),
-                                                         __fdiv_rn(acc[j + 4 * u + 3], scale)))
-                        << 16);
-            } else {
-              w32[u] = 0u;
-            }
-          }
-          *reinterpret_cast<uint4*>(dst + j) = pk;
+        for (int u = 0; u < 16; ++u) {
+          w32[u] = 0u;
+          if (scale != 0.0f)
+            w32[u] = static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(acc[4 * u], scale),
+                                                      __fdiv_rn(acc[4 * u + 1], scale))) |
+                     (static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(acc[4 * u + 2], scale),
+                                                       __fdiv_rn(acc[4 * u + 3], scale)))
+                      << 16);
         }
+        const bool any = __any_sync(0xffffffffu, pair >= 0 && pair < P);
+        stage_and_store(my_staging, lane, d, &tmC, nt * 128 + half * 64, y0, any);
         if (half == 0) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
       } else {
-        const int col = nt * kBN + half * 128;
-        if (pair >= 0 && pair < P && col < args.N) {
-          float* dst = args.ystage + static_cast<size_t>(pair) * args.N + col;
+        const bool valid = pair >= 0 && pair < P;
+        if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
+        const bool any = __any_sync(0xffffffffu, valid) && (nt * kBN + half * 128 < args.N);
 #pragma unroll
-          for (int j = 0; j < 128; j += 4)
-            *reinterpret_cast<float4*>(dst + j) =
-                make_float4(wroute * acc[j], wroute * acc[j + 1], wroute * acc[j + 2], wroute * acc[j + 3]);
-        } else if (pair != P && (pair < 0 || pair > P)) {
-          raise_device_error(FP8MOE_DEVERR_PAIR_ID);
+        for (int ch = 0; ch < 8; ++ch) {        // 8 chunks of 16 fp32 columns
+          uint4 d[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            d[u] = make_uint4(__float_as_uint(wroute * acc[ch * 16 + 4 * u]),
+                              __float_as_uint(wroute * acc[ch * 16 + 4 * u + 1]),
+                              __float_as_uint(wroute * acc[ch * 16 + 4 * u + 2]),
+                              __float_as_uint(wroute * acc[ch * 16 + 4 * u + 3]));
+          stage_and_store(my_staging, lane, d, &tmC, nt * kBN + half * 128 + ch * 16, y0, any);
         }
       }
     }
     if (!ok) abort_all(s);
+    if (lane == 0) bulk_wait_all();            // stores complete before the CTA exits
+    __syncwarp();
+  }
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* tiles = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* tiles_a = tiles;                                  // kStages x 16 KB
+  uint8_t* tiles_b = tiles + kStages * kStageA;              // kStages x 32 KB
+  uint8_t* staging = tiles + kStages * (kStageA + kStageB);  // kEpiWarps x 2 KB
+  GemmSmem* s = reinterpret_cast<GemmSmem*>(staging + kEpiWarps * kStagingBytes);
+  volatile int* abort_flag = &s->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s->full[i], 1);
+      mbar_init(&s->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s->tfull[i], 1);
+      mbar_init(&s->tempty[i], kEpiWarps);
+      mbar_init(&s->xbar[i], kEpiWarps);
+    }
+    for (int i = 0; i < kScaleSlots; ++i) {
+      mbar_init(&s->sfull[i], 32);
+      mbar_init(&s->sempty[i], kEpiWarps);
+    }
+    s->abort = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (MODE != kModeDense || args.c_tma) prefetch_tensormap(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s->tmem_base;
+
+  const int m_blocks = (MODE == kModeDense) ? (args.M + kBM - 1) / kBM : moe_m_blocks(args);
+  const int total_tiles = m_blocks * args.n_tiles;
+  const int num_kb = args.num_kb;
+  const int P = args.T * args.topk;
+
+  if (warp >= 4) {
+    warpgroup_reg_alloc<kRegsEpilogue>();
+    epilogue_role<MODE>(args, s, staging, &tmC, tmem_base, warp, lane, m_blocks, total_tiles, num_kb, P);
+  } else {
+    warpgroup_reg_dealloc<kRegsWg0>();     // one instruction for all four warps of warpgroup 0
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t sphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        int mb, nt;
+        tile_coords(tile, m_blocks, args.n_tiles, args.group_m, mb, nt);
+        const int e = (MODE == kModeDense) ? 0 : moe_expert(args, mb);
+        const int brow0 = (MODE == kModeMoeUp) ? e * args.b_rows_per_expert + nt * 128
+                                               : e * args.b_rows_per_expert + nt * kBN;
+        const int brow1 = (MODE == kModeMoeUp) ? brow0 + args.N : brow0 + 128;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&s->empty[stage], sphase ^ 1u, abort_flag)) { ok = false; break; }
+          if (lane == 0) {
+            uint8_t* sa_tile = tiles_a + stage * kStageA;
+            uint8_t* sb_tile = tiles_b + stage * kStageB;
+            mbar_arrive_expect_tx(&s->full[stage], kStageA + kStageB);
+            tma_load_2d(sa_tile, &tmA, &s->full[stage], kb * kBK, mb * kBM);
+            tma_load_2d(sb_tile, &tmB, &s->full[stage], kb * kBK, brow0);
+            tma_load_2d(sb_tile + kStageB / 2, &tmB, &s->full[stage], kb * kBK, brow1);
+          }
+          __syncwarp();
+          if (++stage == kStages) { stage = 0; sphase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        abort_all(s);
+        // let copies already in flight land before the CTA's shared memory goes away
+        const unsigned long long t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 10000000ull) {}
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------ scale loader
+      int sslot = 0;
+      uint32_t scphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        int mb, nt;
+        tile_coords(tile, m_blocks, args.n_tiles, args.group_m, mb, nt);
+        const int e = (MODE == kModeDense) ? 0 : moe_expert(args, mb);
+        // this lane's four rows of the tile: 4*lane .. 4*lane+3
+        const float* sa_src[4];
+  #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = mb * kBM + 4 * lane + i;
+          sa_src[i] = (MODE == kModeDense) ? args.a_scale + static_cast<size_t>(min(r, args.M - 1)) * num_kb
+                                           : args.a_scale + r;   // + kb * M
+        }
+        const size_t kstride = (MODE == kModeDense) ? 1 : static_cast<size_t>(args.M);
+        int nb0, nb1;
+        if (MODE == kModeMoeUp) {
+          nb0 = nt;
+          nb1 = args.N / 128 + nt;
+        } else {
+          nb0 = min(2 * nt, args.nb_valid - 1);
+          nb1 = min(2 * nt + 1, args.nb_valid - 1);
+        }
+        const float* sw_src0 = args.b_scale + (static_cast<size_t>(e) * args.nb_per_expert + nb0) * num_kb;
+        const float* sw_src1 = args.b_scale + (static_cast<size_t>(e) * args.nb_per_expert + nb1) * num_kb;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&s->sempty[sslot], scphase ^ 1u, abort_flag)) { ok = false; break; }
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) cp_async_4(&s->sa[sslot][4 * lane + i], sa_src[i] + kb * kstride);
+          if (lane == 0) {
+            cp_async_4(&s->sw[sslot][0], sw_src0 + kb);
+            cp_async_4(&s->sw[sslot][1], sw_src1 + kb);
+          }
+          cp_async_mbar_arrive(&s->sfull[sslot]);
+          if (++sslot == kScaleSlots) { sslot = 0; scphase ^= 1u; }
+        }
+      }
+      if (!ok) abort_all(s);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        int stage = 0, buf = 0;
+        uint32_t sphase = 0, tphase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&s->full[stage], sphase, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&s->tempty[buf], tphase ^ 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(tiles_a + stage * kStageA);
+            const uint32_t b_addr = smem_u32(tiles_b + stage * kStageB);
+            const uint32_t d_tmem = tmem_base + buf * kBN;
+  #pragma unroll
+            for (int k = 0; k < kBK / kUmmaK; ++k)
+              umma_f8(d_tmem, umma_desc_sw128(a_addr + k * kUmmaK), umma_desc_sw128(b_addr + k * kUmmaK), kIdesc,
+                      k > 0 ? 1u : 0u);
+            umma_commit(&s->empty[stage]);
+            umma_commit(&s->tfull[buf]);
+            if (++stage == kStages) { stage = 0; sphase ^= 1u; }
+            if (++buf == 2) { buf = 0; tphase ^= 1u; }
+          }
+        }
+        if (!ok) abort_all(s);
+      }
+      __syncwarp();
+    }                                    // warp 3 idles
   }
 
   tc_fence_before();
@@ -424,28 +468,55 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   }
 }
 
-// out[t, :] = bf16( y[t*K + 0] + y[t*K + 1] + ... + y[t*K + K-1] ), fp32 adds in slot
-// order (the routing weight is already in y). One thread per 8 columns.
+// Copies each sorted slot's token row of a8 [T, H] (and its H/128 scales from
+// a1_scale [H/128, T]) into slot order, and records pair -> slot. Padding slots
+// are skipped: the GEMMs treat rows independently and never store them.
+constexpr int kGatherWarps = 8;
+__global__ void __launch_bounds__(32 * kGatherWarps)
+moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_scale,
+                  const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ num_valid_ids, int T,
+                  int topk, int H, int cap, uint8_t* __restrict__ a8s, float* __restrict__ s1s,
+                  int32_t* __restrict__ slot_of_pair) {
+  const int lane = threadIdx.x & 31;
+  const int P = T * topk;
+  const int nv = min(max(*num_valid_ids, 0), cap);
+  const int KB = H / 128;
+  const int vec_per_row = H / 16;
+  for (int slot = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); slot < nv; slot += gridDim.x * kGatherWarps) {
+    const int sid = sorted_ids[slot];
+    if (sid < 0 || sid >= P) continue;
+    const int t = sid / topk;
+    const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
+    uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+    for (int kb = lane; kb < KB; kb += 32)
+      s1s[static_cast<size_t>(kb) * cap + slot] = a1_scale[static_cast<size_t>(kb) * T + t];
+    if (lane == 0) slot_of_pair[sid] = slot;
+  }
+}
+
+// out[t, :] = bf16( y[slot(t,0)] + y[slot(t,1)] + ... + y[slot(t,K-1)] ), fp32 adds
+// in slot order k (the routing weight is already in y). One thread per 8 columns.
 __global__ void __launch_bounds__(256)
-moe_combine_kernel(const float* __restrict__ ystage, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
+moe_combine_kernel(const float* __restrict__ ystage, const int32_t* __restrict__ slot_of_pair, int T, int K, int H,
+                   __nv_bfloat16* __restrict__ out) {
   const int cpr = H / 8;
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<size_t>(T) * cpr) return;
   const int t = static_cast<int>(idx / cpr);
   const int c = static_cast<int>(idx % cpr) * 8;
   float sum[8];
-  const float* y = ystage + static_cast<size_t>(t) * K * H + c;
-  {
+  for (int k = 0; k < K; ++k) {
+    const float* y = ystage + static_cast<size_t>(slot_of_pair[t * K + k]) * H + c;
     const float4 a = *reinterpret_cast<const float4*>(y);
     const float4 b = *reinterpret_cast<const float4*>(y + 4);
-    sum[0] = a.x; sum[1] = a.y; sum[2] = a.z; sum[3] = a.w;
-    sum[4] = b.x; sum[5] = b.y; sum[6] = b.z; sum[7] = b.w;
-  }
-  for (int k = 1; k < K; ++k) {
-    const float4 a = *reinterpret_cast<const float4*>(y + static_cast<size_t>(k) * H);
-    const float4 b = *reinterpret_cast<const float4*>(y + static_cast<size_t>(k) * H + 4);
-    sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
-    sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
+    if (k == 0) {
+      sum[0] = a.x; sum[1] = a.y; sum[2] = a.z; sum[3] = a.w;
+      sum[4] = b.x; sum[5] = b.y; sum[6] = b.z; sum[7] = b.w;
+    } else {
+      sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
+      sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
+    }
   }
   __align__(16) __nv_bfloat162 pk[4];
 #pragma unroll

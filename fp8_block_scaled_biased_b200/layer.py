@@ -68,5 +68,5 @@ class MoELayer:
                                         self.w1_scale, self.w2_scale, workspace=self.workspace)
         return self.out
 
-    # kernels launched by one forward: route, sort, quant, gate/up GEMM, down GEMM, combine
-    LAUNCHES_PER_FORWARD = 6
+    # kernels launched by one forward: route, sort, quant, gather, gate/up GEMM, down GEMM, combine
+    LAUNCHES_PER_FORWARD = 7
