@@ -151,20 +151,13 @@ int make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Epilogue store map: boxes of 32 rows x 64 bytes, 64-byte swizzle (the staging layout).
-int make_store_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t rows,
-                   uint64_t cols, uint64_t ld_bytes) {
-  return make_map_2d(map, dtype, elem_bytes, base, rows, cols, ld_bytes, 64 / elem_bytes, 32,
-                     CU_TENSOR_MAP_SWIZZLE_64B);
-}
-
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Scratch of the fused MoE call, all slot-ordered (capacity rows): the gathered
-// FP8 activations and their scales, pair -> slot, the re-quantised intermediate
-// and its scales, and the weighted down-projection rows.
+// Scratch of the fused MoE call: the slot-ordered FP8 activations and their
+// scales (capacity rows), the slot-ordered re-quantised intermediate and its
+// scales, and the weighted down-projection rows of every pair (by pair id).
 struct MoeWorkspace {
-  size_t a8s_off, s1s_off, inv_off, a2_off, s2_off, y_off, total;
+  size_t a8s_off, s1s_off, a2_off, s2_off, y_off, total;
 };
 
 MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I) {
@@ -177,10 +170,9 @@ MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I
   };
   w.a8s_off = take(capacity * static_cast<size_t>(H));
   w.s1s_off = take(static_cast<size_t>(H / 128) * capacity * sizeof(float));
-  w.inv_off = take(static_cast<size_t>(T) * topk * sizeof(int32_t));
   w.a2_off = take(capacity * static_cast<size_t>(I));
   w.s2_off = take(static_cast<size_t>(I / 128) * capacity * sizeof(float));
-  w.y_off = take(capacity * static_cast<size_t>(H) * sizeof(float));
+  w.y_off = take(static_cast<size_t>(T) * topk * H * sizeof(float));
   w.total = off;
   return w;
 }
@@ -193,8 +185,14 @@ struct TimingState {
 thread_local TimingState g_timing;
 
 void timing_record(int i, cudaStream_t st) {
-  // external record: inside a stream capture this becomes an event node of the graph
-  if (g_timing.on && g_timing.ev[i]) cudaEventRecordWithFlags(g_timing.ev[i], st, cudaEventRecordExternal);
+  if (!g_timing.on || !g_timing.ev[i]) return;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cap);
+  // inside a stream capture an external record becomes an event node of the graph
+  if (cap == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(g_timing.ev[i], st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(g_timing.ev[i], st);
 }
 
 int choose_group_m(int n_tiles) {
@@ -369,16 +367,9 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   if (!aligned16(A) || !aligned16(B)) return fail(FP8MOE_EINVAL, "A and B must be 16-byte aligned");
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
-  CUtensorMap ma, mb, mc;
+  CUtensorMap ma, mb;
   if (int rc = make_operand_map(&ma, A, M, K)) return rc;
   if (int rc = make_operand_map(&mb, B, N, K)) return rc;
-  const bool c_tma = (ldc % 8 == 0) && aligned16(C);
-  if (c_tma) {
-    if (int rc = make_store_map(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, M, N, static_cast<uint64_t>(ldc) * 2))
-      return rc;
-  } else {
-    mc = ma;   // unused: the kernel stores C directly
-  }
   GemmArgs a{};
   a.M = M;
   a.N = N;
@@ -391,12 +382,12 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   a.nb_valid = a.nb_per_expert;
   a.C = reinterpret_cast<__nv_bfloat16*>(C);
   a.ldc = ldc;
-  a.c_tma = c_tma ? 1 : 0;
+  a.c_vec = (ldc % 8 == 0) && aligned16(C);
   a.b_rows_per_expert = 0;
   const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * a.n_tiles;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   blockscale_gemm_kernel<kModeDense><<<grid, kGemmThreads, kGemmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      ma, mb, mc, a);
+      ma, mb, a);
   return check_gemm_launch("fp8_blockscale_gemm", blockscale_gemm_kernel<kModeDense>, kGemmThreads, kGemmSmemBytes);
 }
 
@@ -440,25 +431,20 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* a8s = ws + lay.a8s_off;
   float* s1s = reinterpret_cast<float*>(ws + lay.s1s_off);
-  int32_t* slot_of_pair = reinterpret_cast<int32_t*>(ws + lay.inv_off);
   uint8_t* a2 = ws + lay.a2_off;
   float* s2 = reinterpret_cast<float*>(ws + lay.s2_off);
   float* ystage = reinterpret_cast<float*>(ws + lay.y_off);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  CUtensorMap m_a8s, m_w1, m_a2_ld, m_a2_st, m_w2, m_y;
+  CUtensorMap m_a8s, m_w1, m_a2, m_w2;
   if (int rc = make_operand_map(&m_a8s, a8s, capacity, H)) return rc;
   if (int rc = make_operand_map(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H)) return rc;
-  if (int rc = make_operand_map(&m_a2_ld, a2, capacity, I)) return rc;
+  if (int rc = make_operand_map(&m_a2, a2, capacity, I)) return rc;
   if (int rc = make_operand_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
-  if (int rc = make_store_map(&m_a2_st, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a2, capacity, I, I)) return rc;
-  if (int rc = make_store_map(&m_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ystage, capacity, H,
-                              static_cast<uint64_t>(H) * 4))
-    return rc;
 
   timing_record(0, st);
   moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, num_valid_ids, T, topk, H,
-                                                            static_cast<int>(capacity), a8s, s1s, slot_of_pair);
+                                                            static_cast<int>(capacity), a8s, s1s);
   if (int rc = check_launch("fused_moe (gather)")) return rc;
 
   GemmArgs up{};
@@ -479,8 +465,10 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   up.topk = topk;
   up.E = E;
   up.b_rows_per_expert = 2 * I;
+  up.a2 = a2;
   up.s2 = s2;
-  blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, m_a2_st, up);
+  up.ystage = ystage;
+  blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, up);
   if (int rc = check_gemm_launch("fused_moe (gate/up GEMM)", blockscale_gemm_kernel<kModeMoeUp>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
@@ -497,7 +485,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   dn.nb_valid = H / 128;
   dn.b_rows_per_expert = H;
   dn.s2 = nullptr;
-  blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2_ld, m_w2, m_y, dn);
+  blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
   if (int rc = check_gemm_launch("fused_moe (down GEMM)", blockscale_gemm_kernel<kModeMoeDown>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
@@ -505,7 +493,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
 
   const size_t threads = static_cast<size_t>(T) * (H / 8);
   moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
-      ystage, slot_of_pair, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
+      ystage, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
   if (int rc = check_launch("fused_moe (combine)")) return rc;
   timing_record(3, st);
   return FP8MOE_OK;

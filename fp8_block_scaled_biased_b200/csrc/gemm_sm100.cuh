@@ -21,8 +21,8 @@
 //   warps 4..11 epilogue: tcgen05.ld the partials, multiply by
 //               a_scale[row, kb] * b_scale[col/128, kb] and add into fp32
 //               registers (the per-128-K promotion), then the mode's output,
-//               staged through a 64-byte-swizzled shared buffer per warp and
-//               written with TMA bulk stores.
+//               transposed through a small shared buffer per warp so that each
+//               store instruction writes whole 64-byte row segments.
 // In the MoE modes the rows are the sorted token-expert slots: A is the
 // slot-ordered activation matrix (gathered by moe_gather_kernel for GEMM1, the
 // re-quantised intermediate for GEMM2), one expert per 128-row block.
@@ -64,8 +64,8 @@ struct GemmArgs {
   const float* b_scale;   // [E][nb_per_expert][num_kb] (dense: E = 1)
   int nb_per_expert;      // 128-row scale blocks per expert matrix
   int nb_valid;           // dense: ceil(N/128) (clamp for the last tile)
-  int c_tma;              // dense: C can be written by TMA (else direct stores)
-  __nv_bfloat16* C;       // dense output (direct-store path)
+  int c_vec;              // dense: C rows allow 16-byte stores (ldc % 8 == 0, C 16-byte aligned)
+  __nv_bfloat16* C;       // dense output [M, ldc]
   int ldc;
   const int32_t* sorted_ids;
   const int32_t* sorted_expert_ids;
@@ -73,7 +73,9 @@ struct GemmArgs {
   const float* sorted_weights;
   int T, topk, E;
   int b_rows_per_expert;  // up: 2I; down: H
+  uint8_t* a2;            // up output [M, I] (slot-ordered FP8 intermediate)
   float* s2;              // up output [I/128, M]
+  float* ystage;          // down output [T*topk, H] (weighted rows by pair id)
 };
 
 struct GemmSmem {
@@ -127,33 +129,37 @@ __device__ __forceinline__ void abort_all(GemmSmem* s) {
   s->abort = 1;
 }
 
-// Writes 64 bytes of row `lane` into the warp's 32 x 64 B staging buffer in the
-// 64-byte-swizzled order a SWIZZLE_64B tensor map reads (16-byte chunk c of row
-// r lives at chunk c ^ ((r >> 1) & 3)), then stores the box with TMA.
-__device__ __forceinline__ void stage_and_store(uint8_t* staging, int lane, const uint4 (&d)[4],
-                                                const CUtensorMap* map, int x, int y, bool any_valid) {
-  if (lane == 0) bulk_wait_read_all();   // previous store from this buffer has read it
-  __syncwarp();
-  uint8_t* row = staging + lane * 64;
-  const int sw = (lane >> 1) & 3;
+// Writes a warp's 32 rows x 64 bytes (row = lane, data d) to global memory with
+// coalesced stores: each lane puts its row into the warp's shared staging buffer
+// (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3): no bank conflicts), then
+// each of four store instructions writes 8 whole 64-byte row segments.
+// row_addr(r) gives the destination of row r's segment, or nullptr to skip it;
+// every lane calls it (it may use warp shuffles).
+template <typename RowAddr>
+__device__ __forceinline__ void store_rows_64B(uint8_t* staging, int lane, const uint4 (&d)[4], RowAddr row_addr) {
+  uint8_t* mine = staging + lane * 64;
+  const int swz = (lane >> 1) & 3;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) = d[c];
-  fence_proxy_async_smem();
+  for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(mine + ((c ^ swz) << 4)) = d[c];
   __syncwarp();
-  if (lane == 0 && any_valid) {
-    tma_store_2d(map, staging, x, y);
-    bulk_commit();
+  const int c = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane >> 2);
+    const uint4 v = *reinterpret_cast<const uint4*>(staging + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    uint8_t* dst = row_addr(r);
+    if (dst) *reinterpret_cast<uint4*>(dst + c * 16) = v;
   }
+  __syncwarp();
 }
 
 // The epilogue warpgroups: promotion of each K block's partial sums into fp32
 // registers, then the mode's output through the per-warp staging buffer.
 template <int MODE>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s, uint8_t* staging,
-                                              const CUtensorMap* tmC_ptr, uint32_t tmem_base, int warp, int lane,
-                                              int m_blocks, int total_tiles, int num_kb, int P) {
+                                              uint32_t tmem_base, int warp, int lane, int m_blocks,
+                                              int total_tiles, int num_kb, int P) {
   volatile int* abort_flag = &s->abort;
-  const CUtensorMap& tmC = *tmC_ptr;
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 4;
     const int half = ew >> 2;                  // which 128 of the 256 MMA columns (up: which 64 of I)
@@ -208,8 +214,15 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         for (int c = 0; c < 4; ++c) {
           if (c + 1 < 4) tmem_ld_32x32b_x32(tb + ((c + 1) < 2 ? col0 : col1) + ((c + 1) & 1) * 32, v[(c + 1) & 1]);
           const float f = (c < 2) ? f0 : f1;
+          const float2 ff = make_float2(f, f);
+          // packed fp32 FMA (two lanes per instruction, each rounded to nearest)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(f, v[c & 1][j], acc[c * 32 + j]);
+          for (int j = 0; j < 32; j += 2) {
+            const float2 r = __ffma2_rn(ff, make_float2(v[c & 1][j], v[c & 1][j + 1]),
+                                        make_float2(acc[c * 32 + j], acc[c * 32 + j + 1]));
+            acc[c * 32 + j] = r.x;
+            acc[c * 32 + j + 1] = r.y;
+          }
           if (c + 1 < 4) {
             tmem_wait_ld();
             reg_fence_32(v[(c + 1) & 1]);
@@ -224,27 +237,30 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
 
       const int y0 = mb * kBM + quarter * 32;   // first row of this warp's 32-row slice
       if (MODE == kModeDense) {
-        const int grow = mb * kBM + row;
-        if (args.c_tma) {
+        __nv_bfloat16* C = args.C;
+        const int ldc = args.ldc, M = args.M, N = args.N;
+        const bool vec = args.c_vec != 0;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
-            const int x = nt * kBN + half * 128 + ch * 32;
-            const bool any = y0 < args.M && x < args.N;
-            uint4 d[4];
-            uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
+        for (int ch = 0; ch < 4; ++ch) {        // 4 chunks of 32 bf16 columns
+          const int x = nt * kBN + half * 128 + ch * 32;
+          uint4 d[4];
+          uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const __nv_bfloat162 p = __floats2bfloat162_rn(acc[ch * 32 + 2 * u], acc[ch * 32 + 2 * u + 1]);
-              w32[u] = *reinterpret_cast<const uint32_t*>(&p);
-            }
-            stage_and_store(my_staging, lane, d, &tmC, x, y0, any);
+          for (int u = 0; u < 16; ++u) {
+            const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[ch * 32 + 2 * u], acc[ch * 32 + 2 * u + 1]);
+            w32[u] = *reinterpret_cast<const uint32_t*>(&pk);
           }
-        } else if (grow < args.M) {
-          __nv_bfloat16* crow = args.C + static_cast<size_t>(grow) * args.ldc;
+          if (vec && x + 32 <= N) {
+            store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
+              const int grow = y0 + r;
+              return grow < M ? reinterpret_cast<uint8_t*>(C + static_cast<size_t>(grow) * ldc + x) : nullptr;
+            });
+          } else if (mb * kBM + row < M) {      // ragged edge or unaligned C: element stores
+            const __nv_bfloat16* vals = reinterpret_cast<const __nv_bfloat16*>(d);
+            __nv_bfloat16* crow = C + static_cast<size_t>(mb * kBM + row) * ldc;
 #pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            const int col = nt * kBN + half * 128 + j;
-            if (col < args.N) crow[col] = __float2bfloat16_rn(acc[j]);
+            for (int u = 0; u < 32; ++u)
+              if (x + u < N) crow[x + u] = vals[u];
           }
         }
       } else if (MODE == kModeMoeUp) {
@@ -253,7 +269,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           const float g = acc[j];
-          const float h = g / (1.0f + expf(-g)) * acc[64 + j];
+          const float h = __fdividef(g, 1.0f + __expf(-g)) * acc[64 + j];
           acc[j] = h;
           amax = fmaxf(amax, fabsf(h));
         }
@@ -265,47 +281,53 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         if (!mbar_wait(&s->xbar[xb], (tcount >> 1) & 1, abort_flag)) { ok = false; break; }
         amax = fmaxf(amax, s->amax_x[xb][half ^ 1][row]);
         const float scale = __fdiv_rn(amax, 448.0f);
+        const float inv = scale != 0.0f ? __frcp_rn(scale) : 0.0f;
         uint4 d[4];
         uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          w32[u] = 0u;
-          if (scale != 0.0f)
-            w32[u] = static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(acc[4 * u], scale),
-                                                      __fdiv_rn(acc[4 * u + 1], scale))) |
-                     (static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(acc[4 * u + 2], scale),
-                                                       __fdiv_rn(acc[4 * u + 3], scale)))
-                      << 16);
-        }
-        const bool any = __any_sync(0xffffffffu, pair >= 0 && pair < P);
-        stage_and_store(my_staging, lane, d, &tmC, nt * 128 + half * 64, y0, any);
+        for (int u = 0; u < 16; ++u)
+          w32[u] = static_cast<uint32_t>(cvt_e4m3x2(acc[4 * u] * inv, acc[4 * u + 1] * inv)) |
+                   (static_cast<uint32_t>(cvt_e4m3x2(acc[4 * u + 2] * inv, acc[4 * u + 3] * inv)) << 16);
+        uint8_t* a2_base = args.a2 + static_cast<size_t>(y0) * args.N + nt * 128 + half * 64;
+        const int ldI = args.N;
+        store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
+          const int pr = __shfl_sync(0xffffffffu, pair, r);
+          return (pr >= 0 && pr < P) ? a2_base + static_cast<size_t>(r) * ldI : nullptr;
+        });
         if (half == 0) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
       } else {
         const bool valid = pair >= 0 && pair < P;
         if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
-        const bool any = __any_sync(0xffffffffu, valid) && (nt * kBN + half * 128 < args.N);
+        const int x0 = nt * kBN + half * 128;
+        if (x0 < args.N) {
+          const int H = args.N;
+          float* y = args.ystage;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {        // 8 chunks of 16 fp32 columns
-          uint4 d[4];
+          for (int ch = 0; ch < 8; ++ch) {      // 8 chunks of 16 fp32 columns
+            uint4 d[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            d[u] = make_uint4(__float_as_uint(wroute * acc[ch * 16 + 4 * u]),
-                              __float_as_uint(wroute * acc[ch * 16 + 4 * u + 1]),
-                              __float_as_uint(wroute * acc[ch * 16 + 4 * u + 2]),
-                              __float_as_uint(wroute * acc[ch * 16 + 4 * u + 3]));
-          stage_and_store(my_staging, lane, d, &tmC, nt * kBN + half * 128 + ch * 16, y0, any);
+            for (int u = 0; u < 4; ++u)
+              d[u] = make_uint4(__float_as_uint(wroute * acc[ch * 16 + 4 * u]),
+                                __float_as_uint(wroute * acc[ch * 16 + 4 * u + 1]),
+                                __float_as_uint(wroute * acc[ch * 16 + 4 * u + 2]),
+                                __float_as_uint(wroute * acc[ch * 16 + 4 * u + 3]));
+            const int x = x0 + ch * 16;
+            store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
+              const int pr = __shfl_sync(0xffffffffu, pair, r);
+              return (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x)
+                                         : nullptr;
+            });
+          }
         }
       }
     }
     if (!ok) abort_all(s);
-    if (lane == 0) bulk_wait_all();            // stores complete before the CTA exits
-    __syncwarp();
   }
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+                       const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* tiles = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -335,7 +357,6 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     fence_mbar_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
-    if (MODE != kModeDense || args.c_tma) prefetch_tensormap(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(&s->tmem_base, kTmemCols);
@@ -353,7 +374,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
   if (warp >= 4) {
     warpgroup_reg_alloc<kRegsEpilogue>();
-    epilogue_role<MODE>(args, s, staging, &tmC, tmem_base, warp, lane, m_blocks, total_tiles, num_kb, P);
+    epilogue_role<MODE>(args, s, staging, tmem_base, warp, lane, m_blocks, total_tiles, num_kb, P);
   } else {
     warpgroup_reg_dealloc<kRegsWg0>();     // one instruction for all four warps of warpgroup 0
     if (warp == 0) {
@@ -469,14 +490,13 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 }
 
 // Copies each sorted slot's token row of a8 [T, H] (and its H/128 scales from
-// a1_scale [H/128, T]) into slot order, and records pair -> slot. Padding slots
-// are skipped: the GEMMs treat rows independently and never store them.
+// a1_scale [H/128, T]) into slot order. Padding slots are skipped: the GEMMs
+// treat rows independently and never store padding rows.
 constexpr int kGatherWarps = 8;
 __global__ void __launch_bounds__(32 * kGatherWarps)
 moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_scale,
                   const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ num_valid_ids, int T,
-                  int topk, int H, int cap, uint8_t* __restrict__ a8s, float* __restrict__ s1s,
-                  int32_t* __restrict__ slot_of_pair) {
+                  int topk, int H, int cap, uint8_t* __restrict__ a8s, float* __restrict__ s1s) {
   const int lane = threadIdx.x & 31;
   const int P = T * topk;
   const int nv = min(max(*num_valid_ids, 0), cap);
@@ -491,32 +511,31 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
     for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
     for (int kb = lane; kb < KB; kb += 32)
       s1s[static_cast<size_t>(kb) * cap + slot] = a1_scale[static_cast<size_t>(kb) * T + t];
-    if (lane == 0) slot_of_pair[sid] = slot;
   }
 }
 
-// out[t, :] = bf16( y[slot(t,0)] + y[slot(t,1)] + ... + y[slot(t,K-1)] ), fp32 adds
-// in slot order k (the routing weight is already in y). One thread per 8 columns.
+// out[t, :] = bf16( y[t*K + 0] + y[t*K + 1] + ... + y[t*K + K-1] ), fp32 adds in
+// slot order k (the routing weight is already in y). One thread per 8 columns.
 __global__ void __launch_bounds__(256)
-moe_combine_kernel(const float* __restrict__ ystage, const int32_t* __restrict__ slot_of_pair, int T, int K, int H,
-                   __nv_bfloat16* __restrict__ out) {
+moe_combine_kernel(const float* __restrict__ ystage, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
   const int cpr = H / 8;
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<size_t>(T) * cpr) return;
   const int t = static_cast<int>(idx / cpr);
   const int c = static_cast<int>(idx % cpr) * 8;
+  const float* y = ystage + static_cast<size_t>(t) * K * H + c;
   float sum[8];
-  for (int k = 0; k < K; ++k) {
-    const float* y = ystage + static_cast<size_t>(slot_of_pair[t * K + k]) * H + c;
+  {
     const float4 a = *reinterpret_cast<const float4*>(y);
     const float4 b = *reinterpret_cast<const float4*>(y + 4);
-    if (k == 0) {
-      sum[0] = a.x; sum[1] = a.y; sum[2] = a.z; sum[3] = a.w;
-      sum[4] = b.x; sum[5] = b.y; sum[6] = b.z; sum[7] = b.w;
-    } else {
-      sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
-      sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
-    }
+    sum[0] = a.x; sum[1] = a.y; sum[2] = a.z; sum[3] = a.w;
+    sum[4] = b.x; sum[5] = b.y; sum[6] = b.z; sum[7] = b.w;
+  }
+  for (int k = 1; k < K; ++k) {
+    const float4 a = *reinterpret_cast<const float4*>(y + static_cast<size_t>(k) * H);
+    const float4 b = *reinterpret_cast<const float4*>(y + static_cast<size_t>(k) * H + 4);
+    sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
+    sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
   }
   __align__(16) __nv_bfloat162 pk[4];
 #pragma unroll
