@@ -40,9 +40,13 @@ _SIGNATURES = {
     "fused_moe_fp8_blockscale_g1u1": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
                                                _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int, _p, _p,
                                                _c_size, _p]),
+    "fused_moe_fp8_blockscale_g1u1_noalloc": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int,
+                                                       _c_int, _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int,
+                                                       _p, _p]),
 }
 EXPORTED = tuple(_SIGNATURES)
 
+NOALLOC_SCRATCH_BYTES = 64 << 20   # FP8MOE_NOALLOC_SCRATCH_BYTES in include/fp8moe.h
 SCALE_ROW_MAJOR = 0
 SCALE_COL_MAJOR = 1
 FP8 = torch.float8_e4m3fn
@@ -266,4 +270,27 @@ def fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_pairs: SortedPairs, to
         _ptr(a1_scale), _ptr(fc1_scale), _ptr(fc2_scale), scale_blk_n, scale_blk_k, _ptr(fc2_smooth_scale),
         _ptr(workspace), workspace.numel(), _stream())
     _check("fused_moe_fp8_blockscale_g1u1", rc)
+    return out
+
+
+def fused_moe_fp8_blockscale_g1u1_noalloc(out, a8, w1, w2, sorted_pairs: SortedPairs, topk, a1_scale, fc1_scale,
+                                          fc2_scale, scale_blk_n=128, scale_blk_k=128, fc2_smooth_scale=None):
+    """fused_moe_fp8_blockscale_g1u1 using the library's built-in scratch (no workspace argument).
+
+    For callers that cannot allocate device memory. Problems needing more than
+    NOALLOC_SCRATCH_BYTES of scratch are rejected; calls share the scratch, so
+    they must not overlap on the GPU.
+    """
+    _cuda(out, torch.bfloat16, "out")
+    _cuda(a8, FP8, "a8")
+    T, H = a8.shape
+    E = w1.shape[0]
+    I = w2.shape[2]
+    sp = sorted_pairs
+    rc = load_library().fused_moe_fp8_blockscale_g1u1_noalloc(
+        _ptr(out), _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights),
+        _ptr(sp.sorted_expert_ids), _ptr(sp.num_valid_ids), T, H, I, E, topk, sp.block_m, sp.capacity,
+        _ptr(a1_scale), _ptr(fc1_scale), _ptr(fc2_scale), scale_blk_n, scale_blk_k, _ptr(fc2_smooth_scale),
+        _stream())
+    _check("fused_moe_fp8_blockscale_g1u1_noalloc", rc)
     return out

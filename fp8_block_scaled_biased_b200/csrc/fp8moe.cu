@@ -499,4 +499,52 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   return FP8MOE_OK;
 }
 
+// ------------------------------------------------------------------ no-allocation variant
+// The fused call's scratch for callers that cannot allocate device memory: one
+// fixed array per device, held for the life of the process. Its name is only a
+// host-side handle; the device address comes from cudaGetSymbolAddress, looked
+// up once per device on the first call (with that device current).
+}  // extern "C"
+
+namespace {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FP8MOE_NOALLOC_SCRATCH_BYTES];
+
+struct NoAllocScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+}  // namespace
+
+extern "C" {
+
+int fused_moe_fp8_blockscale_g1u1_noalloc(uint16_t* out, const uint8_t* a8, const uint8_t* w1, const uint8_t* w2,
+                                          const int32_t* sorted_ids, const float* sorted_weights,
+                                          const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T,
+                                          int H, int I, int E, int topk, int block_m, size_t capacity,
+                                          const float* a1_scale, const float* fc1_scale, const float* fc2_scale,
+                                          int scale_blk_n, int scale_blk_k, const float* fc2_smooth_scale,
+                                          void* stream) {
+  if (T < 0 || topk < 1 || H < 1 || I < 1) return fail(FP8MOE_EINVAL, "bad T, topk, H or I");
+  const size_t need = moe_workspace_layout(capacity, T, topk, H, I).total;
+  if (need > FP8MOE_NOALLOC_SCRATCH_BYTES)
+    return fail(FP8MOE_EUNSUPPORTED,
+                "fused_moe_fp8_blockscale_g1u1_noalloc: this problem needs %zu bytes of scratch, more than the "
+                "built-in %llu bytes; use fused_moe_fp8_blockscale_g1u1 with a caller-provided workspace",
+                need, static_cast<unsigned long long>(FP8MOE_NOALLOC_SCRATCH_BYTES));
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8MOE_ECUDA, "device ordinal %d unsupported", dev);
+  NoAllocScratch& sc = g_noalloc[dev];
+  std::call_once(sc.once, [&] { sc.err = cudaGetSymbolAddress(&sc.ptr, g_noalloc_scratch); });
+  if (sc.err != cudaSuccess || !sc.ptr)
+    return fail(FP8MOE_ECUDA, "scratch address lookup: %s", cudaGetErrorString(sc.err));
+  return fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_ids, sorted_weights, sorted_expert_ids,
+                                       num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
+                                       fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, sc.ptr,
+                                       FP8MOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 }  // extern "C"

@@ -220,6 +220,47 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/*
+ * Fused g1u1 MoE without any device allocation by the caller.
+ * (No counterpart in the source pages: an addition for callers that cannot
+ * allocate.)
+ *
+ * Same computation, arguments, layouts and limits as
+ * fused_moe_fp8_blockscale_g1u1, minus the workspace: the call uses a scratch
+ * array built into this library instead. It is for callers that must not
+ * allocate device memory at the point of the call, for example a serving loop
+ * whose memory manager owns all device memory after start-up, or a
+ * latency-critical path that cannot afford cudaMalloc's implicit device-wide
+ * synchronisation.
+ *
+ * The scratch is a fixed FP8MOE_NOALLOC_SCRATCH_BYTES array that every GPU
+ * loading the library keeps until the process exits. A problem whose scratch
+ * (fused_moe_fp8_blockscale_g1u1_workspace for the given capacity) is larger
+ * is rejected with FP8MOE_EUNSUPPORTED before anything is launched. The first
+ * call on a device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before capturing any stream on that device. All calls
+ * on a device share the one array and it keeps whatever the previous call left
+ * in it (nothing in it has to start at zero: every byte a call reads, that
+ * call has written first), so calls that can overlap on the GPU (different
+ * streams without ordering between them) race and corrupt each other: order
+ * them on one stream.
+ */
+#define FP8MOE_NOALLOC_SCRATCH_BYTES (64ull << 20)
+int fused_moe_fp8_blockscale_g1u1_noalloc(uint16_t* out, const uint8_t* a8,
+                                          const uint8_t* w1, const uint8_t* w2,
+                                          const int32_t* sorted_ids,
+                                          const float* sorted_weights,
+                                          const int32_t* sorted_expert_ids,
+                                          const int32_t* num_valid_ids,
+                                          int T, int H, int I, int E, int topk,
+                                          int block_m, size_t capacity,
+                                          const float* a1_scale,
+                                          const float* fc1_scale,
+                                          const float* fc2_scale, int scale_blk_n,
+                                          int scale_blk_k,
+                                          const float* fc2_smooth_scale,
+                                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif
