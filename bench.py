@@ -1,6 +1,6 @@
 """Benchmark of the fused FP8 block-scaled MoE layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed|tiny|profile]
                     [--impl ours|reference]
 
 One step = one forward of the whole layer on the device: biased grouped top-k
@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 from fp8_block_scaled_biased_b200 import inputs as I  # noqa: E402
 
-WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED}
+WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED, "profile": I.PROFILE}
 L2_FLUSH_BYTES = 256 << 20
 EXPERT_W1_BYTES = lambda c: 2 * c.I * c.H + (2 * c.I // 128) * (c.H // 128) * 4   # noqa: E731
 EXPERT_W2_BYTES = lambda c: c.H * c.I + (c.H // 128) * (c.I // 128) * 4            # noqa: E731

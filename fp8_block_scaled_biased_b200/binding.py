@@ -172,7 +172,12 @@ def alloc_sorted(T, topk, E, block_m, device) -> SortedPairs:
         block_m=block_m)
 
 
-def moe_align_sort(topk_ids, topk_weights, num_experts, block_m, out: SortedPairs | None = None) -> SortedPairs:
+def moe_align_sort_workspace_bytes(T, topk, E, block_m):
+    return load_library().moe_align_sort_workspace(T, topk, E, block_m)
+
+
+def moe_align_sort(topk_ids, topk_weights, num_experts, block_m, out: SortedPairs | None = None,
+                   workspace=None) -> SortedPairs:
     _cuda(topk_ids, torch.int32, "topk_ids")
     _cuda(topk_weights, torch.float32, "topk_weights")
     T, topk = topk_ids.shape
@@ -182,11 +187,12 @@ def moe_align_sort(topk_ids, topk_weights, num_experts, block_m, out: SortedPair
     if out is None:
         out = alloc_sorted(T, topk, num_experts, block_m, topk_ids.device)
     lib = load_library()
-    ws_bytes = lib.moe_align_sort_workspace(T, topk, num_experts, block_m)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=topk_ids.device)
+    if workspace is None:
+        workspace = torch.empty(lib.moe_align_sort_workspace(T, topk, num_experts, block_m), dtype=torch.uint8,
+                                device=topk_ids.device)
     rc = lib.moe_align_sort(_ptr(topk_ids), _ptr(topk_weights), ld, T, topk, num_experts, block_m,
                             _ptr(out.sorted_ids), _ptr(out.sorted_weights), _ptr(out.sorted_expert_ids),
-                            _ptr(out.num_valid_ids), out.capacity, _ptr(ws), ws_bytes, _stream())
+                            _ptr(out.num_valid_ids), out.capacity, _ptr(workspace), workspace.numel(), _stream())
     _check("moe_align_sort", rc)
     return out
 

@@ -97,8 +97,8 @@ int device_setup(int* sm_count) {
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeUp>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown>();
     if (r == cudaSuccess)
-      r = cudaFuncSetAttribute(align_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (2 + kSortWarps) * kSortMaxExperts * static_cast<int>(sizeof(int)));
+      r = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSortWarps * kSortMaxExperts * static_cast<int>(sizeof(int)));
     d.err = static_cast<int>(r);
   });
   if (d.err == -1) return fail(FP8MOE_EUNSUPPORTED, "device %d is not sm_100 (B200)", dev);
@@ -300,13 +300,16 @@ size_t moe_align_sort_capacity(int T, int topk, int E, int block_m) {
   return static_cast<size_t>(T) * topk + static_cast<size_t>(E) * (block_m - 1);
 }
 
-size_t moe_align_sort_workspace(int, int, int, int) { return 0; }
+size_t moe_align_sort_workspace(int T, int topk, int E, int block_m) {
+  if (T < 0 || topk < 1 || E < 1 || block_m < 1) return 0;
+  const size_t pairs = static_cast<size_t>(T) * topk;
+  const size_t nchunks = (pairs + kSortChunk - 1) / kSortChunk;
+  return round_up(nchunks * E * sizeof(int32_t), 256) + round_up(E * sizeof(int32_t), 256);
+}
 
 int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, int T, int topk, int E, int block_m,
                    int32_t* sorted_ids, float* sorted_weights, int32_t* sorted_expert_ids, int32_t* num_valid_ids,
                    size_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (T < 0 || topk < 1) return fail(FP8MOE_EINVAL, "T >= 0 and topk >= 1 required");
   if (E < 1 || E > kSortMaxExperts) return fail(FP8MOE_EUNSUPPORTED, "E must be in [1, %d]", kSortMaxExperts);
   if (block_m < 1 || block_m > 1024) return fail(FP8MOE_EINVAL, "block_m must be in [1, 1024]");
@@ -316,12 +319,30 @@ int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, i
     return fail(FP8MOE_EINVAL, "capacity %zu < required %zu", capacity, moe_align_sort_capacity(T, topk, E, block_m));
   if (!sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids || (T > 0 && (!topk_ids || !topk_weights)))
     return fail(FP8MOE_EINVAL, "null pointer argument");
+  const size_t need = moe_align_sort_workspace(T, topk, E, block_m);
+  if (!workspace || workspace_bytes < need)
+    return fail(FP8MOE_EWORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
-  const size_t smem = static_cast<size_t>(2 + kSortWarps) * E * sizeof(int);
-  align_sort_kernel<<<1, kSortThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      topk_ids, topk_weights, ld, T, topk, E, block_m, sorted_ids, sorted_weights, sorted_expert_ids, num_valid_ids);
-  return check_launch("moe_align_sort");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int pairs = T * topk;
+  const int nchunks = (pairs + kSortChunk - 1) / kSortChunk;
+  int32_t* counts = static_cast<int32_t*>(workspace);                       // [nchunks][E]
+  int32_t* seg_start = counts + round_up(static_cast<size_t>(nchunks) * E * sizeof(int32_t), 256) / sizeof(int32_t);
+  if (nchunks > 0) {
+    sort_count_kernel<<<nchunks, kSortChunk, E * sizeof(int), st>>>(topk_ids, ld, T, topk, E, counts);
+    if (int rc = check_launch("moe_align_sort (count)")) return rc;
+  }
+  sort_scan_kernel<<<1, kSortChunk, 2 * E * sizeof(int), st>>>(counts, seg_start, nchunks, T, topk, E, block_m,
+                                                               sorted_ids, sorted_weights, sorted_expert_ids,
+                                                               num_valid_ids);
+  if (int rc = check_launch("moe_align_sort (scan)")) return rc;
+  if (nchunks > 0) {
+    sort_scatter_kernel<<<nchunks, kSortChunk, static_cast<size_t>(kSortWarps) * E * sizeof(int), st>>>(
+        topk_ids, topk_weights, ld, T, topk, E, counts, seg_start, sorted_ids, sorted_weights);
+    if (int rc = check_launch("moe_align_sort (scatter)")) return rc;
+  }
+  return FP8MOE_OK;
 }
 
 // ------------------------------------------------------------------ S3 quant

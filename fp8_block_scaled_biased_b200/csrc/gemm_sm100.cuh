@@ -508,7 +508,21 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
     const int t = sid / topk;
     const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
     uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+    // issue a batch of loads before their stores, so the row costs one round trip per batch
+    constexpr int kBatch = 16;
+    for (int v0 = 0; v0 < vec_per_row; v0 += 32 * kBatch) {
+      uint4 buf[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < vec_per_row) buf[i] = src[v];
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < vec_per_row) dst[v] = buf[i];
+      }
+    }
     for (int kb = lane; kb < KB; kb += 32)
       s1s[static_cast<size_t>(kb) * cap + slot] = a1_scale[static_cast<size_t>(kb) * T + t];
   }

@@ -7,18 +7,23 @@
 // segment padded to a multiple of block_m with id T*topk and weight 0; one
 // expert id per block; experts without pairs get no block.
 //
-// One CTA does it all: a shared-memory histogram, a scan over experts, then a
-// stable scatter in chunks of 1024 pairs (one per thread) in which a pair's
-// slot is its expert's running base + the count of same-expert pairs in lower
-// warps of the chunk + its rank among same-expert lanes of its warp.
+// Three kernels over chunks of kSortChunk consecutive pairs (one CTA each):
+//   1. sort_count_kernel: per-chunk expert histogram -> counts[chunk][E];
+//   2. sort_scan_kernel (one CTA): each expert's padded segment start, and for
+//      every (chunk, expert) the number of that expert's pairs in earlier
+//      chunks; block expert ids, padding slots and num_valid_ids;
+//   3. sort_scatter_kernel: stable rank of each pair inside its chunk (count of
+//      same-expert pairs in lower warps + rank among same-expert lanes of its
+//      warp) added to its expert's segment start and earlier chunks' count.
+// Stable by construction: no atomics decide an order.
 #pragma once
 
 #include "common.cuh"
 
 namespace fp8moe {
 
-constexpr int kSortThreads = 1024;
-constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kSortChunk = 1024;                 // pairs per CTA = threads per CTA
+constexpr int kSortWarps = kSortChunk / 32;
 constexpr int kSortMaxExperts = 1024;
 
 __device__ __forceinline__ int read_pair_expert(const int32_t* ids, int ld, int K, int p, int E) {
@@ -27,96 +32,120 @@ __device__ __forceinline__ int read_pair_expert(const int32_t* ids, int ld, int 
   return (e >= 0 && e < E) ? e : -1;
 }
 
-// dynamic shared memory: cnt[E] | base[E] | warp_cnt[kSortWarps][E]
-__global__ void __launch_bounds__(kSortThreads, 1)
-align_sort_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, int ld, int T, int K, int E,
-                  int block_m, int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w,
-                  int32_t* __restrict__ sorted_e, int32_t* __restrict__ num_valid) {
-  extern __shared__ int sm_sort[];
-  int* cnt = sm_sort;
-  int* base = cnt + E;
-  int* warp_cnt = base + E;
-  __shared__ int s_bad;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// 1. counts[c][e] = pairs of chunk c routed to expert e.
+__global__ void __launch_bounds__(kSortChunk)
+sort_count_kernel(const int32_t* __restrict__ ids, int ld, int T, int K, int E, int32_t* __restrict__ counts) {
+  extern __shared__ int sm_cnt[];
   const int P = T * K;
-
-  for (int e = tid; e < E; e += kSortThreads) cnt[e] = 0;
-  if (tid == 0) s_bad = 0;
+  for (int e = threadIdx.x; e < E; e += kSortChunk) sm_cnt[e] = 0;
   __syncthreads();
-
-  // 1. histogram
-  for (int p = tid; p < P; p += kSortThreads) {
+  const int p = blockIdx.x * kSortChunk + threadIdx.x;
+  if (p < P) {
     const int e = read_pair_expert(ids, ld, K, p, E);
     if (e >= 0)
-      atomicAdd(&cnt[e], 1);
+      atomicAdd(&sm_cnt[e], 1);
     else
-      s_bad = 1;
+      raise_device_error(FP8MOE_DEVERR_EXPERT_ID);
   }
   __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kSortChunk) counts[static_cast<size_t>(blockIdx.x) * E + e] = sm_cnt[e];
+}
 
-  // 2. padded segment starts (exclusive scan of ceil(cnt/bm)*bm over experts, by warp 0)
+// 2. One CTA. counts[c][e] becomes the number of expert-e pairs in chunks before
+//    c; seg_start[e] is expert e's padded segment start. Segment tails are
+//    padded; block expert ids and num_valid_ids are written.
+__global__ void __launch_bounds__(kSortChunk)
+sort_scan_kernel(int32_t* __restrict__ counts, int32_t* __restrict__ seg_start, int nchunks, int T, int K, int E,
+                 int block_m, int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w,
+                 int32_t* __restrict__ sorted_e, int32_t* __restrict__ num_valid) {
+  extern __shared__ int sm_scan[];
+  int* total = sm_scan;          // [E] pairs per expert
+  int* start = sm_scan + E;      // [E] padded segment start
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int P = T * K;
+  // per expert: exclusive prefix over chunks (in place), eight chunks' loads in flight at a time
+  for (int e = tid; e < E; e += kSortChunk) {
+    int run = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = (c0 + i < nchunks) ? counts[static_cast<size_t>(c0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (c0 + i < nchunks) counts[static_cast<size_t>(c0 + i) * E + e] = run;
+        run += v[i];
+      }
+    }
+    total[e] = run;
+  }
+  __syncthreads();
+  // padded segment starts: exclusive scan of ceil(total/bm)*bm over experts (warp 0)
   if (warp == 0) {
     int carry = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
-      const int c = (e < E) ? cnt[e] : 0;
-      const int len = (c + block_m - 1) / block_m * block_m;
+      const int len = (e < E) ? (total[e] + block_m - 1) / block_m * block_m : 0;
       int incl = len;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
-      if (e < E) base[e] = carry + incl - len;
+      if (e < E) start[e] = carry + incl - len;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      *num_valid = carry;
-      if (s_bad) raise_device_error(FP8MOE_DEVERR_EXPERT_ID);
+    if (lane == 0) *num_valid = carry;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kSortChunk) seg_start[e] = start[e];
+  // block expert ids and padding slots
+  for (int e = warp; e < E; e += kSortWarps) {
+    const int c = total[e];
+    const int s0 = start[e];
+    const int len = (c + block_m - 1) / block_m * block_m;
+    for (int j = lane; j < len / block_m; j += 32) sorted_e[s0 / block_m + j] = e;
+    for (int sl = s0 + c + lane; sl < s0 + len; sl += 32) {
+      sorted_ids[sl] = P;
+      sorted_w[sl] = 0.0f;
+    }
+  }
+}
+
+// 3. Stable scatter of chunk blockIdx.x.
+__global__ void __launch_bounds__(kSortChunk)
+sort_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, int ld, int T, int K, int E,
+                    const int32_t* __restrict__ before, const int32_t* __restrict__ seg_start,
+                    int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w) {
+  extern __shared__ int warp_cnt[];   // [kSortWarps][E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int P = T * K;
+  const int p = blockIdx.x * kSortChunk + tid;
+  const int e = (p < P) ? read_pair_expert(ids, ld, K, p, E) : -1;
+  float wv = 0.0f;
+  if (e >= 0) {
+    const int t = p / K, k = p - t * K;
+    wv = w[static_cast<size_t>(t) * ld + k];
+  }
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(same & ((1u << lane) - 1u));
+  for (int i = tid; i < kSortWarps * E; i += kSortChunk) warp_cnt[i] = 0;
+  __syncthreads();
+  if (e >= 0 && rank == 0) warp_cnt[warp * E + e] = __popc(same);
+  __syncthreads();
+  // per expert: exclusive prefix over the warps of this chunk, from the chunk's first slot
+  for (int ex = tid; ex < E; ex += kSortChunk) {
+    int run = seg_start[ex] + before[static_cast<size_t>(blockIdx.x) * E + ex];
+    for (int wi = 0; wi < kSortWarps; ++wi) {
+      const int v = warp_cnt[wi * E + ex];
+      warp_cnt[wi * E + ex] = run;
+      run += v;
     }
   }
   __syncthreads();
-
-  // 3. block expert ids and padding slots
-  for (int e = warp; e < E; e += kSortWarps) {
-    const int c = cnt[e];
-    const int start = base[e];
-    const int len = (c + block_m - 1) / block_m * block_m;
-    for (int j = lane; j < len / block_m; j += 32) sorted_e[start / block_m + j] = e;
-    for (int s = start + c + lane; s < start + len; s += 32) {
-      sorted_ids[s] = P;
-      sorted_w[s] = 0.0f;
-    }
-  }
-
-  // 4. stable scatter, 1024 pairs per round
-  for (int c0 = 0; c0 < P; c0 += kSortThreads) {
-    const int p = c0 + tid;
-    const int e = (p < P) ? read_pair_expert(ids, ld, K, p, E) : -1;
-    const unsigned same = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(same & ((1u << lane) - 1u));
-    for (int i = tid; i < kSortWarps * E; i += kSortThreads) warp_cnt[i] = 0;
-    __syncthreads();
-    if (e >= 0 && rank == 0) warp_cnt[warp * E + e] = __popc(same);
-    __syncthreads();
-    // per expert: exclusive prefix over warps, from the expert's running base
-    for (int ex = tid; ex < E; ex += kSortThreads) {
-      int run = base[ex];
-      for (int wi = 0; wi < kSortWarps; ++wi) {
-        const int v = warp_cnt[wi * E + ex];
-        warp_cnt[wi * E + ex] = run;
-        run += v;
-      }
-      base[ex] = run;
-    }
-    __syncthreads();
-    if (e >= 0) {
-      const int slot = warp_cnt[warp * E + e] + rank;
-      const int t = p / K, k = p - t * K;
-      sorted_ids[slot] = p;
-      sorted_w[slot] = w[static_cast<size_t>(t) * ld + k];
-    }
-    __syncthreads();
+  if (e >= 0) {
+    const int slot = warp_cnt[warp * E + e] + rank;
+    sorted_ids[slot] = p;
+    sorted_w[slot] = wv;
   }
 }
 

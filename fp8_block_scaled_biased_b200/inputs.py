@@ -72,7 +72,11 @@ SKEWED = MoEConfig("skewed_t16384_h7168_e256", T=16384, H=7168, E=256, G=8, TG=4
                    hot_experts=16)
 GEMM = GemmConfig("gemm_m2048_n4096_k7168", M=2048, N=4096, K=7168)
 
-MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED)}
+# The decode/prefill layer shape with 32 experts (1.4 GB of weights, more than
+# L2) and 512 tokens: small enough for full-set profiler captures.
+PROFILE = MoEConfig("profile_t512_h7168_e32", T=512, H=7168, E=32, G=8, TG=4, K=8, I=2048)
+
+MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, PROFILE)}
 
 
 @dataclass

@@ -40,6 +40,8 @@ class MoELayer:
         self.topk_w = torch.empty(T, cfg.K, dtype=torch.float32, device=dev)
         self.topk_ids = torch.empty(T, cfg.K, dtype=torch.int32, device=dev)
         self.sorted = B.alloc_sorted(T, cfg.K, cfg.E, self.block_m, dev)
+        self.sort_workspace = torch.empty(B.moe_align_sort_workspace_bytes(T, cfg.K, cfg.E, self.block_m),
+                                          dtype=torch.uint8, device=dev)
         self.a8 = torch.empty(T, cfg.H, dtype=B.FP8, device=dev)
         self.a8_scale = torch.empty(cfg.H // 128, T, dtype=torch.float32, device=dev)
         self.out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
@@ -62,11 +64,13 @@ class MoELayer:
         if T != self.max_tokens:
             raise ValueError(f"layer buffers are sized for {self.max_tokens} tokens, got {T}")
         B.moe_biased_grouped_topk(logits, bias, self.topk_w, self.topk_ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
-        B.moe_align_sort(self.topk_ids, self.topk_w, cfg.E, self.block_m, out=self.sorted)
+        B.moe_align_sort(self.topk_ids, self.topk_w, cfg.E, self.block_m, out=self.sorted,
+                         workspace=self.sort_workspace)
         B.fp8_per_token_group_quant(x, 128, column_major_scales=True, q=self.a8, scales=self.a8_scale)
         B.fused_moe_fp8_blockscale_g1u1(self.out, self.a8, self.w1, self.w2, self.sorted, cfg.K, self.a8_scale,
                                         self.w1_scale, self.w2_scale, workspace=self.workspace)
         return self.out
 
-    # kernels launched by one forward: route, sort, quant, gather, gate/up GEMM, down GEMM, combine
-    LAUNCHES_PER_FORWARD = 7
+    # kernels launched by one forward: route, sort (count, scan, scatter), quant, gather, gate/up GEMM,
+    # down GEMM, combine
+    LAUNCHES_PER_FORWARD = 9
