@@ -186,6 +186,13 @@ __host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// 32-byte store (one full sector) of eight 32-bit words; p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // ---------------------------------------------------------------- FP8 conversion
 // Two fp32 -> two E4M3 codes, round to nearest even, saturating (hardware cvt).
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {

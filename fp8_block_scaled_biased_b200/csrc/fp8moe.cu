@@ -403,7 +403,7 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   a.nb_valid = a.nb_per_expert;
   a.C = reinterpret_cast<__nv_bfloat16*>(C);
   a.ldc = ldc;
-  a.c_vec = (ldc % 8 == 0) && aligned16(C);
+  a.c_vec = (ldc % 16 == 0) && (reinterpret_cast<uintptr_t>(C) & 31u) == 0;   // 32-byte row stores
   a.b_rows_per_expert = 0;
   const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * a.n_tiles;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);

@@ -20,9 +20,10 @@
 //               8-slot ring (cp.async); warp 3 idles;
 //   warps 4..11 epilogue: tcgen05.ld the partials, multiply by
 //               a_scale[row, kb] * b_scale[col/128, kb] and add into fp32
-//               registers (the per-128-K promotion), then the mode's output,
-//               transposed through a small shared buffer per warp so that each
-//               store instruction writes whole 64-byte row segments.
+//               registers (the per-128-K promotion), then the mode's output:
+//               32-byte (whole-sector) stores of each thread's row, or for the
+//               down GEMM's fp32 rows a transpose through a small shared buffer
+//               per warp so that each store writes 8 whole 64-byte row segments.
 // In the MoE modes the rows are the sorted token-expert slots: A is the
 // slot-ordered activation matrix (gathered by moe_gather_kernel for GEMM1, the
 // re-quantised intermediate for GEMM2), one expert per 128-row block.
@@ -64,7 +65,7 @@ struct GemmArgs {
   const float* b_scale;   // [E][nb_per_expert][num_kb] (dense: E = 1)
   int nb_per_expert;      // 128-row scale blocks per expert matrix
   int nb_valid;           // dense: ceil(N/128) (clamp for the last tile)
-  int c_vec;              // dense: C rows allow 16-byte stores (ldc % 8 == 0, C 16-byte aligned)
+  int c_vec;              // dense: C rows allow 32-byte stores (ldc % 16 == 0, C 32-byte aligned)
   __nv_bfloat16* C;       // dense output [M, ldc]
   int ldc;
   const int32_t* sorted_ids;
@@ -235,32 +236,31 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
       }
       if (!ok) break;
 
-      const int y0 = mb * kBM + quarter * 32;   // first row of this warp's 32-row slice
+      // Outputs. Dense and gate/up: each thread writes its own row with 32-byte
+      // stores (whole sectors) straight from registers.
       if (MODE == kModeDense) {
-        __nv_bfloat16* C = args.C;
-        const int ldc = args.ldc, M = args.M, N = args.N;
-        const bool vec = args.c_vec != 0;
+        const int grow = mb * kBM + row;
+        const int x0 = nt * kBN + half * 128;
+        if (grow < args.M) {
+          __nv_bfloat16* crow = args.C + static_cast<size_t>(grow) * args.ldc;
+          const bool vec = args.c_vec != 0 && x0 + 128 <= args.N;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {        // 4 chunks of 32 bf16 columns
-          const int x = nt * kBN + half * 128 + ch * 32;
-          uint4 d[4];
-          uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
+          for (int ch = 0; ch < 8; ++ch) {      // 8 chunks of 16 bf16 columns
+            uint32_t w[8];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[ch * 32 + 2 * u], acc[ch * 32 + 2 * u + 1]);
-            w32[u] = *reinterpret_cast<const uint32_t*>(&pk);
-          }
-          if (vec && x + 32 <= N) {
-            store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
-              const int grow = y0 + r;
-              return grow < M ? reinterpret_cast<uint8_t*>(C + static_cast<size_t>(grow) * ldc + x) : nullptr;
-            });
-          } else if (mb * kBM + row < M) {      // ragged edge or unaligned C: element stores
-            const __nv_bfloat16* vals = reinterpret_cast<const __nv_bfloat16*>(d);
-            __nv_bfloat16* crow = C + static_cast<size_t>(mb * kBM + row) * ldc;
+            for (int u = 0; u < 8; ++u) {
+              const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[ch * 16 + 2 * u], acc[ch * 16 + 2 * u + 1]);
+              w[u] = *reinterpret_cast<const uint32_t*>(&pk);
+            }
+            const int x = x0 + ch * 16;
+            if (vec) {
+              st_global_v8(crow + x, w);
+            } else {                            // ragged edge or unaligned C: element stores
+              const __nv_bfloat16* vals = reinterpret_cast<const __nv_bfloat16*>(w);
 #pragma unroll
-            for (int u = 0; u < 32; ++u)
-              if (x + u < N) crow[x + u] = vals[u];
+              for (int u = 0; u < 16; ++u)
+                if (x + u < args.N) crow[x + u] = vals[u];
+            }
           }
         }
       } else if (MODE == kModeMoeUp) {
@@ -282,20 +282,24 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         amax = fmaxf(amax, s->amax_x[xb][half ^ 1][row]);
         const float scale = __fdiv_rn(amax, 448.0f);
         const float inv = scale != 0.0f ? __frcp_rn(scale) : 0.0f;
-        uint4 d[4];
-        uint32_t* w32 = reinterpret_cast<uint32_t*>(d);
+        if (pair >= 0 && pair < P) {
+          uint8_t* dst = args.a2 + static_cast<size_t>(slot) * args.N + nt * 128 + half * 64;
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          w32[u] = static_cast<uint32_t>(cvt_e4m3x2(acc[4 * u] * inv, acc[4 * u + 1] * inv)) |
-                   (static_cast<uint32_t>(cvt_e4m3x2(acc[4 * u + 2] * inv, acc[4 * u + 3] * inv)) << 16);
-        uint8_t* a2_base = args.a2 + static_cast<size_t>(y0) * args.N + nt * 128 + half * 64;
-        const int ldI = args.N;
-        store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
-          const int pr = __shfl_sync(0xffffffffu, pair, r);
-          return (pr >= 0 && pr < P) ? a2_base + static_cast<size_t>(r) * ldI : nullptr;
-        });
+          for (int ch = 0; ch < 2; ++ch) {      // 2 x 32 codes
+            uint32_t w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int j = ch * 32 + 4 * u;
+              w[u] = static_cast<uint32_t>(cvt_e4m3x2(acc[j] * inv, acc[j + 1] * inv)) |
+                     (static_cast<uint32_t>(cvt_e4m3x2(acc[j + 2] * inv, acc[j + 3] * inv)) << 16);
+            }
+            st_global_v8(dst + ch * 32, w);
+          }
+        }
         if (half == 0) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
       } else {
+        // 512 bytes of fp32 per row: a transpose through the warp's staging buffer
+        // lets each store instruction write 8 whole 64-byte row segments
         const bool valid = pair >= 0 && pair < P;
         if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
         const int x0 = nt * kBN + half * 128;
