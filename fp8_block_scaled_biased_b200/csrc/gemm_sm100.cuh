@@ -424,7 +424,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         const int e = (MODE == kModeDense) ? 0 : moe_expert(args, mb);
         // this lane's four rows of the tile: 4*lane .. 4*lane+3
         const float* sa_src[4];
-  #pragma unroll
+#pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = mb * kBM + 4 * lane + i;
           sa_src[i] = (MODE == kModeDense) ? args.a_scale + static_cast<size_t>(min(r, args.M - 1)) * num_kb
@@ -443,7 +443,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         const float* sw_src1 = args.b_scale + (static_cast<size_t>(e) * args.nb_per_expert + nb1) * num_kb;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&s->sempty[sslot], scphase ^ 1u, abort_flag)) { ok = false; break; }
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 4; ++i) cp_async_4(&s->sa[sslot][4 * lane + i], sa_src[i] + kb * kstride);
           if (lane == 0) {
             cp_async_4(&s->sw[sslot][0], sw_src0 + kb);
@@ -469,7 +469,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const uint32_t a_addr = smem_u32(tiles_a + stage * kStageA);
             const uint32_t b_addr = smem_u32(tiles_b + stage * kStageB);
             const uint32_t d_tmem = tmem_base + buf * kBN;
-  #pragma unroll
+#pragma unroll
             for (int k = 0; k < kBK / kUmmaK; ++k)
               umma_f8(d_tmem, umma_desc_sw128(a_addr + k * kUmmaK), umma_desc_sw128(b_addr + k * kUmmaK), kIdesc,
                       k > 0 ? 1u : 0u);
