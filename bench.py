@@ -26,7 +26,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -40,6 +39,7 @@ from fp8_block_scaled_biased_b200 import inputs as I  # noqa: E402
 
 WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED, "profile": I.PROFILE}
 L2_FLUSH_BYTES = 256 << 20
+METRIC = "fused FP8-blockscale MoE layer tokens/s and TFLOPS at 1 B200; % of FP8/HBM roofline"
 EXPERT_W1_BYTES = lambda c: 2 * c.I * c.H + (2 * c.I // 128) * (c.H // 128) * 4   # noqa: E731
 EXPERT_W2_BYTES = lambda c: c.H * c.I + (c.H // 128) * (c.I // 128) * 4            # noqa: E731
 
@@ -54,55 +54,74 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+def _nvml_handle(local):
+    """NVML handle of CUDA device `local`, matched by PCI address (CUDA and NVML orders may differ)."""
+    import pynvml
+    pynvml.nvmlInit()
+    props = torch.cuda.get_device_properties(local)
+    bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus), bus
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+
+class ClockSampler:
+    """SM clock, power and clock-event reasons of the benchmarked GPU, sampled
+    every 10 ms (NVML, read-only queries) while the timed region runs."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, local, period_s=0.01):
+        self.local = local
+        self.period = period_s
+        self.samples = []
+        self.err = None
+        self._stop = threading.Event()
+        self.thread = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            self.nv, self.h, self.bus = _nvml_handle(self.local)
+            self.max_mhz = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - sampling is best effort; the reason is reported
+            self.err = f"nvml unavailable: {type(e).__name__}: {e}"
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, pw, rs))
+            except Exception as e:  # noqa: BLE001
+                self.err = f"nvml query failed: {e}"
+                return
+            time.sleep(self.period)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "not sampled"]}
+        self._stop.set()
+        self.thread.join(timeout=5)
+        reasons = set()
+        for _, _, rs in self.samples:
+            for name, const in self.REASONS:
+                if rs & getattr(self.nv, const, 0):
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [x[0] for x in self.samples]
+        pw = [x[1] for x in self.samples]
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+               "sm_mhz_min": min(sm) if sm else None, "power_w_median": statistics.median(pw) if pw else None,
+               "reasons": sorted(reasons), "samples": len(sm), "period_ms": self.period * 1e3,
+               "source": f"nvml, device {self.bus}"}
+        if self.err:
+            out["error"] = self.err
+        return out
 
 
 def dist_setup(args):
@@ -152,6 +171,34 @@ def layer_work(cfg, ids):
                 gemm1_flops=gemm1_flops)
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gate/up GEMM
+# launch from a one-pass ncu capture of this bench's own command, keyed by
+# workload, with the SHA-256 of the GEMM kernel sources the capture ran. A
+# figure whose sources have changed since is not reported.
+GATE_UP_TRAFFIC = {}
+GEMM_SOURCES = ("fp8_block_scaled_biased_b200/csrc/gemm_sm100.cuh", "fp8_block_scaled_biased_b200/csrc/common.cuh")
+
+
+def gemm_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gate_up_traffic(workload, override):
+    if override is not None:
+        return override, "given on the command line"
+    rec = GATE_UP_TRAFFIC.get(workload)
+    if rec is None:
+        return None, "no capture for this workload"
+    if rec["sha256"] != gemm_source_sha():
+        return None, "kernel sources changed since the capture"
+    return rec["bytes"], rec["capture"]
+
+
 def run_ours(args, world, rank, local):
     from fp8_block_scaled_biased_b200 import binding as B
     from fp8_block_scaled_biased_b200.layer import MoELayer
@@ -193,7 +240,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     wall0 = time.perf_counter()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)                       # evict L2 between steps (outside the events)
@@ -236,9 +283,10 @@ def run_ours(args, world, rank, local):
     peaks = load_peaks()
     fp8_peak_tflops = 2.0 * peaks["bf16_tflops"]           # nominal FP8:BF16 dense ratio 2:1
     hbm = peaks["hbm_gbs"]
-    g1_ms = statistics.mean(k[0] for k in kernel_ms)
-    g2_ms = statistics.mean(k[1] for k in kernel_ms)
-    cmb_ms = statistics.mean(k[2] for k in kernel_ms)
+    gat_ms = statistics.mean(k[0] for k in kernel_ms)
+    g1_ms = statistics.mean(k[1] for k in kernel_ms)
+    g2_ms = statistics.mean(k[2] for k in kernel_ms)
+    cmb_ms = statistics.mean(k[3] for k in kernel_ms)
     g1_t_bytes = work["gemm1_bytes"] / hbm / 1e9 * 1e3      # ms at peak HBM
     g1_t_flops = work["gemm1_flops"] / (fp8_peak_tflops * 1e12) * 1e3
     if g1_t_bytes >= g1_t_flops:
@@ -248,13 +296,13 @@ def run_ours(args, world, rank, local):
         roofline = {"kernel": "moe_gate_up_gemm", "bound": "tensor",
                     "achieved": work["gemm1_flops"] / (g1_ms * 1e-3) / 1e12, "peak": fp8_peak_tflops, "unit": "TFLOP/s"}
     roofline["frac"] = roofline["achieved"] / roofline["peak"]
-    roofline["traffic"] = args.traffic
+    roofline["traffic"], roofline["traffic_source"] = gate_up_traffic(cfg.name, args.traffic)
     roofline["peak_source"] = peaks["source"] + (" (fp8 = 2 x bf16)" if roofline["bound"] == "tensor" else "")
     t_layer_roof = max(work["flops"] / (fp8_peak_tflops * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
 
     tokens = cfg.T * world
     result = {
-        "metric": "fused FP8-blockscale MoE layer tokens/s at 1 B200 (TFLOPS and % of FP8/HBM roofline alongside)",
+        "metric": METRIC,
         "value": tokens / (ms_per_step * 1e-3),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -276,8 +324,8 @@ def run_ours(args, world, rank, local):
                            "flops": work["flops"], "bytes": work["layer_bytes"],
                            "touched_experts": work["n_experts"], "fp8_peak_tflops": fp8_peak_tflops,
                            "hbm_gbs": hbm},
-        "kernels_ms": {"moe_gate_up_gemm": g1_ms, "moe_down_gemm": g2_ms, "moe_combine": cmb_ms,
-                       "route_sort_quant": ms_per_step - g1_ms - g2_ms - cmb_ms},
+        "kernels_ms": {"moe_gather": gat_ms, "moe_gate_up_gemm": g1_ms, "moe_down_gemm": g2_ms, "moe_combine": cmb_ms,
+                       "route_sort_quant": ms_per_step - gat_ms - g1_ms - g2_ms - cmb_ms},
         "roofline": roofline,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": act.logits.numel() * 4 + act.x.numel() * 2,
@@ -292,56 +340,78 @@ def run_ours(args, world, rank, local):
     return result
 
 
-def cpu_baseline(cfg, n_tokens, device="cuda"):
-    """The oracle, as it stands, on a seeded sample of the workload's tokens (host cores)."""
-    from oracle import fp8moe_oracle as O
+class OracleSample:
+    """The oracle, as it stands, over a seeded sample of a workload's tokens.
 
-    act = I.moe_activations(cfg)
-    g = torch.Generator().manual_seed(1234)
-    tokens = torch.sort(torch.randperm(cfg.T, generator=g)[:n_tokens]).values
-    # raw expert weights: the same draws the device layer used (generator on `device`), copied to the host
-    w_ref, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
-    experts = torch.unique(ids_ref[tokens]).tolist()
-    raw = {e: (I.expert_weight_raw(cfg, "w1", e, device).cpu(), I.expert_weight_raw(cfg, "w2", e, device).cpu())
-           for e in experts}
-    threads = torch.get_num_threads()
-    t0 = time.perf_counter()
-    w, ids = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
-    a8, asc = O.quant_1x128(act.x[tokens])
+    Setup (untimed, like the device layer's weight loading): the activations are
+    drawn, the sample's experts found and their raw weights, drawn exactly as
+    the device layer draws them (generator on `device`), quantised to FP8 in
+    128x128 blocks. step() then times one pass of the path over the sample:
+    routing, align/sort, 1x128 activation quantisation and the MoE layer with
+    its combine. Every step computes the whole sample from scratch.
+    """
 
-    def get(e):
-        q1, s1 = O.quant_128x128(raw[e][0])
-        q2, s2 = O.quant_128x128(raw[e][1])
-        return q1, s1, q2, s2
+    def __init__(self, cfg, n_tokens, device="cuda"):
+        from oracle import fp8moe_oracle as O
+        self.O, self.cfg = O, cfg
+        act = I.moe_activations(cfg)
+        g = torch.Generator().manual_seed(1234)
+        tok = torch.sort(torch.randperm(cfg.T, generator=g)[:n_tokens]).values
+        self.logits, self.x = act.logits[tok].contiguous(), act.x[tok].contiguous()
+        self.bias = act.bias
+        _, ids = O.biased_grouped_topk(self.logits, self.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+        self.experts = torch.unique(ids).tolist()
+        self.weights = {}
+        for e in self.experts:
+            w1 = I.expert_weight_raw(cfg, "w1", e, device).cpu()
+            w2 = I.expert_weight_raw(cfg, "w2", e, device).cpu()
+            self.weights[e] = (*O.quant_128x128(w1), *O.quant_128x128(w2))
+        self.n = n_tokens
 
-    O.moe_layer(a8, asc, ids[tokens], w[tokens], get)
-    dt = time.perf_counter() - t0
-    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n_tokens} seeded tokens of {cfg.name} (routing on all {cfg.T} tokens, "
-                      f"{len(experts)} experts quantised and applied), {dt:.1f} s"}
+    def step(self):
+        O, cfg = self.O, self.cfg
+        t0 = time.perf_counter()
+        w, ids = O.biased_grouped_topk(self.logits, self.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+        O.align_sort(ids, w, cfg.E, 128)
+        a8, asc = O.quant_1x128(self.x)
+        O.moe_layer(a8, asc, ids, w, self.weights.__getitem__)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, n_tokens, device="cuda", min_seconds=10.0):
+    """The oracle on the host cores: repeated passes over an n-token sample until min_seconds have run."""
+    runner = OracleSample(cfg, n_tokens, device)
+    times = []
+    while sum(times) < min_seconds:
+        times.append(runner.step())
+    sec = sum(times) / len(times)
+    return {"value": n_tokens / sec, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"{n_tokens} seeded tokens of {cfg.name} ({len(runner.experts)} experts, weights quantised "
+                      f"before timing), {len(times)} passes in {sum(times):.1f} s"}
 
 
 def run_reference(args, world, rank):
     cfg = WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    times = []
-    n = args.cpu_sample_tokens
-    for i in range(args.warmup + args.steps):
-        r = cpu_baseline(cfg, n, device=dev)
-        if i >= args.warmup:
-            times.append(n / r["value"])
+    runner = OracleSample(cfg, args.ref_sample_tokens, device=dev)
+    for _ in range(args.warmup):
+        runner.step()
+    times = [runner.step() for _ in range(args.steps)]
     sec = statistics.mean(times)
+    n = args.ref_sample_tokens
     value = n / sec
     return {
         "impl": "reference",
-        "metric": "fused FP8-blockscale MoE layer tokens/s at 1 B200 (TFLOPS and % of FP8/HBM roofline alongside)",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp64 oracle (fp32 where a routing choice or FP8 code is decided)",
+        "dtype": "f64 (fp32 where a routing choice or an FP8 code is decided)",
         "data": "synthetic (seeded)",
-        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "topk": cfg.K, "I": cfg.I},
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "groups": cfg.G,
+                   "topk_group": cfg.TG, "topk": cfg.K, "I": cfg.I},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
-                         "sample": f"{n} seeded tokens of {cfg.name} per step"},
+                         "sample": f"{n} seeded tokens of {cfg.name} per step ({len(runner.experts)} experts, "
+                                   "weights quantised before timing)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -349,13 +419,16 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=2)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=8,
+                    help="tokens of the workload the oracle runs for cpu_baseline")
+    ap.add_argument("--ref-sample-tokens", type=int, default=1,
+                    help="tokens of the workload the oracle runs per step under --impl reference")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the gate/up GEMM from an ncu capture (reported as is)")
     args = ap.parse_args()

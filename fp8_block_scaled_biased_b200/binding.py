@@ -116,8 +116,8 @@ def timing_enable(on: bool = True):
 
 
 def timing_last():
-    """(gate/up GEMM ms, down GEMM ms, combine ms) of the most recent fused MoE call; waits for it."""
-    ms = (ctypes.c_float * 3)()
+    """(gather ms, gate/up GEMM ms, down GEMM ms, combine ms) of the most recent fused MoE call; waits for it."""
+    ms = (ctypes.c_float * 4)()
     _check("fp8moe_timing_last", load_library().fp8moe_timing_last(ms))
     return tuple(ms)
 

@@ -63,11 +63,13 @@ int fp8moe_device_status(void* stream);
 
 /* Measurement hook (not part of the pages' API). While enabled for the calling
  * thread, each fused_moe_fp8_blockscale_g1u1 call records CUDA events on its
- * stream before the gate/up GEMM, after it, after the down GEMM and after the
- * combine. fp8moe_timing_last() waits for the last of those events and writes
- * the three kernel durations of the most recent call in milliseconds
- * (ms[0] gate/up GEMM, ms[1] down GEMM, ms[2] combine). Returns FP8MOE_OK or
- * FP8MOE_ECUDA. Events are created on first use on the current device. */
+ * stream before the slot-order gather, after it, after the gate/up GEMM, after
+ * the down GEMM and after the combine. fp8moe_timing_last() waits for the last
+ * of those events and writes the four kernel durations of the most recent call
+ * in milliseconds (ms[0] gather, ms[1] gate/up GEMM, ms[2] down GEMM,
+ * ms[3] combine; `ms` holds 4 floats). Returns FP8MOE_OK, FP8MOE_EINVAL (null
+ * pointer, timing never enabled) or FP8MOE_ECUDA. Events are created on first
+ * use on the current device. */
 int fp8moe_timing_enable(int on);
 int fp8moe_timing_last(float* ms);
 

@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py, on the CPU: the reference arm's JSON line (one
+rank and two gloo ranks), the traffic table's source check and the algorithmic
+work counts the roofline divides by."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+import bench
+from fp8_block_scaled_biased_b200 import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _json_lines(text):
+    out = []
+    for ln in text.splitlines():
+        ln = ln.strip()
+        if ln.startswith("{"):
+            out.append(json.loads(ln))
+    return out
+
+
+def test_reference_arm_line_on_one_rank():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == I.TINY.name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_two_gloo_ranks_print_one_line():
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", "29541", "bench.py", "--impl", "reference",
+           "--workload", "tiny", "--gpus", "2", "--steps", "1", "--warmup", "1"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_traffic_reported_only_for_unchanged_sources(monkeypatch):
+    sha = bench.gemm_source_sha()
+    monkeypatch.setattr(bench, "GATE_UP_TRAFFIC", {
+        "w_same": {"bytes": 123.0, "sha256": sha, "capture": "c"},
+        "w_old": {"bytes": 456.0, "sha256": "0" * 64, "capture": "c"},
+    })
+    assert bench.gate_up_traffic("w_same", None) == (123.0, "c")
+    assert bench.gate_up_traffic("w_old", None)[0] is None
+    assert bench.gate_up_traffic("w_none", None)[0] is None
+    assert bench.gate_up_traffic("w_old", 7.0) == (7.0, "given on the command line")
+
+
+def test_layer_work_counts():
+    cfg = I.TINY
+    ids = torch.tensor([[0, 1, 2, 3]] * cfg.T, dtype=torch.int32)
+    w = bench.layer_work(cfg, ids)
+    P = cfg.T * cfg.K
+    assert w["n_experts"] == 4
+    assert w["flops"] == 2 * P * cfg.H * 2 * cfg.I + 2 * P * cfg.I * cfg.H
+    assert w["gemm1_flops"] == 2 * P * cfg.H * 2 * cfg.I
+    w1 = 2 * cfg.I * cfg.H + (2 * cfg.I // 128) * (cfg.H // 128) * 4
+    assert w["gemm1_bytes"] == (4 * w1 + cfg.T * cfg.H + cfg.T * (cfg.H // 128) * 4
+                                + P * cfg.I + P * (cfg.I // 128) * 4)
+
+
+@pytest.mark.parametrize("n", [1, 3])
+def test_oracle_sample_step_is_repeatable(n):
+    r = bench.OracleSample(I.TINY, n, device="cpu")
+    assert r.step() > 0 and r.step() > 0
+    assert len(r.experts) >= 1 and set(r.weights) == set(r.experts)
