@@ -172,7 +172,7 @@ MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I
   w.s1s_off = take(static_cast<size_t>(H / 128) * capacity * sizeof(float));
   w.a2_off = take(capacity * static_cast<size_t>(I));
   w.s2_off = take(static_cast<size_t>(I / 128) * capacity * sizeof(float));
-  w.y_off = take(static_cast<size_t>(T) * topk * H * sizeof(float));
+  w.y_off = take(static_cast<size_t>(T) * topk * H * sizeof(__nv_bfloat16));
   w.total = off;
   return w;
 }
@@ -180,7 +180,7 @@ MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I
 struct TimingState {
   bool on = false;
   int dev = -1;
-  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 };
 thread_local TimingState g_timing;
 
@@ -232,9 +232,9 @@ int fp8moe_timing_enable(int on) {
 
 int fp8moe_timing_last(float* ms) {
   if (!ms) return fail(FP8MOE_EINVAL, "null pointer argument");
-  if (!g_timing.ev[3]) return fail(FP8MOE_EINVAL, "timing was never enabled");
-  cudaError_t e = cudaEventSynchronize(g_timing.ev[3]);
-  for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&ms[i], g_timing.ev[i], g_timing.ev[i + 1]);
+  if (!g_timing.ev[4]) return fail(FP8MOE_EINVAL, "timing was never enabled");
+  cudaError_t e = cudaEventSynchronize(g_timing.ev[4]);
+  for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&ms[i], g_timing.ev[i], g_timing.ev[i + 1]);
   if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "timing read: %s", cudaGetErrorString(e));
   return FP8MOE_OK;
 }
@@ -454,7 +454,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   float* s1s = reinterpret_cast<float*>(ws + lay.s1s_off);
   uint8_t* a2 = ws + lay.a2_off;
   float* s2 = reinterpret_cast<float*>(ws + lay.s2_off);
-  float* ystage = reinterpret_cast<float*>(ws + lay.y_off);
+  __nv_bfloat16* ystage = reinterpret_cast<__nv_bfloat16*>(ws + lay.y_off);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   CUtensorMap m_a8s, m_w1, m_a2, m_w2;
@@ -467,6 +467,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, num_valid_ids, T, topk, H,
                                                             static_cast<int>(capacity), a8s, s1s);
   if (int rc = check_launch("fused_moe (gather)")) return rc;
+  timing_record(1, st);
 
   GemmArgs up{};
   up.M = static_cast<int>(capacity);
@@ -493,7 +494,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (int rc = check_gemm_launch("fused_moe (gate/up GEMM)", blockscale_gemm_kernel<kModeMoeUp>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
-  timing_record(1, st);
+  timing_record(2, st);
 
   GemmArgs dn = up;
   dn.N = H;
@@ -510,13 +511,13 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (int rc = check_gemm_launch("fused_moe (down GEMM)", blockscale_gemm_kernel<kModeMoeDown>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
-  timing_record(2, st);
+  timing_record(3, st);
 
   const size_t threads = static_cast<size_t>(T) * (H / 8);
   moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
       ystage, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
   if (int rc = check_launch("fused_moe (combine)")) return rc;
-  timing_record(3, st);
+  timing_record(4, st);
   return FP8MOE_OK;
 }
 

@@ -76,7 +76,7 @@ struct GemmArgs {
   int b_rows_per_expert;  // up: 2I; down: H
   uint8_t* a2;            // up output [M, I] (slot-ordered FP8 intermediate)
   float* s2;              // up output [I/128, M]
-  float* ystage;          // down output [T*topk, H] (weighted rows by pair id)
+  __nv_bfloat16* ystage;  // down output [T*topk, H] (weighted rows by pair id, bf16)
 };
 
 struct GemmSmem {
@@ -298,24 +298,29 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         }
         if (half == 0) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
       } else {
-        // 512 bytes of fp32 per row: a transpose through the warp's staging buffer
+        // 256 bytes of bf16 per row: a transpose through the warp's staging buffer
         // lets each store instruction write 8 whole 64-byte row segments
         const bool valid = pair >= 0 && pair < P;
         if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
         const int x0 = nt * kBN + half * 128;
         if (x0 < args.N) {
           const int H = args.N;
-          float* y = args.ystage;
+          __nv_bfloat16* y = args.ystage;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {      // 8 chunks of 16 fp32 columns
+          for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
             uint4 d[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              d[u] = make_uint4(__float_as_uint(wroute * acc[ch * 16 + 4 * u]),
-                                __float_as_uint(wroute * acc[ch * 16 + 4 * u + 1]),
-                                __float_as_uint(wroute * acc[ch * 16 + 4 * u + 2]),
-                                __float_as_uint(wroute * acc[ch * 16 + 4 * u + 3]));
-            const int x = x0 + ch * 16;
+            for (int u = 0; u < 4; ++u) {
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int j = ch * 32 + u * 8 + 2 * q;
+                const __nv_bfloat162 pk = __floats2bfloat162_rn(wroute * acc[j], wroute * acc[j + 1]);
+                w[q] = *reinterpret_cast<const uint32_t*>(&pk);
+              }
+              d[u] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            const int x = x0 + ch * 32;
             store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
               const int pr = __shfl_sync(0xffffffffu, pair, r);
               return (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x)
@@ -535,25 +540,26 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
 // out[t, :] = bf16( y[t*K + 0] + y[t*K + 1] + ... + y[t*K + K-1] ), fp32 adds in
 // slot order k (the routing weight is already in y). One thread per 8 columns.
 __global__ void __launch_bounds__(256)
-moe_combine_kernel(const float* __restrict__ ystage, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
+moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
   const int cpr = H / 8;
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<size_t>(T) * cpr) return;
   const int t = static_cast<int>(idx / cpr);
   const int c = static_cast<int>(idx % cpr) * 8;
-  const float* y = ystage + static_cast<size_t>(t) * K * H + c;
+  const __nv_bfloat16* y = ystage + static_cast<size_t>(t) * K * H + c;
   float sum[8];
-  {
-    const float4 a = *reinterpret_cast<const float4*>(y);
-    const float4 b = *reinterpret_cast<const float4*>(y + 4);
-    sum[0] = a.x; sum[1] = a.y; sum[2] = a.z; sum[3] = a.w;
-    sum[4] = b.x; sum[5] = b.y; sum[6] = b.z; sum[7] = b.w;
-  }
-  for (int k = 1; k < K; ++k) {
-    const float4 a = *reinterpret_cast<const float4*>(y + static_cast<size_t>(k) * H);
-    const float4 b = *reinterpret_cast<const float4*>(y + static_cast<size_t>(k) * H + 4);
-    sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
-    sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
+  // fp32 sum in k order (0.0f + y0 == y0 exactly, so the order is fixed from the first term)
+  for (int k = 0; k < K; ++k) {
+    const uint4 v = *reinterpret_cast<const uint4*>(y + static_cast<size_t>(k) * H);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+      sum[2 * u] += f.x;
+      sum[2 * u + 1] += f.y;
+    }
   }
   __align__(16) __nv_bfloat162 pk[4];
 #pragma unroll

@@ -199,8 +199,9 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B,
  *   g = blockscale(a8[t], w1[e]) (fp32), h = silu(g[:I]) * g[I:],
  *   a2 = 1x128 FP8 quantisation of h (as fp8_per_token_group_quant),
  *   y_p = blockscale(a2, w2[e]),
- *   out[t] = bf16( sum_{k=0..topk-1} w_{t,k} * y_{t,k} ) summed in slot order,
- * which makes the output independent of scheduling (deterministic).
+ *   out[t] = bf16( sum_{k=0..topk-1} bf16(w_{t,k} * y_{t,k}) ), each weighted
+ * row rounded once to bf16 and the topk rows summed in fp32 in k order, which
+ * makes the output independent of scheduling (deterministic).
  * Limits: scale_blk_n == scale_blk_k == 128; H % 128 == 0; I % 128 == 0;
  * fc2_smooth_scale must be NULL (the pages do not define it); workspace >=
  * fused_moe_fp8_blockscale_g1u1_workspace(); capacity >= the sort's padded

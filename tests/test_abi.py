@@ -38,7 +38,7 @@ def test_capacity_and_workspace_formulas(lib):
     assert lib.moe_align_sort_capacity(16, 4, 16, 1) == 64
     cap = 64 * 8 + 256 * 127
     need = lib.fused_moe_fp8_blockscale_g1u1_workspace(64, 8, 256, 7168, 2048, 128)
-    assert need >= cap * 2048 + 16 * cap * 4 + 64 * 8 * 7168 * 4
+    assert need >= cap * 7168 + 56 * cap * 4 + cap * 2048 + 16 * cap * 4 + 64 * 8 * 7168 * 2
     assert lib.fp8moe_moe_block_m() == 128
 
 

@@ -229,3 +229,24 @@ def test_fused_moe_full_size_sampled_tokens(big_layer, cfg, n_sample):
     assert_moe_close(out.cpu()[tokens], ref)
     out2 = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
     assert torch.equal(out, out2)
+
+
+def test_timing_hook_reports_each_fused_kernel():
+    """The measurement hook times gather, gate/up GEMM, down GEMM and combine of the latest call."""
+    cfg = MID
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    act = I.moe_activations(cfg)
+    args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    layer.forward(*args)
+    B.timing_enable(True)
+    try:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        layer.forward(*args)
+        end.record()
+        ms = B.timing_last()
+        torch.cuda.synchronize()
+    finally:
+        B.timing_enable(False)
+    assert len(ms) == 4 and all(m > 0 for m in ms), ms
+    assert sum(ms) <= start.elapsed_time(end) * 1.05 + 0.01
