@@ -54,6 +54,7 @@ constexpr int kStageB = kBN * kBK;
 constexpr int kStagingBytes = 32 * 64;        // per epilogue warp: 32 rows x 64 bytes
 constexpr uint32_t kTmemCols = 512;           // two 256-column partial buffers
 constexpr uint32_t kIdesc = umma_idesc_e4m3_f32(kBM, kBN);
+constexpr uint32_t kIdescHalf = umma_idesc_e4m3_f32(kBM / 2, kBN);   // M=64: tiles with <= 64 occupied rows
 
 struct GemmArgs {
   int M;                  // dense: rows of A; MoE: capacity (sorted slots)
@@ -125,6 +126,16 @@ __device__ __forceinline__ int moe_expert(const GemmArgs& a, int mb) {
   return e;
 }
 
+// MoE tile whose second half holds only padding slots (an expert's last block
+// with at most 64 pairs): its MMAs run with M=64. The sort puts an expert's
+// pairs before its padding, so slot 64 of the block decides.
+template <int MODE>
+__device__ __forceinline__ bool moe_half_tile(const GemmArgs& a, int mb, int P) {
+  if (MODE == kModeDense) return false;
+  const int id = a.sorted_ids[mb * kBM + kBM / 2];
+  return id < 0 || id >= P;
+}
+
 __device__ __forceinline__ void abort_all(GemmSmem* s) {
   if (!s->abort) raise_device_error(FP8MOE_DEVERR_TIMEOUT);
   s->abort = 1;
@@ -177,20 +188,27 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
       int mb, nt;
       tile_coords(tile, m_blocks, args.n_tiles, args.group_m, mb, nt);
-      const int slot = mb * kBM + row;
-      int pair = 0;
+      // An M=64 tile keeps its row r in TMEM lane (r % 16) + 32 * (r / 16): lanes
+      // 0..15 of each warp hold rows 16*quarter + lane, lanes 16..31 hold none.
+      const bool m64 = moe_half_tile<MODE>(args, mb, P);
+      const int trow = m64 ? (lane < 16 ? quarter * 16 + lane : -1) : row;
+      const bool has_row = trow >= 0;
+      const int slot = mb * kBM + (has_row ? trow : 0);
+      int pair = P;
       float wroute = 0.0f;
-      if (MODE != kModeDense) {                 // needed only at the end: load early
+      if (MODE != kModeDense && has_row) {      // needed only at the end: load early
         pair = args.sorted_ids[slot];
         if (MODE == kModeMoeDown) wroute = args.sorted_weights[slot];
       }
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      // a warp whose 32 rows are all padding skips the promotion (its outputs are never stored)
+      const bool warp_active = MODE == kModeDense || __any_sync(0xffffffffu, pair >= 0 && pair < P);
 
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&s->sfull[sslot], scphase, abort_flag)) { ok = false; break; }
-        const float sa = s->sa[sslot][row];
+        const float sa = s->sa[sslot][has_row ? trow : 0];
         const float swa = s->sw[sslot][0], swb = s->sw[sslot][1];
         __syncwarp();
         if (lane == 0) mbar_arrive(&s->sempty[sslot]);
@@ -205,6 +223,13 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
 
         if (!mbar_wait(&s->tfull[buf], tphase, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        if (!warp_active) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s->tempty[buf]);
+          if (++buf == 2) { buf = 0; tphase ^= 1u; }
+          continue;
+        }
         const uint32_t tb = lane_base + buf * kBN;
         // four 32-column chunks; the load of chunk c+1 overlaps the FMAs of chunk c
         float v[2][32];
@@ -296,7 +321,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
             st_global_v8(dst + ch * 32, w);
           }
         }
-        if (half == 0) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
+        if (half == 0 && has_row) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
       } else {
         // 256 bytes of bf16 per row: a transpose through the warp's staging buffer
         // lets each store instruction write 8 whole 64-byte row segments
@@ -467,6 +492,9 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         uint32_t sphase = 0, tphase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+          int mb, nt;
+          tile_coords(tile, m_blocks, args.n_tiles, args.group_m, mb, nt);
+          const uint32_t idesc = moe_half_tile<MODE>(args, mb, P) ? kIdescHalf : kIdesc;
           for (int kb = 0; kb < num_kb; ++kb) {
             if (!mbar_wait(&s->full[stage], sphase, abort_flag)) { ok = false; break; }
             if (!mbar_wait(&s->tempty[buf], tphase ^ 1u, abort_flag)) { ok = false; break; }
@@ -476,7 +504,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const uint32_t d_tmem = tmem_base + buf * kBN;
 #pragma unroll
             for (int k = 0; k < kBK / kUmmaK; ++k)
-              umma_f8(d_tmem, umma_desc_sw128(a_addr + k * kUmmaK), umma_desc_sw128(b_addr + k * kUmmaK), kIdesc,
+              umma_f8(d_tmem, umma_desc_sw128(a_addr + k * kUmmaK), umma_desc_sw128(b_addr + k * kUmmaK), idesc,
                       k > 0 ? 1u : 0u);
             umma_commit(&s->empty[stage]);
             umma_commit(&s->tfull[buf]);
