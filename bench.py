@@ -175,7 +175,15 @@ def layer_work(cfg, ids):
 # launch from a one-pass ncu capture of this bench's own command, keyed by
 # workload, with the SHA-256 of the GEMM kernel sources the capture ran. A
 # figure whose sources have changed since is not reported.
-GATE_UP_TRAFFIC = {}
+GATE_UP_TRAFFIC = {
+    "prefill_t4096_h7168_e256": {
+        "bytes": 7.072e9,
+        "sha256": "03cdf80666cd5b10c7062d3d1c719ace32434e1badaf8143ffa30a28d5ffc7c6",
+        "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
+                   "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean; "
+                   "profiles/launches_prefill_t4096.md)",
+    },
+}
 GEMM_SOURCES = ("fp8_block_scaled_biased_b200/csrc/gemm_sm100.cuh", "fp8_block_scaled_biased_b200/csrc/common.cuh")
 
 
@@ -324,6 +332,7 @@ def run_ours(args, world, rank, local):
                            "flops": work["flops"], "bytes": work["layer_bytes"],
                            "touched_experts": work["n_experts"], "fp8_peak_tflops": fp8_peak_tflops,
                            "hbm_gbs": hbm},
+        "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
         "kernels_ms": {"moe_gather": gat_ms, "moe_gate_up_gemm": g1_ms, "moe_down_gemm": g2_ms, "moe_combine": cmb_ms,
                        "route_sort_quant": ms_per_step - gat_ms - g1_ms - g2_ms - cmb_ms},
         "roofline": roofline,
@@ -390,7 +399,130 @@ def cpu_baseline(cfg, n_tokens, device="cuda", min_seconds=10.0):
                       f"before timing), {len(times)} passes in {sum(times):.1f} s"}
 
 
+def run_gemm(args, world, rank, local):
+    """The standalone block-scale GEMM (C = A . B^T with 1x128 / 128x128 FP8 scales), A pre-quantised."""
+    from fp8_block_scaled_biased_b200 import binding as B
+
+    cfg = I.GEMM
+    dev = torch.device("cuda", local)
+    a, b = I.gemm_inputs(cfg, device=dev)
+    qa, sa = B.fp8_per_token_group_quant(a, 128)
+    qb, sb = B.fp8_per_block_quant(b)
+    c = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        B.fp8_blockscale_gemm(qa, qb, sa, sb, out=c)
+    torch.cuda.synchronize()
+
+    def timed(flush_l2):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            if flush_l2:
+                flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            B.fp8_blockscale_gemm(qa, qb, sa, sb, out=c)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = [x.elapsed_time(y) for x, y in ev]
+        return max_over_ranks(sum(ms), world) / args.steps, ms
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    ms_flushed, per_step = timed(True)
+    clocks = sampler.stop()
+    ms_warm, _ = timed(False)
+    if B.device_status():
+        raise RuntimeError("device error word set by the GEMM")
+
+    # end to end: pinned host A (FP8 codes + scales) in, bf16 C out
+    h_qa, h_sa = qa.cpu().pin_memory(), sa.cpu().pin_memory()
+    h_c = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16).pin_memory()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0[i].record(stream)
+        qa.copy_(h_qa, non_blocking=True)
+        sa.copy_(h_sa, non_blocking=True)
+        B.fp8_blockscale_gemm(qa, qb, sa, sb, out=c)
+        h_c.copy_(c, non_blocking=True)
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(x.elapsed_time(y) for x, y in zip(e0, e1)), world) / args.steps
+
+    flops = 2.0 * cfg.M * cfg.N * cfg.K
+    peaks = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    tf = flops * world / (ms_flushed * 1e-3) / 1e12
+    result = {
+        "metric": "FP8 block-scale GEMM TFLOP/s at 1 B200 (C = A.B^T, 1x128 / 128x128 fp32 scales, bf16 out)",
+        "value": tf, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_flushed, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3fn x fp8_e4m3fn -> fp32 accumulate, bf16 out", "data": "synthetic (seeded)",
+        "config": {"workload": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K,
+                   "l2": "flushed between steps (256 MB write)", "parallelism": f"dp{world} (independent GEMMs)"},
+        "l2_warm": {"ms_per_step": ms_warm, "tflops": flops / (ms_warm * 1e-3) / 1e12},
+        "step_ms": {"median": statistics.median(per_step), "min": min(per_step), "max": max(per_step)},
+        "roofline": {"kernel": "fp8_blockscale_gemm", "bound": "tensor", "achieved": flops / (ms_flushed * 1e-3) / 1e12,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": flops / (ms_flushed * 1e-3) / 1e12 / fp8_peak,
+                     "traffic": None, "peak_source": peaks["source"] + " (fp8 = 2 x bf16)"},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": qa.numel() + sa.numel() * 4, "d2h_bytes_per_step": c.numel() * 2},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import fp8moe_oracle as O
+        rows = torch.arange(0, cfg.M, cfg.M // 8)
+        qa_h, sa_h = O.quant_1x128(a[rows].cpu())
+        qb_h, sb_h = O.quant_128x128(b.cpu())
+        t0 = time.perf_counter()
+        O.blockscale_gemm(qa_h, sa_h, qb_h, sb_h)
+        dt = time.perf_counter() - t0
+        result["cpu_baseline"] = {"value": 2.0 * len(rows) * cfg.N * cfg.K / dt / 1e12, "unit": "TFLOP/s",
+                                  "cores": torch.get_num_threads(), "kind": "oracle",
+                                  "sample": f"{len(rows)} of {cfg.M} rows, operands quantised before timing, {dt:.1f} s"}
+    return result
+
+
+def run_reference_gemm(args, world):
+    """The oracle's block-scale GEMM on a fixed sample of 8 rows of A per step (operands quantised before timing)."""
+    from oracle import fp8moe_oracle as O
+    cfg = I.GEMM
+    a, b = I.gemm_inputs(cfg, device="cpu")
+    rows = torch.arange(0, cfg.M, cfg.M // 8)
+    qa, sa = O.quant_1x128(a[rows])
+    qb, sb = O.quant_128x128(b)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        O.blockscale_gemm(qa, sa, qb, sb)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = statistics.mean(times)
+    value = 2.0 * len(rows) * cfg.N * cfg.K / sec / 1e12
+    return {
+        "impl": "reference",
+        "metric": "FP8 block-scale GEMM TFLOP/s at 1 B200 (C = A.B^T, 1x128 / 128x128 fp32 scales, bf16 out)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": f"{len(rows)} of {cfg.M} rows of A per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, world, rank):
+    if args.workload == "gemm":
+        return run_reference_gemm(args, world)
     cfg = WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     runner = OracleSample(cfg, args.ref_sample_tokens, device=dev)
@@ -421,7 +553,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["gemm"], default="prefill",
+                    help="MoE layer workload, or gemm: the standalone block-scale GEMM (M=2048, N=4096, K=7168)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -440,7 +573,7 @@ def main():
             if rank == 0:
                 print(json.dumps(run_reference(args, world, rank)), flush=True)
         else:
-            res = run_ours(args, world, rank, local)
+            res = run_gemm(args, world, rank, local) if args.workload == "gemm" else run_ours(args, world, rank, local)
             if rank == 0:
                 print(json.dumps(res), flush=True)
     finally:

@@ -81,3 +81,12 @@ def test_oracle_sample_step_is_repeatable(n):
     r = bench.OracleSample(I.TINY, n, device="cpu")
     assert r.step() > 0 and r.step() > 0
     assert len(r.experts) >= 1 and set(r.weights) == set(r.experts)
+
+
+def test_reference_arm_gemm_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "gemm",
+                        "--steps", "1", "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = _json_lines(r.stdout)[-1]
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["config"]["workload"] == I.GEMM.name
