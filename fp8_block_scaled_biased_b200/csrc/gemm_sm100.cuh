@@ -599,8 +599,17 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
         if (v < vec_per_row) dst[v] = buf[i];
       }
     }
-    for (int kb = lane; kb < KB; kb += 32)
-      s1s[static_cast<size_t>(kb) * cap + slot] = a1_scale[static_cast<size_t>(kb) * T + t];
+  }
+  // scales: one lane per slot of a 32-slot group, so each store instruction
+  // writes 128 contiguous bytes of a row of s1s
+  const int nwarps = gridDim.x * kGatherWarps;
+  for (int s0 = (blockIdx.x * kGatherWarps + (threadIdx.x >> 5)) * 32; s0 < nv; s0 += nwarps * 32) {
+    const int slot = s0 + lane;
+    const int sid = slot < nv ? sorted_ids[slot] : -1;
+    if (sid < 0 || sid >= P) continue;
+    const int t = sid / topk;
+    for (int kb = 0; kb < KB; ++kb)
+      s1s[static_cast<size_t>(kb) * cap + slot] = __ldg(a1_scale + static_cast<size_t>(kb) * T + t);
   }
 }
 

@@ -32,7 +32,10 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float scale) {
 }
 
 // One warp per row; each half-warp (16 lanes x 8 bf16) covers one 128-wide group.
-// K % 8 == 0; a last group shorter than 128 uses its valid elements.
+// K % 8 == 0; a last group shorter than 128 uses its valid elements. Each lane
+// issues the loads of kQuantUnroll groups before using them, so a row costs
+// one memory round trip per 2 * kQuantUnroll groups.
+constexpr int kQuantUnroll = 4;
 __global__ void __launch_bounds__(32 * kQuantWarps)
 quant_1x128_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, int M, int K, uint8_t* __restrict__ q,
                    float* __restrict__ scales, int col_major) {
@@ -42,36 +45,40 @@ quant_1x128_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, int M, int K, 
   const int half = lane >> 4, hl = lane & 15;
   const int KB = (K + 127) / 128;
   const __nv_bfloat16* row = x + static_cast<size_t>(m) * ld_x;
-  for (int g0 = 0; g0 < KB; g0 += 2) {
-    const int g = g0 + half;
-    const int col = g * 128 + hl * 8;
-    float v[8];
-    const bool in = (g < KB) && (col < K);
-    if (in) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(row + col);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  for (int g0 = 0; g0 < KB; g0 += 2 * kQuantUnroll) {
+    uint4 raw[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int g = g0 + 2 * u + half;
+      const int col = g * 128 + hl * 8;
+      raw[u] = (g < KB && col < K) ? __ldg(reinterpret_cast<const uint4*>(row + col)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int g = g0 + 2 * u + half;
+      const int col = g * 128 + hl * 8;
+      const bool in = (g < KB) && (col < K);
+      float v[8];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 f = __bfloat1622float2(h2[i]);
         v[2 * i] = f.x;
         v[2 * i + 1] = f.y;
       }
-    } else {
+      float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-    }
-    float amax = 0.0f;
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float scale = __fdiv_rn(amax, kFp8Max);
-    if (in) *reinterpret_cast<uint2*>(q + static_cast<size_t>(m) * K + col) = quant8(v, scale);
-    if (g < KB && hl == 0) {
-      if (col_major)
-        scales[static_cast<size_t>(g) * M + m] = scale;
-      else
-        scales[static_cast<size_t>(m) * KB + g] = scale;
+      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const float scale = __fdiv_rn(amax, kFp8Max);
+      if (in) *reinterpret_cast<uint2*>(q + static_cast<size_t>(m) * K + col) = quant8(v, scale);
+      if (g < KB && hl == 0) {
+        if (col_major)
+          scales[static_cast<size_t>(g) * M + m] = scale;
+        else
+          scales[static_cast<size_t>(m) * KB + g] = scale;
+      }
     }
   }
 }
