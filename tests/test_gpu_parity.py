@@ -196,7 +196,15 @@ MID = I.MoEConfig("mid_t256_h1024_e32", T=256, H=1024, E=32, G=4, TG=2, K=4, I=5
 SKEW_SMALL = I.MoEConfig("skew_t512_h512_e64", T=512, H=512, E=64, G=8, TG=4, K=8, I=256, hot_experts=4, seed=2)
 
 
-@pytest.mark.parametrize("cfg", [I.TINY, MID, SKEW_SMALL], ids=lambda c: c.name)
+# Odd shapes: one token and one expert with H % 256 == 128 (the down GEMM's last column
+# tile is half valid) and a single I block; E not a power of two with topk 5 and a ragged T;
+# few experts, so each holds several row blocks (multi-block groups, M=64 tails).
+ODD_ONE = I.MoEConfig("odd_t1_h384_e8_k1", T=1, H=384, E=8, G=1, TG=1, K=1, I=128, renorm=False, scale=1.0, seed=3)
+ODD_E24 = I.MoEConfig("odd_t37_h640_e24_k5", T=37, H=640, E=24, G=4, TG=3, K=5, I=384, seed=4)
+FEW_EXPERTS = I.MoEConfig("few_t300_h256_e6_k2", T=300, H=256, E=6, G=2, TG=1, K=2, I=256, seed=5)
+
+
+@pytest.mark.parametrize("cfg", [I.TINY, MID, SKEW_SMALL, ODD_ONE, ODD_E24, FEW_EXPERTS], ids=lambda c: c.name)
 def test_fused_moe_full_small_layers(cfg):
     layer = MoELayer(cfg, DEV).load_synthetic_weights()
     act = I.moe_activations(cfg)
@@ -250,3 +258,16 @@ def test_timing_hook_reports_each_fused_kernel():
         B.timing_enable(False)
     assert len(ms) == 4 and all(m > 0 for m in ms), ms
     assert sum(ms) <= start.elapsed_time(end) * 1.05 + 0.01
+
+
+def test_fused_moe_zero_tokens_is_a_no_op():
+    cfg = I.TINY
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    out = torch.full((0, cfg.H), 7.0, dtype=torch.bfloat16, device=DEV)
+    a8 = torch.empty(0, cfg.H, dtype=torch.float8_e4m3fn, device=DEV)
+    a1 = torch.empty(cfg.H // 128, 0, dtype=torch.float32, device=DEV)
+    sorted_pairs = B.alloc_sorted(0, cfg.K, cfg.E, layer.block_m, DEV)
+    B.fused_moe_fp8_blockscale_g1u1(out, a8, layer.w1, layer.w2, sorted_pairs, cfg.K, a1, layer.w1_scale,
+                                    layer.w2_scale)
+    torch.cuda.synchronize()
+    assert out.numel() == 0
