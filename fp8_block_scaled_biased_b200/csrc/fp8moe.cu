@@ -359,7 +359,9 @@ int fp8_per_token_group_quant(const uint16_t* x, int ld_x, int M, int K, int gro
   if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7u)) return fail(FP8MOE_EINVAL, "x must be 16-byte and q 8-byte aligned");
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
-  const dim3 grid((M + kQuantWarps - 1) / kQuantWarps);
+  const long long warps = static_cast<long long>(M) * ((K + 128 * kQuantSpan - 1) / (128 * kQuantSpan));
+  if ((warps + kQuantWarps - 1) / kQuantWarps >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "M too large");
+  const dim3 grid(static_cast<unsigned>((warps + kQuantWarps - 1) / kQuantWarps));
   quant_1x128_kernel<<<grid, 32 * kQuantWarps, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), ld_x, M, K, q, scales, scale_layout == FP8MOE_SCALE_COL_MAJOR);
   return check_launch("fp8_per_token_group_quant");

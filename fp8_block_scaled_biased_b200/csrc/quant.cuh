@@ -31,21 +31,25 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float scale) {
   return make_uint2(lo, hi);
 }
 
-// One warp per row; each half-warp (16 lanes x 8 bf16) covers one 128-wide group.
-// K % 8 == 0; a last group shorter than 128 uses its valid elements. Each lane
-// issues the loads of kQuantUnroll groups before using them, so a row costs
-// one memory round trip per 2 * kQuantUnroll groups.
+// One warp per (row, span of 2 * kQuantUnroll groups); each half-warp (16 lanes
+// x 8 bf16) covers one 128-wide group. K % 8 == 0; a last group shorter than
+// 128 uses its valid elements. Each lane issues the loads of its kQuantUnroll
+// groups before using them, so a warp costs one memory round trip.
 constexpr int kQuantUnroll = 4;
+constexpr int kQuantSpan = 2 * kQuantUnroll;     // groups per warp
 __global__ void __launch_bounds__(32 * kQuantWarps)
 quant_1x128_kernel(const __nv_bfloat16* __restrict__ x, int ld_x, int M, int K, uint8_t* __restrict__ q,
                    float* __restrict__ scales, int col_major) {
   const int lane = threadIdx.x & 31;
-  const int m = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
-  if (m >= M) return;
-  const int half = lane >> 4, hl = lane & 15;
   const int KB = (K + 127) / 128;
+  const int spans = (KB + kQuantSpan - 1) / kQuantSpan;
+  const long long w = static_cast<long long>(blockIdx.x) * kQuantWarps + (threadIdx.x >> 5);
+  if (w >= static_cast<long long>(M) * spans) return;
+  const int m = static_cast<int>(w / spans);
+  const int half = lane >> 4, hl = lane & 15;
   const __nv_bfloat16* row = x + static_cast<size_t>(m) * ld_x;
-  for (int g0 = 0; g0 < KB; g0 += 2 * kQuantUnroll) {
+  {
+    const int g0 = static_cast<int>(w % spans) * kQuantSpan;
     uint4 raw[kQuantUnroll];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
