@@ -288,9 +288,20 @@ int moe_biased_grouped_topk(const float* gating_output, int ld_in, const float* 
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
   const dim3 grid((T + kRouteWarps - 1) / kRouteWarps);
-  route_kernel<<<grid, 32 * kRouteWarps, 0, static_cast<cudaStream_t>(stream)>>>(
-      gating_output, ld_in, correction_bias, topk_weights, topk_ids, ld_out, T, E, topk, num_expert_group,
-      topk_group, need_renorm ? 1 : 0, routed_scaling_factor, per_lane);
+  const int vec4 = (ld_in % 4 == 0) && aligned16(gating_output) && aligned16(correction_bias);
+  auto launch = [&](auto kernel) {
+    kernel<<<grid, 32 * kRouteWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+        gating_output, ld_in, correction_bias, topk_weights, topk_ids, ld_out, T, E, topk, num_expert_group,
+        topk_group, need_renorm ? 1 : 0, routed_scaling_factor, per_lane, vec4);
+  };
+  switch (per_lane) {
+    case 1: launch(route_kernel<1>); break;
+    case 2: launch(route_kernel<2>); break;
+    case 4: launch(route_kernel<4>); break;
+    case 8: launch(route_kernel<8>); break;
+    case 16: launch(route_kernel<16>); break;
+    default: launch(route_kernel<0>); break;
+  }
   return check_launch("moe_biased_grouped_topk");
 }
 

@@ -47,11 +47,16 @@ __device__ __forceinline__ bool ranks_before(float v1, int i1, float v0, int i0)
 
 // Each lane owns `per_lane` consecutive experts; a lane's experts never span two
 // groups (per_lane divides the group size), so a group is lanes_per_group
-// consecutive lanes.
+// consecutive lanes. PL > 0 fixes per_lane at compile time (the usual 1, 2, 4,
+// 8, 16); PL == 0 takes it from the argument. vec4: rows and bias allow 16-byte
+// loads of a lane's experts (PL % 4 == 0 only).
+template <int PL>
 __global__ void __launch_bounds__(32 * kRouteWarps)
 route_kernel(const float* __restrict__ logits, int ld_in, const float* __restrict__ bias,
              float* __restrict__ topk_w, int32_t* __restrict__ topk_ids, int ld_out, int T, int E, int K,
-             int G, int TG, int renorm, float factor, int per_lane) {
+             int G, int TG, int renorm, float factor, int per_lane_arg, int vec4) {
+  constexpr int kPL = PL > 0 ? PL : kRouteMaxPerLane;
+  const int per_lane = PL > 0 ? PL : per_lane_arg;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -59,14 +64,31 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
   const int lanes_per_group = per_group / per_lane;
   const int e0 = lane * per_lane;
 
-  float s[kRouteMaxPerLane], b[kRouteMaxPerLane];
+  float s[kPL], b[kPL];
   const float* row = logits + static_cast<size_t>(t) * ld_in;
+  float x[kPL], bs[kPL];
+  if (PL % 4 == 0 && PL > 0 && vec4 && e0 < E) {
 #pragma unroll
-  for (int j = 0; j < kRouteMaxPerLane; ++j) {
-    const int e = e0 + j;
-    if (j < per_lane && e < E) {
-      s[j] = sigmoid_f32_recipe(row[e]);
-      b[j] = __fadd_rn(s[j], bias[e]);
+    for (int j = 0; j < kPL; j += 4) {
+      const float4 xv = __ldg(reinterpret_cast<const float4*>(row + e0 + j));
+      const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + e0 + j));
+      x[j] = xv.x; x[j + 1] = xv.y; x[j + 2] = xv.z; x[j + 3] = xv.w;
+      bs[j] = bv.x; bs[j + 1] = bv.y; bs[j + 2] = bv.z; bs[j + 3] = bv.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPL; ++j) {
+      const int e = e0 + j;
+      const bool in = j < per_lane && e < E;
+      x[j] = in ? __ldg(row + e) : 0.0f;
+      bs[j] = in ? __ldg(bias + e) : 0.0f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kPL; ++j) {
+    if (j < per_lane && e0 + j < E) {
+      s[j] = sigmoid_f32_recipe(x[j]);
+      b[j] = __fadd_rn(s[j], bs[j]);
     } else {
       s[j] = 0.0f;
       b[j] = -INFINITY;
@@ -77,7 +99,7 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
   // not depend on which index holds a tied value).
   float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < kRouteMaxPerLane; ++j) {
+  for (int j = 0; j < kPL; ++j) {
     if (j < per_lane) {
       if (b[j] > t1) {
         t2 = t1;
@@ -117,7 +139,7 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
   const int my_group = (e0 < E) ? e0 / per_group : 0;
   const bool my_group_kept = (e0 < E) && ((gmask >> my_group) & 1u);
 #pragma unroll
-  for (int j = 0; j < kRouteMaxPerLane; ++j)
+  for (int j = 0; j < kPL; ++j)
     if (!my_group_kept) b[j] = -INFINITY;
 
   // Top-k by repeated warp argmax over (b desc, index asc).
@@ -127,7 +149,7 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < kRouteMaxPerLane; ++j) {
+    for (int j = 0; j < kPL; ++j) {
       if (j < per_lane && (e0 + j) < E && ranks_before(b[j], e0 + j, bv, bi)) {
         bv = b[j];
         bi = e0 + j;
@@ -146,7 +168,7 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
     const int owner = bi / per_lane;
     float sw = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kRouteMaxPerLane; ++j) {
+    for (int j = 0; j < kPL; ++j) {
       if (lane == owner && e0 + j == bi) {
         sw = s[j];
         b[j] = -INFINITY;
