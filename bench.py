@@ -188,11 +188,12 @@ GEMM_SOURCES = ("fp8_block_scaled_biased_b200/csrc/gemm_sm100.cuh", "fp8_block_s
 
 
 def gemm_source_sha():
+    """SHA-256 of the GEMM kernel sources with all whitespace removed (layout-only edits keep it)."""
     import hashlib
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+            h.update(b"".join(f.read().split()))
     return h.hexdigest()
 
 

@@ -211,191 +211,191 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
                                               uint32_t tmem_base, int warp, int lane, int m_blocks,
                                               int total_tiles, int num_kb, int P) {
   volatile int* abort_flag = &s->abort;
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 4;
-    const int half = ew >> 2;                  // which 128 of the 256 MMA columns (up: which 64 of I)
-    const int quarter = warp & 3;              // TMEM lanes this warp may access
-    const int row = quarter * 32 + lane;       // tile row = TMEM lane
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint8_t* my_staging = staging + ew * kStagingBytes;
-    // TMEM columns of this thread's two 64-column segments
-    const int col0 = (MODE == kModeMoeUp) ? half * 64 : half * 128;
-    const int col1 = (MODE == kModeMoeUp) ? kBN / 2 + half * 64 : half * 128 + 64;
-    int buf = 0, sslot = 0, tcount = 0;
-    uint32_t tphase = 0, scphase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
-      int mb, nt;
-      tile_coords<MODE>(args, tile, m_blocks, mb, nt);
-      // An M=64 tile keeps its row r in TMEM lane (r % 16) + 32 * (r / 16): lanes
-      // 0..15 of each warp hold rows 16*quarter + lane, lanes 16..31 hold none.
-      const bool m64 = moe_half_tile<MODE>(args, mb, P);
-      const int trow = m64 ? (lane < 16 ? quarter * 16 + lane : -1) : row;
-      const bool has_row = trow >= 0;
-      const int slot = mb * kBM + (has_row ? trow : 0);
-      int pair = P;
-      float wroute = 0.0f;
-      if (MODE != kModeDense && has_row) {      // needed only at the end: load early
-        pair = args.sorted_ids[slot];
-        if (MODE == kModeMoeDown) wroute = args.sorted_weights[slot];
+  // ------------------------------------------------------------ epilogue
+  const int ew = warp - 4;
+  const int half = ew >> 2;                  // which 128 of the 256 MMA columns (up: which 64 of I)
+  const int quarter = warp & 3;              // TMEM lanes this warp may access
+  const int row = quarter * 32 + lane;       // tile row = TMEM lane
+  const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+  uint8_t* my_staging = staging + ew * kStagingBytes;
+  // TMEM columns of this thread's two 64-column segments
+  const int col0 = (MODE == kModeMoeUp) ? half * 64 : half * 128;
+  const int col1 = (MODE == kModeMoeUp) ? kBN / 2 + half * 64 : half * 128 + 64;
+  int buf = 0, sslot = 0, tcount = 0;
+  uint32_t tphase = 0, scphase = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
+    int mb, nt;
+    tile_coords<MODE>(args, tile, m_blocks, mb, nt);
+    // An M=64 tile keeps its row r in TMEM lane (r % 16) + 32 * (r / 16): lanes
+    // 0..15 of each warp hold rows 16*quarter + lane, lanes 16..31 hold none.
+    const bool m64 = moe_half_tile<MODE>(args, mb, P);
+    const int trow = m64 ? (lane < 16 ? quarter * 16 + lane : -1) : row;
+    const bool has_row = trow >= 0;
+    const int slot = mb * kBM + (has_row ? trow : 0);
+    int pair = P;
+    float wroute = 0.0f;
+    if (MODE != kModeDense && has_row) {      // needed only at the end: load early
+      pair = args.sorted_ids[slot];
+      if (MODE == kModeMoeDown) wroute = args.sorted_weights[slot];
+    }
+    float acc[128];
+#pragma unroll
+    for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+    // a warp whose 32 rows are all padding skips the promotion (its outputs are never stored)
+    const bool warp_active = MODE == kModeDense || __any_sync(0xffffffffu, pair >= 0 && pair < P);
+
+    for (int kb = 0; kb < num_kb; ++kb) {
+      if (!mbar_wait(&s->sfull[sslot], scphase, abort_flag)) { ok = false; break; }
+      const float sa = s->sa[sslot][has_row ? trow : 0];
+      const float swa = s->sw[sslot][0], swb = s->sw[sslot][1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s->sempty[sslot]);
+      if (++sslot == kScaleSlots) { sslot = 0; scphase ^= 1u; }
+      float f0, f1;
+      if (MODE == kModeMoeUp) {
+        f0 = sa * swa;
+        f1 = sa * swb;
+      } else {
+        f0 = f1 = sa * (half ? swb : swa);
       }
-      float acc[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-      // a warp whose 32 rows are all padding skips the promotion (its outputs are never stored)
-      const bool warp_active = MODE == kModeDense || __any_sync(0xffffffffu, pair >= 0 && pair < P);
 
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&s->sfull[sslot], scphase, abort_flag)) { ok = false; break; }
-        const float sa = s->sa[sslot][has_row ? trow : 0];
-        const float swa = s->sw[sslot][0], swb = s->sw[sslot][1];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s->sempty[sslot]);
-        if (++sslot == kScaleSlots) { sslot = 0; scphase ^= 1u; }
-        float f0, f1;
-        if (MODE == kModeMoeUp) {
-          f0 = sa * swa;
-          f1 = sa * swb;
-        } else {
-          f0 = f1 = sa * (half ? swb : swa);
-        }
-
-        if (!mbar_wait(&s->tfull[buf], tphase, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (!warp_active) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s->tempty[buf]);
-          if (++buf == 2) { buf = 0; tphase ^= 1u; }
-          continue;
-        }
-        const uint32_t tb = lane_base + buf * kBN;
-        // four 32-column chunks; the load of chunk c+1 overlaps the FMAs of chunk c
-        float v[2][32];
-        tmem_ld_32x32b_x32(tb + col0, v[0]);
-        tmem_wait_ld();
-        reg_fence_32(v[0]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c + 1 < 4) tmem_ld_32x32b_x32(tb + ((c + 1) < 2 ? col0 : col1) + ((c + 1) & 1) * 32, v[(c + 1) & 1]);
-          const float f = (c < 2) ? f0 : f1;
-          const float2 ff = make_float2(f, f);
-          // packed fp32 FMA (two lanes per instruction, each rounded to nearest)
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float2 r = __ffma2_rn(ff, make_float2(v[c & 1][j], v[c & 1][j + 1]),
-                                        make_float2(acc[c * 32 + j], acc[c * 32 + j + 1]));
-            acc[c * 32 + j] = r.x;
-            acc[c * 32 + j + 1] = r.y;
-          }
-          if (c + 1 < 4) {
-            tmem_wait_ld();
-            reg_fence_32(v[(c + 1) & 1]);
-          }
-        }
+      if (!mbar_wait(&s->tfull[buf], tphase, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (!warp_active) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s->tempty[buf]);
         if (++buf == 2) { buf = 0; tphase ^= 1u; }
+        continue;
       }
-      if (!ok) break;
+      const uint32_t tb = lane_base + buf * kBN;
+      // four 32-column chunks; the load of chunk c+1 overlaps the FMAs of chunk c
+      float v[2][32];
+      tmem_ld_32x32b_x32(tb + col0, v[0]);
+      tmem_wait_ld();
+      reg_fence_32(v[0]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c + 1 < 4) tmem_ld_32x32b_x32(tb + ((c + 1) < 2 ? col0 : col1) + ((c + 1) & 1) * 32, v[(c + 1) & 1]);
+        const float f = (c < 2) ? f0 : f1;
+        const float2 ff = make_float2(f, f);
+        // packed fp32 FMA (two lanes per instruction, each rounded to nearest)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 r = __ffma2_rn(ff, make_float2(v[c & 1][j], v[c & 1][j + 1]),
+                                      make_float2(acc[c * 32 + j], acc[c * 32 + j + 1]));
+          acc[c * 32 + j] = r.x;
+          acc[c * 32 + j + 1] = r.y;
+        }
+        if (c + 1 < 4) {
+          tmem_wait_ld();
+          reg_fence_32(v[(c + 1) & 1]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s->tempty[buf]);
+      if (++buf == 2) { buf = 0; tphase ^= 1u; }
+    }
+    if (!ok) break;
 
-      // Outputs. Dense and gate/up: each thread writes its own row with 32-byte
-      // stores (whole sectors) straight from registers.
-      if (MODE == kModeDense) {
-        const int grow = mb * kBM + row;
-        const int x0 = nt * kBN + half * 128;
-        if (grow < args.M) {
-          __nv_bfloat16* crow = args.C + static_cast<size_t>(grow) * args.ldc;
-          const bool vec = args.c_vec != 0 && x0 + 128 <= args.N;
+    // Outputs. Dense and gate/up: each thread writes its own row with 32-byte
+    // stores (whole sectors) straight from registers.
+    if (MODE == kModeDense) {
+      const int grow = mb * kBM + row;
+      const int x0 = nt * kBN + half * 128;
+      if (grow < args.M) {
+        __nv_bfloat16* crow = args.C + static_cast<size_t>(grow) * args.ldc;
+        const bool vec = args.c_vec != 0 && x0 + 128 <= args.N;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {      // 8 chunks of 16 bf16 columns
-            uint32_t w[8];
+        for (int ch = 0; ch < 8; ++ch) {      // 8 chunks of 16 bf16 columns
+          uint32_t w[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[ch * 16 + 2 * u], acc[ch * 16 + 2 * u + 1]);
-              w[u] = *reinterpret_cast<const uint32_t*>(&pk);
-            }
-            const int x = x0 + ch * 16;
-            if (vec) {
-              st_global_v8(crow + x, w);
-            } else {                            // ragged edge or unaligned C: element stores
-              const __nv_bfloat16* vals = reinterpret_cast<const __nv_bfloat16*>(w);
+          for (int u = 0; u < 8; ++u) {
+            const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[ch * 16 + 2 * u], acc[ch * 16 + 2 * u + 1]);
+            w[u] = *reinterpret_cast<const uint32_t*>(&pk);
+          }
+          const int x = x0 + ch * 16;
+          if (vec) {
+            st_global_v8(crow + x, w);
+          } else {                            // ragged edge or unaligned C: element stores
+            const __nv_bfloat16* vals = reinterpret_cast<const __nv_bfloat16*>(w);
 #pragma unroll
-              for (int u = 0; u < 16; ++u)
-                if (x + u < args.N) crow[x + u] = vals[u];
-            }
+            for (int u = 0; u < 16; ++u)
+              if (x + u < args.N) crow[x + u] = vals[u];
           }
         }
-      } else if (MODE == kModeMoeUp) {
-        // h = silu(gate) * up for this thread's 64 intermediate columns
-        float amax = 0.0f;
+      }
+    } else if (MODE == kModeMoeUp) {
+      // h = silu(gate) * up for this thread's 64 intermediate columns
+      float amax = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float g = acc[j];
-          const float h = __fdividef(g, 1.0f + __expf(-g)) * acc[64 + j];
-          acc[j] = h;
-          amax = fmaxf(amax, fabsf(h));
-        }
-        // the 128-wide requantisation group spans both column halves of the row
-        const int xb = tcount & 1;
-        s->amax_x[xb][half][row] = amax;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s->xbar[xb]);
-        if (!mbar_wait(&s->xbar[xb], (tcount >> 1) & 1, abort_flag)) { ok = false; break; }
-        amax = fmaxf(amax, s->amax_x[xb][half ^ 1][row]);
-        const float scale = __fdiv_rn(amax, 448.0f);
-        const float inv = scale != 0.0f ? __frcp_rn(scale) : 0.0f;
-        if (pair >= 0 && pair < P) {
-          uint8_t* dst = args.a2 + static_cast<size_t>(slot) * args.N + nt * 128 + half * 64;
+      for (int j = 0; j < 64; ++j) {
+        const float g = acc[j];
+        const float h = __fdividef(g, 1.0f + __expf(-g)) * acc[64 + j];
+        acc[j] = h;
+        amax = fmaxf(amax, fabsf(h));
+      }
+      // the 128-wide requantisation group spans both column halves of the row
+      const int xb = tcount & 1;
+      s->amax_x[xb][half][row] = amax;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s->xbar[xb]);
+      if (!mbar_wait(&s->xbar[xb], (tcount >> 1) & 1, abort_flag)) { ok = false; break; }
+      amax = fmaxf(amax, s->amax_x[xb][half ^ 1][row]);
+      const float scale = __fdiv_rn(amax, 448.0f);
+      const float inv = scale != 0.0f ? __frcp_rn(scale) : 0.0f;
+      if (pair >= 0 && pair < P) {
+        uint8_t* dst = args.a2 + static_cast<size_t>(slot) * args.N + nt * 128 + half * 64;
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {      // 2 x 32 codes
-            uint32_t w[8];
+        for (int ch = 0; ch < 2; ++ch) {      // 2 x 32 codes
+          uint32_t w[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int j = ch * 32 + 4 * u;
-              w[u] = static_cast<uint32_t>(cvt_e4m3x2(acc[j] * inv, acc[j + 1] * inv)) |
-                     (static_cast<uint32_t>(cvt_e4m3x2(acc[j + 2] * inv, acc[j + 3] * inv)) << 16);
-            }
-            st_global_v8(dst + ch * 32, w);
+          for (int u = 0; u < 8; ++u) {
+            const int j = ch * 32 + 4 * u;
+            w[u] = static_cast<uint32_t>(cvt_e4m3x2(acc[j] * inv, acc[j + 1] * inv)) |
+                   (static_cast<uint32_t>(cvt_e4m3x2(acc[j + 2] * inv, acc[j + 3] * inv)) << 16);
           }
+          st_global_v8(dst + ch * 32, w);
         }
-        if (half == 0 && has_row) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
-      } else {
-        // 256 bytes of bf16 per row: a transpose through the warp's staging buffer
-        // lets each store instruction write 8 whole 64-byte row segments
-        const bool valid = pair >= 0 && pair < P;
-        if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
-        const int x0 = nt * kBN + half * 128;
-        if (x0 < args.N) {
-          const int H = args.N;
-          __nv_bfloat16* y = args.ystage;
+      }
+      if (half == 0 && has_row) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
+    } else {
+      // 256 bytes of bf16 per row: a transpose through the warp's staging buffer
+      // lets each store instruction write 8 whole 64-byte row segments
+      const bool valid = pair >= 0 && pair < P;
+      if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
+      const int x0 = nt * kBN + half * 128;
+      if (x0 < args.N) {
+        const int H = args.N;
+        __nv_bfloat16* y = args.ystage;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
-            uint4 d[4];
+        for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
+          uint4 d[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint32_t w[4];
+          for (int u = 0; u < 4; ++u) {
+            uint32_t w[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int j = ch * 32 + u * 8 + 2 * q;
-                const __nv_bfloat162 pk = __floats2bfloat162_rn(wroute * acc[j], wroute * acc[j + 1]);
-                w[q] = *reinterpret_cast<const uint32_t*>(&pk);
-              }
-              d[u] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int q = 0; q < 4; ++q) {
+              const int j = ch * 32 + u * 8 + 2 * q;
+              const __nv_bfloat162 pk = __floats2bfloat162_rn(wroute * acc[j], wroute * acc[j + 1]);
+              w[q] = *reinterpret_cast<const uint32_t*>(&pk);
             }
-            const int x = x0 + ch * 32;
-            store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
-              const int pr = __shfl_sync(0xffffffffu, pair, r);
-              return (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x)
-                                         : nullptr;
-            });
+            d[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
+          const int x = x0 + ch * 32;
+          store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
+            const int pr = __shfl_sync(0xffffffffu, pair, r);
+            return (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x)
+                                       : nullptr;
+          });
         }
       }
     }
-    if (!ok) abort_all(s);
   }
+  if (!ok) abort_all(s);
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
