@@ -1,5 +1,6 @@
 """The FP8 block-scaled MoE layer as one object: weights resident on the device,
-buffers preallocated, forward = route -> align/sort -> 1x128 quant -> fused g1u1 MoE.
+buffers preallocated, forward = route -> align/sort (and, on a side stream at the same
+time, 1x128 quant) -> fused g1u1 MoE.
 
 This mirrors the composition the pages' asm_moe wrapper performs ("Accelerate
 DeepSeek-R1 Inference: Integrate AITER into SGLang", section "Blockscale FP8
@@ -34,6 +35,11 @@ class MoELayer:
             self.w2_scale = torch.empty(E, H // 128, Im // 128, dtype=torch.float32, device=dev)
         self.block_m = B.moe_block_m()
         self._alloc(self.max_tokens)
+        # The activation quantisation depends only on x, so it runs on a side stream
+        # while routing and sorting run on the caller's stream.
+        self._side = torch.cuda.Stream(device=dev) if dev.type == "cuda" else None
+        self._fork = torch.cuda.Event() if dev.type == "cuda" else None
+        self._join = torch.cuda.Event() if dev.type == "cuda" else None
 
     def _alloc(self, T):
         cfg, dev = self.cfg, self.device
@@ -63,10 +69,16 @@ class MoELayer:
         T = x.shape[0]
         if T != self.max_tokens:
             raise ValueError(f"layer buffers are sized for {self.max_tokens} tokens, got {T}")
+        main = torch.cuda.current_stream(self.device)
+        self._fork.record(main)
+        self._side.wait_event(self._fork)
+        with torch.cuda.stream(self._side):
+            B.fp8_per_token_group_quant(x, 128, column_major_scales=True, q=self.a8, scales=self.a8_scale)
+            self._join.record(self._side)
         B.moe_biased_grouped_topk(logits, bias, self.topk_w, self.topk_ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
         B.moe_align_sort(self.topk_ids, self.topk_w, cfg.E, self.block_m, out=self.sorted,
                          workspace=self.sort_workspace)
-        B.fp8_per_token_group_quant(x, 128, column_major_scales=True, q=self.a8, scales=self.a8_scale)
+        main.wait_event(self._join)
         B.fused_moe_fp8_blockscale_g1u1(self.out, self.a8, self.w1, self.w2, self.sorted, cfg.K, self.a8_scale,
                                         self.w1_scale, self.w2_scale, workspace=self.workspace)
         return self.out
