@@ -477,8 +477,9 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (int rc = make_operand_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
 
   timing_record(0, st);
-  moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, num_valid_ids, T, topk, H,
-                                                            static_cast<int>(capacity), a8s, s1s);
+  moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, sorted_expert_ids,
+                                                            num_valid_ids, T, topk, H, static_cast<int>(capacity),
+                                                            a8s, s1s);
   if (int rc = check_launch("fused_moe (gather)")) return rc;
   timing_record(1, st);
 

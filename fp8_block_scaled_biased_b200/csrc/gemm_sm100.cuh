@@ -571,11 +571,16 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 constexpr int kGatherWarps = 8;
 __global__ void __launch_bounds__(32 * kGatherWarps)
 moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_scale,
-                  const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ num_valid_ids, int T,
-                  int topk, int H, int cap, uint8_t* __restrict__ a8s, float* __restrict__ s1s) {
+                  const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ sorted_expert_ids,
+                  const int32_t* __restrict__ num_valid_ids, int T, int topk, int H, int cap,
+                  uint8_t* __restrict__ a8s, float* __restrict__ s1s) {
   const int lane = threadIdx.x & 31;
   const int P = T * topk;
   const int nv = min(max(*num_valid_ids, 0), cap);
+  // The gate/up GEMM's tile order needs each expert's blocks to be contiguous, as the
+  // sort's ascending expert order makes them: flag a decreasing pair of block ids.
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b + 1 < nv / kBM; b += gridDim.x * blockDim.x)
+    if (sorted_expert_ids[b] > sorted_expert_ids[b + 1]) raise_device_error(FP8MOE_DEVERR_BLOCK_ORDER);
   const int KB = H / 128;
   const int vec_per_row = H / 16;
   for (int slot = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); slot < nv; slot += gridDim.x * kGatherWarps) {

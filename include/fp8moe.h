@@ -50,7 +50,8 @@ enum fp8moe_device_error {
   FP8MOE_DEVERR_TIMEOUT = 1u,     /* a bounded wait inside a GEMM kernel expired  */
   FP8MOE_DEVERR_EXPERT_ID = 2u,   /* an expert id outside [0, E) was met          */
   FP8MOE_DEVERR_PAIR_ID = 4u,     /* a sorted pair id outside [0, T*topk] was met */
-  FP8MOE_DEVERR_NUM_VALID = 8u    /* num_valid_ids above capacity or not a multiple of block_m */
+  FP8MOE_DEVERR_NUM_VALID = 8u,   /* num_valid_ids above capacity or not a multiple of block_m */
+  FP8MOE_DEVERR_BLOCK_ORDER = 16u /* sorted_expert_ids decreases somewhere: not a moe_align_sort result */
 };
 
 /* Message describing the calling thread's most recent failure ("" if none). */
@@ -192,7 +193,9 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B,
  * w1         fp8 [E, 2I, H]; rows [0, I) of each expert are the gate
  *            projection, rows [I, 2I) the up projection
  * w2         fp8 [E, H, I]
- * sorted_*   the outputs of moe_align_sort with block_m == fp8moe_moe_block_m()
+ * sorted_*   the outputs of moe_align_sort with block_m == fp8moe_moe_block_m(); a
+ *            sorted_expert_ids that decreases from one block to the next is flagged
+ *            FP8MOE_DEVERR_BLOCK_ORDER (the output is then unspecified)
  * a1_scale   fp32 [H/128, T] (transposed 1x128 scales of a8)
  * fc1_scale  fp32 [E, 2I/128, H/128];  fc2_scale fp32 [E, H/128, I/128]
  * For every pair p = (t, k) with expert e:

@@ -271,3 +271,21 @@ def test_fused_moe_zero_tokens_is_a_no_op():
                                     layer.w2_scale)
     torch.cuda.synchronize()
     assert out.numel() == 0
+
+
+def test_fused_moe_flags_unsorted_block_experts():
+    """Block expert ids that decrease (not a moe_align_sort result) raise the device error bit."""
+    cfg = MID
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    act = I.moe_activations(cfg)
+    layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    assert B.device_status() == 0
+    sp = layer.sorted
+    nblocks = int(sp.num_valid_ids.item()) // layer.block_m
+    ids = sp.sorted_expert_ids[:nblocks].clone()
+    assert nblocks >= 2 and int(ids[0]) < int(ids[-1])
+    sp.sorted_expert_ids[:nblocks] = torch.flip(ids, [0])
+    B.fused_moe_fp8_blockscale_g1u1(layer.out, layer.a8, layer.w1, layer.w2, sp, cfg.K, layer.a8_scale,
+                                    layer.w1_scale, layer.w2_scale, workspace=layer.workspace)
+    assert B.device_status() & 16
+    assert B.device_status() == 0          # read and cleared
