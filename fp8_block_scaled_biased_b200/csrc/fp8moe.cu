@@ -13,9 +13,12 @@
 
 #include "common.cuh"
 #include "gemm_sm100.cuh"
+#include "moe_aux.cuh"
 #include "quant.cuh"
 #include "route.cuh"
 #include "sort.cuh"
+
+static_assert(fp8moe::kMoeBlockRows == fp8moe::kBM, "sorted blocks are GEMM tiles");
 
 using namespace fp8moe;
 

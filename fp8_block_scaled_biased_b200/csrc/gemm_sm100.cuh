@@ -565,87 +565,4 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   }
 }
 
-// Copies each sorted slot's token row of a8 [T, H] (and its H/128 scales from
-// a1_scale [H/128, T]) into slot order. Padding slots are skipped: the GEMMs
-// treat rows independently and never store padding rows.
-constexpr int kGatherWarps = 8;
-__global__ void __launch_bounds__(32 * kGatherWarps)
-moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_scale,
-                  const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ sorted_expert_ids,
-                  const int32_t* __restrict__ num_valid_ids, int T, int topk, int H, int cap,
-                  uint8_t* __restrict__ a8s, float* __restrict__ s1s) {
-  const int lane = threadIdx.x & 31;
-  const int P = T * topk;
-  const int nv = min(max(*num_valid_ids, 0), cap);
-  // The gate/up GEMM's tile order needs each expert's blocks to be contiguous, as the
-  // sort's ascending expert order makes them: flag a decreasing pair of block ids.
-  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b + 1 < nv / kBM; b += gridDim.x * blockDim.x)
-    if (sorted_expert_ids[b] > sorted_expert_ids[b + 1]) raise_device_error(FP8MOE_DEVERR_BLOCK_ORDER);
-  const int KB = H / 128;
-  const int vec_per_row = H / 16;
-  for (int slot = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); slot < nv; slot += gridDim.x * kGatherWarps) {
-    const int sid = sorted_ids[slot];
-    if (sid < 0 || sid >= P) continue;
-    const int t = sid / topk;
-    const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
-    uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
-    // issue a batch of loads before their stores, so the row costs one round trip per batch
-    constexpr int kBatch = 16;
-    for (int v0 = 0; v0 < vec_per_row; v0 += 32 * kBatch) {
-      uint4 buf[kBatch];
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int v = v0 + i * 32 + lane;
-        if (v < vec_per_row) buf[i] = src[v];
-      }
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int v = v0 + i * 32 + lane;
-        if (v < vec_per_row) dst[v] = buf[i];
-      }
-    }
-  }
-  // scales: one lane per slot of a 32-slot group, so each store instruction
-  // writes 128 contiguous bytes of a row of s1s
-  const int nwarps = gridDim.x * kGatherWarps;
-  for (int s0 = (blockIdx.x * kGatherWarps + (threadIdx.x >> 5)) * 32; s0 < nv; s0 += nwarps * 32) {
-    const int slot = s0 + lane;
-    const int sid = slot < nv ? sorted_ids[slot] : -1;
-    if (sid < 0 || sid >= P) continue;
-    const int t = sid / topk;
-    for (int kb = 0; kb < KB; ++kb)
-      s1s[static_cast<size_t>(kb) * cap + slot] = __ldg(a1_scale + static_cast<size_t>(kb) * T + t);
-  }
-}
-
-// out[t, :] = bf16( y[t*K + 0] + y[t*K + 1] + ... + y[t*K + K-1] ), fp32 adds in
-// slot order k (the routing weight is already in y). One thread per 8 columns.
-__global__ void __launch_bounds__(256)
-moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
-  const int cpr = H / 8;
-  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<size_t>(T) * cpr) return;
-  const int t = static_cast<int>(idx / cpr);
-  const int c = static_cast<int>(idx % cpr) * 8;
-  const __nv_bfloat16* y = ystage + static_cast<size_t>(t) * K * H + c;
-  float sum[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
-  // fp32 sum in k order (0.0f + y0 == y0 exactly, so the order is fixed from the first term)
-  for (int k = 0; k < K; ++k) {
-    const uint4 v = *reinterpret_cast<const uint4*>(y + static_cast<size_t>(k) * H);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
-      sum[2 * u] += f.x;
-      sum[2 * u + 1] += f.y;
-    }
-  }
-  __align__(16) __nv_bfloat162 pk[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) pk[u] = __floats2bfloat162_rn(sum[2 * u], sum[2 * u + 1]);
-  *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<const uint4*>(pk);
-}
-
 }  // namespace fp8moe
