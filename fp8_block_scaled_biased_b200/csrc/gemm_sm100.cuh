@@ -22,8 +22,9 @@
 //               a_scale[row, kb] * b_scale[col/128, kb] and add into fp32
 //               registers (the per-128-K promotion), then the mode's output:
 //               32-byte (whole-sector) stores of each thread's row, or for the
-//               down GEMM's fp32 rows a transpose through a small shared buffer
-//               per warp so that each store writes 8 whole 64-byte row segments.
+//               down GEMM's weighted bf16 rows a transpose through a small
+//               shared buffer per warp so that each store writes 8 whole 64-byte
+//               row segments.
 // In the MoE modes the rows are the sorted token-expert slots: A is the
 // slot-ordered activation matrix (gathered by moe_gather_kernel for GEMM1, the
 // re-quantised intermediate for GEMM2), one expert per 128-row block.
