@@ -396,7 +396,7 @@ def run_ours(args, world, rank, local):
                 "method": "pinned host buffers through layer.forward; two-deep pipeline: step i+1's H2D and "
                           "step i-1's D2H overlap step i's forward on separate copy streams",
                 "serial": {"value": tokens / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}},
-        "gpu_launches": args.steps * layer.LAUNCHES_PER_FORWARD,
+        "gpu_launches": args.steps * layer.launches_per_forward,
         "clocks": clocks,
         "wall_s_timed": wall,
     }

@@ -102,6 +102,9 @@ int device_setup(int* sm_count) {
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSortWarps * kSortMaxExperts * static_cast<int>(sizeof(int)));
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(sort_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (kSortWarps + 2) * kSortMaxExperts * static_cast<int>(sizeof(int)));
     d.err = static_cast<int>(r);
   });
   if (d.err == -1) return fail(FP8MOE_EUNSUPPORTED, "device %d is not sm_100 (B200)", dev);
@@ -341,6 +344,12 @@ int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int pairs = T * topk;
   const int nchunks = (pairs + kSortChunk - 1) / kSortChunk;
+  if (nchunks <= 1) {                   // one chunk: count, scan and scatter in a single CTA
+    sort_small_kernel<<<1, kSortChunk, static_cast<size_t>(kSortWarps + 2) * E * sizeof(int), st>>>(
+        topk_ids, topk_weights, ld, T, topk, E, block_m, sorted_ids, sorted_weights, sorted_expert_ids,
+        num_valid_ids);
+    return check_launch("moe_align_sort (single chunk)");
+  }
   int32_t* counts = static_cast<int32_t*>(workspace);                       // [nchunks][E]
   int32_t* seg_start = counts + round_up(static_cast<size_t>(nchunks) * E * sizeof(int32_t), 256) / sizeof(int32_t);
   if (nchunks > 0) {

@@ -149,4 +149,86 @@ sort_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w
   }
 }
 
+// All three steps in one CTA when the pairs fit one chunk (P <= kSortChunk, a
+// decode-sized batch): the chunk histogram is the per-warp counts summed, the
+// segment starts come from it directly, and there are no earlier chunks.
+// Shared memory: total[E], start[E], warp_cnt[kSortWarps][E].
+__global__ void __launch_bounds__(kSortChunk)
+sort_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, int ld, int T, int K, int E,
+                  int block_m, int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w,
+                  int32_t* __restrict__ sorted_e, int32_t* __restrict__ num_valid) {
+  extern __shared__ int sm_small[];
+  int* total = sm_small;
+  int* start = sm_small + E;
+  int* warp_cnt = sm_small + 2 * E;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int P = T * K;
+  for (int i = tid; i < E; i += kSortChunk) total[i] = 0;
+  for (int i = tid; i < kSortWarps * E; i += kSortChunk) warp_cnt[i] = 0;
+  __syncthreads();
+  const int p = tid;
+  int e = -1;
+  float wv = 0.0f;
+  if (p < P) {
+    e = read_pair_expert(ids, ld, K, p, E);
+    if (e >= 0) {
+      const int t = p / K, k = p - t * K;
+      wv = w[static_cast<size_t>(t) * ld + k];
+    } else {
+      raise_device_error(FP8MOE_DEVERR_EXPERT_ID);
+    }
+  }
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(same & ((1u << lane) - 1u));
+  if (e >= 0 && rank == 0) {
+    warp_cnt[warp * E + e] = __popc(same);
+    atomicAdd(&total[e], __popc(same));
+  }
+  __syncthreads();
+  // padded segment starts: exclusive scan of ceil(total/bm)*bm over experts (warp 0)
+  if (warp == 0) {
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int ex = e0 + lane;
+      const int len = (ex < E) ? (total[ex] + block_m - 1) / block_m * block_m : 0;
+      int incl = len;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (ex < E) start[ex] = carry + incl - len;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) *num_valid = carry;
+  }
+  __syncthreads();
+  // per expert: each warp's first slot (exclusive prefix over warps from the segment start)
+  for (int ex = tid; ex < E; ex += kSortChunk) {
+    int run = start[ex];
+    for (int wi = 0; wi < kSortWarps; ++wi) {
+      const int v = warp_cnt[wi * E + ex];
+      warp_cnt[wi * E + ex] = run;
+      run += v;
+    }
+  }
+  // block expert ids and padding slots
+  for (int ex = warp; ex < E; ex += kSortWarps) {
+    const int c = total[ex];
+    const int s0 = start[ex];
+    const int len = (c + block_m - 1) / block_m * block_m;
+    for (int j = lane; j < len / block_m; j += 32) sorted_e[s0 / block_m + j] = ex;
+    for (int sl = s0 + c + lane; sl < s0 + len; sl += 32) {
+      sorted_ids[sl] = P;
+      sorted_w[sl] = 0.0f;
+    }
+  }
+  __syncthreads();
+  if (e >= 0) {
+    const int slot = warp_cnt[warp * E + e] + rank;
+    sorted_ids[slot] = p;
+    sorted_w[slot] = wv;
+  }
+}
+
 }  // namespace fp8moe

@@ -83,6 +83,9 @@ class MoELayer:
                                         self.w1_scale, self.w2_scale, workspace=self.workspace)
         return self.out
 
-    # kernels launched by one forward: route, sort (count, scan, scatter), quant, gather, gate/up GEMM,
-    # down GEMM, combine
-    LAUNCHES_PER_FORWARD = 9
+    @property
+    def launches_per_forward(self):
+        """Kernels one forward launches: route, sort (count, scan and scatter; one kernel when the
+        T*topk pairs fit one 1024-pair chunk), quant, gather, gate/up GEMM, down GEMM, combine."""
+        sort_kernels = 1 if self.max_tokens * self.cfg.K <= 1024 else 3
+        return 6 + sort_kernels
