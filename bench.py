@@ -177,8 +177,8 @@ def layer_work(cfg, ids):
 # figure whose sources have changed since is not reported.
 GATE_UP_TRAFFIC = {
     "prefill_t4096_h7168_e256": {
-        "bytes": 7.018e9,
-        "sha256": "998ae1aec86c49a587c3a1435c85ad4e8197439c994b52ec361ae50cfc801721",
+        "bytes": 6.907e9,
+        "sha256": "43a889b0ef6edc1cdb12947d1aef764571339206807851e70a06ac3c707053e5",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
                    "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean; "
                    "profiles/launches_prefill_t4096.md)",
