@@ -177,8 +177,8 @@ def layer_work(cfg, ids):
 # figure whose sources have changed since is not reported.
 GATE_UP_TRAFFIC = {
     "prefill_t4096_h7168_e256": {
-        "bytes": 6.907e9,
-        "sha256": "43a889b0ef6edc1cdb12947d1aef764571339206807851e70a06ac3c707053e5",
+        "bytes": 6.839e9,
+        "sha256": "4fa34e3ec083d9bbe4964de41a517166aa645f173e329cde31b816d35b71a28e",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
                    "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean; "
                    "profiles/launches_prefill_t4096.md)",

@@ -71,6 +71,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same wait for a role with slack (a tile or more ahead of its consumers):
+// it sleeps between polls, so that it takes no issue slots from the warps that
+// share its scheduler.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (;;) {
+    __nanosleep(500);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // cp.async (LSU asynchronous copy) of 4 bytes global -> shared, and an arrive
 // on an mbarrier once all of this thread's earlier cp.async have landed.
 __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {

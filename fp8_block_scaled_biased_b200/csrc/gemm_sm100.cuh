@@ -17,7 +17,10 @@
 //               of two 256-column TMEM buffers, fresh (not accumulated) so the
 //               buffer holds that block's partial sums;
 //   warp 2      scale loader: each K block's row and column scales into an
-//               8-slot ring (cp.async); warp 3 idles;
+//               8-slot ring (cp.async);
+//   warp 3      tile info: one tile ahead, the tile's coordinates, its MMA
+//               shape and its rows' pair ids and routing weights into a 2-slot
+//               shared ring for the MMA issuer and the epilogue;
 //   warps 4..11 epilogue: tcgen05.ld the partials, multiply by
 //               a_scale[row, kb] * b_scale[col/128, kb] and add into fp32
 //               registers (the per-128-K promotion), then the mode's output:
@@ -89,11 +92,18 @@ struct GemmSmem {
   uint64_t sfull[kScaleSlots];
   uint64_t sempty[kScaleSlots];
   uint64_t xbar[2];                       // up: amax exchange between the two column halves
+  uint64_t tifull[2];                     // tile-info ring (warp 3 -> MMA issuer + epilogue)
+  uint64_t tiempty[2];
   uint32_t tmem_base;
   int abort;
   float sa[kScaleSlots][kBM];
   float sw[kScaleSlots][4];
   float amax_x[2][2][kBM];
+  // tile-info ring: the tile's coordinates, whether it runs with M=64, and per
+  // row the pair id and routing weight (MoE), prepared one tile ahead
+  int ti_mb[2], ti_nt[2], ti_m64[2];
+  int ti_pair[2][kBM];
+  float ti_w[2][kBM];
 };
 
 constexpr size_t kGemmSmemBytes =
@@ -166,16 +176,6 @@ __device__ __forceinline__ int moe_expert(const GemmArgs& a, int mb) {
   return e;
 }
 
-// MoE tile whose second half holds only padding slots (an expert's last block
-// with at most 64 pairs): its MMAs run with M=64. The sort puts an expert's
-// pairs before its padding, so slot 64 of the block decides.
-template <int MODE>
-__device__ __forceinline__ bool moe_half_tile(const GemmArgs& a, int mb, int P) {
-  if (MODE == kModeDense) return false;
-  const int id = a.sorted_ids[mb * kBM + kBM / 2];
-  return id < 0 || id >= P;
-}
-
 __device__ __forceinline__ void abort_all(GemmSmem* s) {
   if (!s->abort) raise_device_error(FP8MOE_DEVERR_TIMEOUT);
   s->abort = 1;
@@ -218,37 +218,45 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
   const int quarter = warp & 3;              // TMEM lanes this warp may access
   const int row = quarter * 32 + lane;       // tile row = TMEM lane
   const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-  uint8_t* my_staging = staging + ew * kStagingBytes;
   // TMEM columns of this thread's two 64-column segments
   const int col0 = (MODE == kModeMoeUp) ? half * 64 : half * 128;
   const int col1 = (MODE == kModeMoeUp) ? kBN / 2 + half * 64 : half * 128 + 64;
-  int buf = 0, sslot = 0, tcount = 0;
-  uint32_t tphase = 0, scphase = 0;
+  int buf = 0, sslot = 0, tislot = 0;
+  uint32_t tphase = 0, scphase = 0, tiphase = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
-    int mb, nt;
-    tile_coords<MODE>(args, tile, m_blocks, mb, nt);
+  for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    // The tile's coordinates and rows. The dense and down epilogues take them
+    // from the tile-info ring (shared memory): the slot is held until the
+    // tile's output is written, and values needed only there are read there, so
+    // that they take no registers during the promotion loop. The gate/up
+    // epilogue loads its own copy from global memory at the tile start and keeps
+    // it in registers, which measured about 4% faster for that GEMM.
+    if (!mbar_wait(&s->tifull[tislot], tiphase, abort_flag)) { ok = false; break; }
     // An M=64 tile keeps its row r in TMEM lane (r % 16) + 32 * (r / 16): lanes
     // 0..15 of each warp hold rows 16*quarter + lane, lanes 16..31 hold none.
-    const bool m64 = moe_half_tile<MODE>(args, mb, P);
-    const int trow = m64 ? (lane < 16 ? quarter * 16 + lane : -1) : row;
-    const bool has_row = trow >= 0;
-    const int slot = mb * kBM + (has_row ? trow : 0);
-    int pair = P;
-    float wroute = 0.0f;
-    if (MODE != kModeDense && has_row) {      // needed only at the end: load early
-      pair = args.sorted_ids[slot];
-      if (MODE == kModeMoeDown) wroute = args.sorted_weights[slot];
+    auto lane_row = [&](bool m64) { return m64 ? (lane < 16 ? quarter * 16 + lane : -1) : row; };
+    int up_mb = 0, up_nt = 0, up_trow = -1, up_pair = P;
+    if (MODE == kModeMoeUp) {
+      tile_coords<MODE>(args, tile, m_blocks, up_mb, up_nt);
+      const int id_half = args.sorted_ids[up_mb * kBM + kBM / 2];
+      up_trow = lane_row(id_half < 0 || id_half >= P);
+      if (up_trow >= 0) up_pair = args.sorted_ids[up_mb * kBM + up_trow];
     }
+    auto tile_row = [&]() { return MODE == kModeMoeUp ? up_trow : lane_row(s->ti_m64[tislot] != 0); };
+    const int sa_row = max(tile_row(), 0);
     float acc[128];
 #pragma unroll
     for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
     // a warp whose 32 rows are all padding skips the promotion (its outputs are never stored)
-    const bool warp_active = MODE == kModeDense || __any_sync(0xffffffffu, pair >= 0 && pair < P);
+    bool warp_active = true;
+    if (MODE != kModeDense) {
+      const int pr = MODE == kModeMoeUp ? up_pair : (tile_row() >= 0 ? s->ti_pair[tislot][sa_row] : P);
+      warp_active = __any_sync(0xffffffffu, pr >= 0 && pr < P);
+    }
 
     for (int kb = 0; kb < num_kb; ++kb) {
       if (!mbar_wait(&s->sfull[sslot], scphase, abort_flag)) { ok = false; break; }
-      const float sa = s->sa[sslot][has_row ? trow : 0];
+      const float sa = s->sa[sslot][sa_row];
       const float swa = s->sw[sslot][0], swb = s->sw[sslot][1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&s->sempty[sslot]);
@@ -271,8 +279,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         continue;
       }
       const uint32_t tb = lane_base + buf * kBN;
-      // four 32-column chunks; the load of chunk c+1 overlaps the FMAs of chunk c
       float v[2][32];
+      // four 32-column chunks; the load of chunk c+1 overlaps the FMAs of chunk c
       tmem_ld_32x32b_x32(tb + col0, v[0]);
       tmem_wait_ld();
       reg_fence_32(v[0]);
@@ -301,6 +309,17 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
     }
     if (!ok) break;
 
+    const int mb = MODE == kModeMoeUp ? up_mb : s->ti_mb[tislot];
+    const int nt = MODE == kModeMoeUp ? up_nt : s->ti_nt[tislot];
+    const int trow = tile_row();
+    const bool has_row = trow >= 0;
+    const int slot = mb * kBM + (has_row ? trow : 0);
+    int pair = P;
+    float wroute = 0.0f;
+    if (MODE != kModeDense && has_row) {
+      pair = MODE == kModeMoeUp ? up_pair : s->ti_pair[tislot][trow];
+      if (MODE == kModeMoeDown) wroute = s->ti_w[tislot][trow];
+    }
     // Outputs. Dense and gate/up: each thread writes its own row with 32-byte
     // stores (whole sectors) straight from registers.
     if (MODE == kModeDense) {
@@ -339,11 +358,13 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         amax = fmaxf(amax, fabsf(h));
       }
       // the 128-wide requantisation group spans both column halves of the row
-      const int xb = tcount & 1;
+      // the ring slot alternates per tile and its phase every two tiles: the
+      // exchange buffer and its phase follow the same pattern
+      const int xb = tislot;
       s->amax_x[xb][half][row] = amax;
       __syncwarp();
       if (lane == 0) mbar_arrive(&s->xbar[xb]);
-      if (!mbar_wait(&s->xbar[xb], (tcount >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&s->xbar[xb], tiphase, abort_flag)) { ok = false; break; }
       amax = fmaxf(amax, s->amax_x[xb][half ^ 1][row]);
       const float scale = __fdiv_rn(amax, 448.0f);
       const float inv = scale != 0.0f ? __frcp_rn(scale) : 0.0f;
@@ -363,7 +384,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
       }
       if (half == 0 && has_row) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
     } else {
-      // 256 bytes of bf16 per row: a transpose through the warp's staging buffer
+      // weighted rows, 256 bytes of bf16 per row: a transpose through the warp's staging buffer
       // lets each store instruction write 8 whole 64-byte row segments
       const bool valid = pair >= 0 && pair < P;
       if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
@@ -371,6 +392,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
       if (x0 < args.N) {
         const int H = args.N;
         __nv_bfloat16* y = args.ystage;
+        uint8_t* my_staging = staging + ew * kStagingBytes;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
           uint4 d[4];
@@ -394,6 +416,9 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s->tiempty[tislot]);
+    if (++tislot == 2) { tislot = 0; tiphase ^= 1u; }
   }
   if (!ok) abort_all(s);
 }
@@ -422,6 +447,8 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       mbar_init(&s->tfull[i], 1);
       mbar_init(&s->tempty[i], kEpiWarps);
       mbar_init(&s->xbar[i], kEpiWarps);
+      mbar_init(&s->tifull[i], 32);
+      mbar_init(&s->tiempty[i], kEpiWarps + 1);   // the epilogue warps and the MMA issuer
     }
     for (int i = 0; i < kScaleSlots; ++i) {
       mbar_init(&s->sfull[i], 32);
@@ -528,13 +555,14 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
-        int stage = 0, buf = 0;
-        uint32_t sphase = 0, tphase = 0;
+        int stage = 0, buf = 0, tislot = 0;
+        uint32_t sphase = 0, tphase = 0, tiphase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-          int mb, nt;
-          tile_coords<MODE>(args, tile, m_blocks, mb, nt);
-          const uint32_t idesc = moe_half_tile<MODE>(args, mb, P) ? kIdescHalf : kIdesc;
+          if (!mbar_wait(&s->tifull[tislot], tiphase, abort_flag)) { ok = false; break; }
+          const uint32_t idesc = s->ti_m64[tislot] ? kIdescHalf : kIdesc;
+          mbar_arrive(&s->tiempty[tislot]);
+          if (++tislot == 2) { tislot = 0; tiphase ^= 1u; }
           for (int kb = 0; kb < num_kb; ++kb) {
             if (!mbar_wait(&s->full[stage], sphase, abort_flag)) { ok = false; break; }
             if (!mbar_wait(&s->tempty[buf], tphase ^ 1u, abort_flag)) { ok = false; break; }
@@ -555,7 +583,49 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         if (!ok) abort_all(s);
       }
       __syncwarp();
-    }                                    // warp 3 idles
+    } else {
+      // ------------------------------------------------------------ tile info
+      // One tile ahead of the epilogue: the coordinates (for the gate/up GEMM a
+      // scan of the block-expert list), the M=64 decision and the rows' pair ids
+      // and routing weights, so that neither the MMA issuer nor the epilogue
+      // waits on dependent global loads at a tile boundary.
+      int tislot = 0;
+      uint32_t tiphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+        int mb, nt;
+        tile_coords<MODE>(args, tile, m_blocks, mb, nt);
+        int ids[4] = {P, P, P, P};
+        float wts[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (MODE != kModeDense) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ids[i] = args.sorted_ids[mb * kBM + 4 * lane + i];
+          if (MODE == kModeMoeDown) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wts[i] = args.sorted_weights[mb * kBM + 4 * lane + i];
+          }
+        }
+        // A MoE tile whose second half holds only padding slots (an expert's last
+        // block with at most 64 pairs) runs its MMAs with M=64. The sort puts an
+        // expert's pairs before its padding, so slot kBM/2 (lane 16's first row) decides.
+        const int id_half = __shfl_sync(0xffffffffu, ids[0], kBM / 8);
+        const int m64 = (MODE != kModeDense) && (id_half < 0 || id_half >= P);
+        if (!mbar_wait_idle(&s->tiempty[tislot], tiphase ^ 1u, abort_flag)) { ok = false; break; }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          s->ti_pair[tislot][4 * lane + i] = ids[i];
+          s->ti_w[tislot][4 * lane + i] = wts[i];
+        }
+        if (lane == 0) {
+          s->ti_mb[tislot] = mb;
+          s->ti_nt[tislot] = nt;
+          s->ti_m64[tislot] = m64;
+        }
+        mbar_arrive(&s->tifull[tislot]);
+        if (++tislot == 2) { tislot = 0; tiphase ^= 1u; }
+      }
+      if (!ok) abort_all(s);
+    }
   }
 
   tc_fence_before();
