@@ -184,9 +184,10 @@ __device__ __forceinline__ void abort_all(GemmSmem* s) {
 // Writes a warp's 32 rows x 64 bytes (row = lane, data d) to global memory with
 // coalesced stores: each lane puts its row into the warp's shared staging buffer
 // (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3): no bank conflicts), then
-// each of four store instructions writes 8 whole 64-byte row segments.
-// row_addr(r) gives the destination of row r's segment, or nullptr to skip it;
-// every lane calls it (it may use warp shuffles).
+// each of four store instructions writes 8 whole 64-byte row segments. In store
+// i a lane writes 16 bytes of row store_rows_row(i, lane); row_addr(i) gives that
+// row segment's destination, or nullptr to skip it.
+__device__ __forceinline__ int store_rows_row(int i, int lane) { return i * 8 + (lane >> 2); }
 template <typename RowAddr>
 __device__ __forceinline__ void store_rows_64B(uint8_t* staging, int lane, const uint4 (&d)[4], RowAddr row_addr) {
   uint8_t* mine = staging + lane * 64;
@@ -197,9 +198,9 @@ __device__ __forceinline__ void store_rows_64B(uint8_t* staging, int lane, const
   const int c = lane & 3;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = i * 8 + (lane >> 2);
+    const int r = store_rows_row(i, lane);
     const uint4 v = *reinterpret_cast<const uint4*>(staging + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-    uint8_t* dst = row_addr(r);
+    uint8_t* dst = row_addr(i);
     if (dst) *reinterpret_cast<uint4*>(dst + c * 16) = v;
   }
   __syncwarp();
@@ -265,6 +266,10 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
       if (MODE == kModeMoeUp) {
         f0 = sa * swa;
         f1 = sa * swb;
+      } else if (MODE == kModeMoeDown) {
+        // the routing weight rides on every block's scale (read from the ring:
+        // no register held across the loop)
+        f0 = f1 = sa * (half ? swb : swa) * s->ti_w[tislot][sa_row];
       } else {
         f0 = f1 = sa * (half ? swb : swa);
       }
@@ -315,11 +320,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
     const bool has_row = trow >= 0;
     const int slot = mb * kBM + (has_row ? trow : 0);
     int pair = P;
-    float wroute = 0.0f;
-    if (MODE != kModeDense && has_row) {
-      pair = MODE == kModeMoeUp ? up_pair : s->ti_pair[tislot][trow];
-      if (MODE == kModeMoeDown) wroute = s->ti_w[tislot][trow];
-    }
+    if (MODE != kModeDense && has_row) pair = MODE == kModeMoeUp ? up_pair : s->ti_pair[tislot][trow];
     // Outputs. Dense and gate/up: each thread writes its own row with 32-byte
     // stores (whole sectors) straight from registers.
     if (MODE == kModeDense) {
@@ -384,8 +385,9 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
       }
       if (half == 0 && has_row) args.s2[static_cast<size_t>(nt) * args.M + slot] = scale;
     } else {
-      // weighted rows, 256 bytes of bf16 per row: a transpose through the warp's staging buffer
-      // lets each store instruction write 8 whole 64-byte row segments
+      // weighted rows (the weight is already in the sums), 256 bytes of bf16 per
+      // row: a transpose through the warp's staging buffer lets each store
+      // instruction write 8 whole 64-byte row segments
       const bool valid = pair >= 0 && pair < P;
       if (!valid && pair != P) raise_device_error(FP8MOE_DEVERR_PAIR_ID);
       const int x0 = nt * kBN + half * 128;
@@ -393,6 +395,13 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         const int H = args.N;
         __nv_bfloat16* y = args.ystage;
         uint8_t* my_staging = staging + ew * kStagingBytes;
+        // destinations of the four rows this lane stores (null for padding rows)
+        uint8_t* dst[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pr = __shfl_sync(0xffffffffu, pair, store_rows_row(i, lane));
+          dst[i] = (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x0) : nullptr;
+        }
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
           uint4 d[4];
@@ -402,17 +411,12 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int j = ch * 32 + u * 8 + 2 * q;
-              const __nv_bfloat162 pk = __floats2bfloat162_rn(wroute * acc[j], wroute * acc[j + 1]);
+              const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[j], acc[j + 1]);
               w[q] = *reinterpret_cast<const uint32_t*>(&pk);
             }
             d[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          const int x = x0 + ch * 32;
-          store_rows_64B(my_staging, lane, d, [&](int r) -> uint8_t* {
-            const int pr = __shfl_sync(0xffffffffu, pair, r);
-            return (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x)
-                                       : nullptr;
-          });
+          store_rows_64B(my_staging, lane, d, [&](int i) -> uint8_t* { return dst[i] ? dst[i] + ch * 64 : nullptr; });
         }
       }
     }
