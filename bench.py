@@ -37,7 +37,8 @@ sys.path.insert(0, ROOT)
 
 from fp8_block_scaled_biased_b200 import inputs as I  # noqa: E402
 
-WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED, "profile": I.PROFILE}
+WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED, "profile": I.PROFILE,
+             "prefill_ep8": I.PREFILL_EP8}
 L2_FLUSH_BYTES = 256 << 20
 METRIC = "fused FP8-blockscale MoE layer tokens/s and TFLOPS at 1 B200; % of FP8/HBM roofline"
 EXPERT_W1_BYTES = lambda c: 2 * c.I * c.H + (2 * c.I // 128) * (c.H // 128) * 4   # noqa: E731
@@ -155,10 +156,24 @@ def max_over_ranks(x, world):
     return t.item()
 
 
-def layer_work(cfg, ids):
-    """Algorithmic FLOPs and HBM bytes of one layer forward (padding excluded)."""
-    n_e = int(torch.unique(ids).numel())
-    P = cfg.T * cfg.K
+def ep_config(cfg):
+    """Config keys of an expert-parallel workload: which rank's experts the layer keeps."""
+    if cfg.ep_ranks <= 0:
+        return {}
+    m = I.expert_mask(cfg)
+    kept = torch.nonzero(m).flatten()
+    return {"expert_parallel": f"rank {cfg.ep_rank} of {cfg.ep_ranks}: experts {int(kept[0])}-{int(kept[-1])} "
+                               "(expert_mask), partial output of every token"}
+
+
+def layer_work(cfg, ids, mask=None):
+    """Algorithmic FLOPs and HBM bytes of one layer forward (padding excluded). With an
+    expert mask only the kept experts' pairs count."""
+    flat = ids.flatten().long().cpu()
+    if mask is not None:
+        flat = flat[mask.cpu().bool()[flat]]
+    n_e = int(torch.unique(flat).numel())
+    P = int(flat.numel())
     flops = 2 * P * cfg.H * 2 * cfg.I + 2 * P * cfg.I * cfg.H
     act_bytes = cfg.T * cfg.E * 4 + cfg.E * 4 + cfg.T * cfg.H * 2 + cfg.T * cfg.H * 2
     layer_bytes = n_e * (EXPERT_W1_BYTES(cfg) + EXPERT_W2_BYTES(cfg)) + act_bytes
@@ -265,22 +280,24 @@ def run_ours(args, world, rank, local):
     layer = MoELayer(cfg, dev).load_synthetic_weights()
     act = I.moe_activations(cfg)
     logits, bias, x = act.logits.to(dev), act.bias.to(dev), act.x.to(dev)
+    mask = I.expert_mask(cfg)
+    mask_dev = mask.to(dev) if mask is not None else None
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     # warm-up (also the first, eager pass through every entry point)
     for _ in range(args.warmup):
-        layer.forward(logits, bias, x)
+        layer.forward(logits, bias, x, expert_mask=mask_dev)
     torch.cuda.synchronize()
     assert B.device_status() == 0, "device error word set during warm-up"
-    work = layer_work(cfg, layer.topk_ids)
+    work = layer_work(cfg, layer.topk_ids, mask)
 
     B.timing_enable(True)          # before capture, so the graph holds the per-kernel event records
     graph = None
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            layer.forward(logits, bias, x)
+            layer.forward(logits, bias, x, expert_mask=mask_dev)
         graph.replay()
         torch.cuda.synchronize()
 
@@ -288,7 +305,7 @@ def run_ours(args, world, rank, local):
         if graph is not None:
             graph.replay()
         else:
-            layer.forward(logits, bias, x)
+            layer.forward(logits, bias, x, expert_mask=mask_dev)
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -380,7 +397,7 @@ def run_ours(args, world, rank, local):
                    "topk_group": cfg.TG, "topk": cfg.K, "I": cfg.I, "block_m": layer.block_m,
                    "parallelism": f"dp{world} (replicated layer, token batches per GPU)",
                    "l2": "flushed between steps (256 MB write); touched expert weights exceed L2 anyway",
-                   "cuda_graph": graph is not None},
+                   "cuda_graph": graph is not None, **ep_config(cfg)},
         "tflops": work["flops"] * world / (ms_per_step * 1e-3) / 1e12,
         "layer_roofline": {"ms": t_layer_roof, "frac": t_layer_roof / ms_per_step,
                            "flops": work["flops"], "bytes": work["layer_bytes"],
@@ -426,7 +443,8 @@ class OracleSample:
         self.logits, self.x = act.logits[tok].contiguous(), act.x[tok].contiguous()
         self.bias = act.bias
         _, ids = O.biased_grouped_topk(self.logits, self.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
-        self.experts = torch.unique(ids).tolist()
+        self.mask = I.expert_mask(cfg)
+        self.experts = [e for e in torch.unique(ids).tolist() if self.mask is None or self.mask[e]]
         self.weights = {}
         for e in self.experts:
             w1 = I.expert_weight_raw(cfg, "w1", e, device).cpu()
@@ -438,9 +456,9 @@ class OracleSample:
         O, cfg = self.O, self.cfg
         t0 = time.perf_counter()
         w, ids = O.biased_grouped_topk(self.logits, self.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
-        O.align_sort(ids, w, cfg.E, 128)
+        O.align_sort(ids, w, cfg.E, 128, expert_mask=self.mask)
         a8, asc = O.quant_1x128(self.x)
-        O.moe_layer(a8, asc, ids, w, self.weights.__getitem__)
+        O.moe_layer(a8, asc, ids, w, self.weights.__getitem__, expert_mask=self.mask)
         return time.perf_counter() - t0
 
 
@@ -597,7 +615,7 @@ def run_reference(args, world, rank):
         "dtype": "f64 (fp32 where a routing choice or an FP8 code is decided)",
         "data": "synthetic (seeded)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "groups": cfg.G,
-                   "topk_group": cfg.TG, "topk": cfg.K, "I": cfg.I},
+                   "topk_group": cfg.TG, "topk": cfg.K, "I": cfg.I, **ep_config(cfg)},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
                          "sample": f"{n} seeded tokens of {cfg.name} per step ({len(runner.experts)} experts, "
                                    "weights quantised before timing)"},

@@ -29,10 +29,14 @@ _SIGNATURES = {
     "fp8moe_timing_last": (_c_int, [ctypes.POINTER(ctypes.c_float)]),
     "moe_biased_grouped_topk": (_c_int, [_p, _c_int, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                          _c_int, _c_float, _p]),
+    "moe_biased_grouped_topk_bf16": (_c_int, [_p, _c_int, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                              _c_int, _c_int, _c_float, _p]),
     "moe_align_sort_capacity": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "moe_align_sort_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "moe_align_sort": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_size, _p,
                                 _c_size, _p]),
+    "moe_align_sort_masked": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p, _c_size,
+                                       _p, _c_size, _p]),
     "fp8_per_token_group_quant": (_c_int, [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_int, _p]),
     "fp8_per_block_quant": (_c_int, [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _p]),
     "fp8_blockscale_gemm": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _p]),
@@ -128,8 +132,12 @@ def moe_block_m() -> int:
 
 def moe_biased_grouped_topk(gating_output, correction_bias, topk_weights, topk_ids, num_expert_group, topk_group,
                             need_renorm, routed_scaling_factor=1.0):
-    """Writes topk_weights fp32 [T, topk] and topk_ids int32 [T, topk] (row stride may exceed topk)."""
-    _cuda(gating_output, torch.float32, "gating_output")
+    """Writes topk_weights fp32 [T, topk] and topk_ids int32 [T, topk] (row stride may exceed topk).
+
+    gating_output is fp32 or bf16 [T, E]; bf16 logits take moe_biased_grouped_topk_bf16."""
+    if gating_output.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"gating_output must be torch.float32 or torch.bfloat16, got {gating_output.dtype}")
+    _cuda(gating_output, gating_output.dtype, "gating_output")
     _cuda(correction_bias, torch.float32, "correction_bias")
     _cuda(topk_weights, torch.float32, "topk_weights")
     _cuda(topk_ids, torch.int32, "topk_ids")
@@ -138,11 +146,13 @@ def moe_biased_grouped_topk(gating_output, correction_bias, topk_weights, topk_i
     ld_out = _row_major(topk_weights, "topk_weights")
     if _row_major(topk_ids, "topk_ids") != ld_out:
         raise ValueError("topk_weights and topk_ids must share a row stride")
-    rc = load_library().moe_biased_grouped_topk(
+    lib = load_library()
+    fn = lib.moe_biased_grouped_topk_bf16 if gating_output.dtype == torch.bfloat16 else lib.moe_biased_grouped_topk
+    rc = fn(
         _ptr(gating_output), _row_major(gating_output, "gating_output"), _ptr(correction_bias.contiguous()),
         _ptr(topk_weights), _ptr(topk_ids), ld_out, T, E, topk, num_expert_group, topk_group, int(bool(need_renorm)),
         float(routed_scaling_factor), _stream())
-    _check("moe_biased_grouped_topk", rc)
+    _check(fn.__name__, rc)
 
 
 def moe_align_sort_capacity(T, topk, E, block_m):
@@ -177,8 +187,14 @@ def moe_align_sort_workspace_bytes(T, topk, E, block_m):
 
 
 def moe_align_sort(topk_ids, topk_weights, num_experts, block_m, out: SortedPairs | None = None,
-                   workspace=None) -> SortedPairs:
+                   workspace=None, expert_mask=None) -> SortedPairs:
+    """Sorted, block-padded pair list. expert_mask (int32 [E] on the device, nonzero = keep)
+    drops the pairs of masked-out experts (moe_align_sort_masked)."""
     _cuda(topk_ids, torch.int32, "topk_ids")
+    if expert_mask is not None:
+        _cuda(expert_mask, torch.int32, "expert_mask")
+        if expert_mask.numel() != num_experts or not expert_mask.is_contiguous():
+            raise ValueError("expert_mask must be a contiguous int32 tensor of num_experts entries")
     _cuda(topk_weights, torch.float32, "topk_weights")
     T, topk = topk_ids.shape
     ld = _row_major(topk_ids, "topk_ids")
@@ -190,10 +206,17 @@ def moe_align_sort(topk_ids, topk_weights, num_experts, block_m, out: SortedPair
     if workspace is None:
         workspace = torch.empty(lib.moe_align_sort_workspace(T, topk, num_experts, block_m), dtype=torch.uint8,
                                 device=topk_ids.device)
-    rc = lib.moe_align_sort(_ptr(topk_ids), _ptr(topk_weights), ld, T, topk, num_experts, block_m,
-                            _ptr(out.sorted_ids), _ptr(out.sorted_weights), _ptr(out.sorted_expert_ids),
-                            _ptr(out.num_valid_ids), out.capacity, _ptr(workspace), workspace.numel(), _stream())
-    _check("moe_align_sort", rc)
+    if expert_mask is None:
+        rc = lib.moe_align_sort(_ptr(topk_ids), _ptr(topk_weights), ld, T, topk, num_experts, block_m,
+                                _ptr(out.sorted_ids), _ptr(out.sorted_weights), _ptr(out.sorted_expert_ids),
+                                _ptr(out.num_valid_ids), out.capacity, _ptr(workspace), workspace.numel(), _stream())
+        _check("moe_align_sort", rc)
+    else:
+        rc = lib.moe_align_sort_masked(_ptr(topk_ids), _ptr(topk_weights), ld, T, topk, num_experts, block_m,
+                                       _ptr(expert_mask), _ptr(out.sorted_ids), _ptr(out.sorted_weights),
+                                       _ptr(out.sorted_expert_ids), _ptr(out.num_valid_ids), out.capacity,
+                                       _ptr(workspace), workspace.numel(), _stream())
+        _check("moe_align_sort_masked", rc)
     return out
 
 

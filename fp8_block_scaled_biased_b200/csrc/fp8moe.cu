@@ -163,7 +163,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // scales (capacity rows), the slot-ordered re-quantised intermediate and its
 // scales, and the weighted down-projection rows of every pair (by pair id).
 struct MoeWorkspace {
-  size_t a8s_off, s1s_off, a2_off, s2_off, y_off, total;
+  size_t a8s_off, s1s_off, a2_off, s2_off, y_off, flag_off, total;
 };
 
 MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I) {
@@ -179,6 +179,7 @@ MoeWorkspace moe_workspace_layout(size_t capacity, int T, int topk, int H, int I
   w.a2_off = take(capacity * static_cast<size_t>(I));
   w.s2_off = take(static_cast<size_t>(I / 128) * capacity * sizeof(float));
   w.y_off = take(static_cast<size_t>(T) * topk * H * sizeof(__nv_bfloat16));
+  w.flag_off = take(16 + static_cast<size_t>(T) * topk);   // listed-pair count, then 1 flag per pair
   w.total = off;
   return w;
 }
@@ -208,6 +209,58 @@ int choose_group_m(int n_tiles) {
 }
 
 }  // namespace
+
+// Routing for fp32 or bf16 logits (the two C entry points below).
+template <typename LT>
+static int route_impl(const char* name, const LT* gating_output, int ld_in, const float* correction_bias,
+                      float* topk_weights, int32_t* topk_ids, int ld_out, int T, int E, int topk,
+                      int num_expert_group, int topk_group, int need_renorm, float routed_scaling_factor,
+                      void* stream) {
+  if (T < 0) return fail(FP8MOE_EINVAL, "T must be >= 0 (got %d)", T);
+  if (E < 1 || E > 32 * kRouteMaxPerLane) return fail(FP8MOE_EUNSUPPORTED, "E must be in [1, 512] (got %d)", E);
+  if (num_expert_group < 1 || num_expert_group > 32 || E % num_expert_group != 0)
+    return fail(FP8MOE_EINVAL, "num_expert_group must divide E and be <= 32 (E=%d, groups=%d)", E,
+                num_expert_group);
+  if (topk_group < 1 || topk_group > num_expert_group)
+    return fail(FP8MOE_EINVAL, "topk_group must be in [1, num_expert_group] (got %d)", topk_group);
+  const int per_group = E / num_expert_group;
+  if (topk < 1 || topk > 32 || topk > topk_group * per_group)
+    return fail(FP8MOE_EINVAL, "topk must be in [1, min(32, topk_group*E/groups)] (got %d)", topk);
+  if (ld_in < E) return fail(FP8MOE_EINVAL, "ld_in (%d) < E (%d)", ld_in, E);
+  if (ld_out < topk) return fail(FP8MOE_EINVAL, "ld_out (%d) < topk (%d)", ld_out, topk);
+  if (T == 0) return FP8MOE_OK;
+  if (!gating_output || !correction_bias || !topk_weights || !topk_ids)
+    return fail(FP8MOE_EINVAL, "null pointer argument");
+  // experts per lane: the smallest divisor of the group size that covers E with 32 lanes
+  const int need = (E + 31) / 32;
+  int per_lane = 0;
+  for (int d = need; d <= per_group; ++d)
+    if (per_group % d == 0) {
+      per_lane = d;
+      break;
+    }
+  if (per_lane == 0 || per_lane > kRouteMaxPerLane)
+    return fail(FP8MOE_EUNSUPPORTED, "group size %d cannot be split over 32 lanes", per_group);
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const dim3 grid((T + kRouteWarps - 1) / kRouteWarps);
+  const uintptr_t lg = reinterpret_cast<uintptr_t>(gating_output);
+  const int vec4 = (ld_in % 4 == 0) && (lg % (4 * sizeof(LT)) == 0) && aligned16(correction_bias);
+  auto launch = [&](auto kernel) {
+    kernel<<<grid, 32 * kRouteWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+        gating_output, ld_in, correction_bias, topk_weights, topk_ids, ld_out, T, E, topk, num_expert_group,
+        topk_group, need_renorm ? 1 : 0, routed_scaling_factor, per_lane, vec4);
+  };
+  switch (per_lane) {
+    case 1: launch(route_kernel<1, LT>); break;
+    case 2: launch(route_kernel<2, LT>); break;
+    case 4: launch(route_kernel<4, LT>); break;
+    case 8: launch(route_kernel<8, LT>); break;
+    case 16: launch(route_kernel<16, LT>); break;
+    default: launch(route_kernel<0, LT>); break;
+  }
+  return check_launch(name);
+}
 
 extern "C" {
 
@@ -266,49 +319,17 @@ int fp8moe_device_status(void* stream) {
 int moe_biased_grouped_topk(const float* gating_output, int ld_in, const float* correction_bias, float* topk_weights,
                             int32_t* topk_ids, int ld_out, int T, int E, int topk, int num_expert_group,
                             int topk_group, int need_renorm, float routed_scaling_factor, void* stream) {
-  if (T < 0) return fail(FP8MOE_EINVAL, "T must be >= 0 (got %d)", T);
-  if (E < 1 || E > 32 * kRouteMaxPerLane) return fail(FP8MOE_EUNSUPPORTED, "E must be in [1, 512] (got %d)", E);
-  if (num_expert_group < 1 || num_expert_group > 32 || E % num_expert_group != 0)
-    return fail(FP8MOE_EINVAL, "num_expert_group must divide E and be <= 32 (E=%d, groups=%d)", E,
-                num_expert_group);
-  if (topk_group < 1 || topk_group > num_expert_group)
-    return fail(FP8MOE_EINVAL, "topk_group must be in [1, num_expert_group] (got %d)", topk_group);
-  const int per_group = E / num_expert_group;
-  if (topk < 1 || topk > 32 || topk > topk_group * per_group)
-    return fail(FP8MOE_EINVAL, "topk must be in [1, min(32, topk_group*E/groups)] (got %d)", topk);
-  if (ld_in < E) return fail(FP8MOE_EINVAL, "ld_in (%d) < E (%d)", ld_in, E);
-  if (ld_out < topk) return fail(FP8MOE_EINVAL, "ld_out (%d) < topk (%d)", ld_out, topk);
-  if (T == 0) return FP8MOE_OK;
-  if (!gating_output || !correction_bias || !topk_weights || !topk_ids)
-    return fail(FP8MOE_EINVAL, "null pointer argument");
-  // experts per lane: the smallest divisor of the group size that covers E with 32 lanes
-  const int need = (E + 31) / 32;
-  int per_lane = 0;
-  for (int d = need; d <= per_group; ++d)
-    if (per_group % d == 0) {
-      per_lane = d;
-      break;
-    }
-  if (per_lane == 0 || per_lane > kRouteMaxPerLane)
-    return fail(FP8MOE_EUNSUPPORTED, "group size %d cannot be split over 32 lanes", per_group);
-  int sms = 0;
-  if (int rc = device_setup(&sms)) return rc;
-  const dim3 grid((T + kRouteWarps - 1) / kRouteWarps);
-  const int vec4 = (ld_in % 4 == 0) && aligned16(gating_output) && aligned16(correction_bias);
-  auto launch = [&](auto kernel) {
-    kernel<<<grid, 32 * kRouteWarps, 0, static_cast<cudaStream_t>(stream)>>>(
-        gating_output, ld_in, correction_bias, topk_weights, topk_ids, ld_out, T, E, topk, num_expert_group,
-        topk_group, need_renorm ? 1 : 0, routed_scaling_factor, per_lane, vec4);
-  };
-  switch (per_lane) {
-    case 1: launch(route_kernel<1>); break;
-    case 2: launch(route_kernel<2>); break;
-    case 4: launch(route_kernel<4>); break;
-    case 8: launch(route_kernel<8>); break;
-    case 16: launch(route_kernel<16>); break;
-    default: launch(route_kernel<0>); break;
-  }
-  return check_launch("moe_biased_grouped_topk");
+  return route_impl("moe_biased_grouped_topk", gating_output, ld_in, correction_bias, topk_weights, topk_ids,
+                    ld_out, T, E, topk, num_expert_group, topk_group, need_renorm, routed_scaling_factor, stream);
+}
+
+int moe_biased_grouped_topk_bf16(const uint16_t* gating_output, int ld_in, const float* correction_bias,
+                                 float* topk_weights, int32_t* topk_ids, int ld_out, int T, int E, int topk,
+                                 int num_expert_group, int topk_group, int need_renorm,
+                                 float routed_scaling_factor, void* stream) {
+  return route_impl("moe_biased_grouped_topk_bf16", reinterpret_cast<const __nv_bfloat16*>(gating_output), ld_in,
+                    correction_bias, topk_weights, topk_ids, ld_out, T, E, topk, num_expert_group, topk_group,
+                    need_renorm, routed_scaling_factor, stream);
 }
 
 // ------------------------------------------------------------------ S2 align/sort
@@ -324,9 +345,10 @@ size_t moe_align_sort_workspace(int T, int topk, int E, int block_m) {
   return round_up(nchunks * E * sizeof(int32_t), 256) + round_up(E * sizeof(int32_t), 256);
 }
 
-int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, int T, int topk, int E, int block_m,
-                   int32_t* sorted_ids, float* sorted_weights, int32_t* sorted_expert_ids, int32_t* num_valid_ids,
-                   size_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
+int moe_align_sort_masked(const int32_t* topk_ids, const float* topk_weights, int ld, int T, int topk, int E,
+                          int block_m, const int32_t* expert_mask, int32_t* sorted_ids, float* sorted_weights,
+                          int32_t* sorted_expert_ids, int32_t* num_valid_ids, size_t capacity, void* workspace,
+                          size_t workspace_bytes, void* stream) {
   if (T < 0 || topk < 1) return fail(FP8MOE_EINVAL, "T >= 0 and topk >= 1 required");
   if (E < 1 || E > kSortMaxExperts) return fail(FP8MOE_EUNSUPPORTED, "E must be in [1, %d]", kSortMaxExperts);
   if (block_m < 1 || block_m > 1024) return fail(FP8MOE_EINVAL, "block_m must be in [1, 1024]");
@@ -346,14 +368,14 @@ int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, i
   const int nchunks = (pairs + kSortChunk - 1) / kSortChunk;
   if (nchunks <= 1) {                   // one chunk: count, scan and scatter in a single CTA
     sort_small_kernel<<<1, kSortChunk, static_cast<size_t>(kSortWarps + 2) * E * sizeof(int), st>>>(
-        topk_ids, topk_weights, ld, T, topk, E, block_m, sorted_ids, sorted_weights, sorted_expert_ids,
+        topk_ids, topk_weights, ld, T, topk, E, expert_mask, block_m, sorted_ids, sorted_weights, sorted_expert_ids,
         num_valid_ids);
     return check_launch("moe_align_sort (single chunk)");
   }
   int32_t* counts = static_cast<int32_t*>(workspace);                       // [nchunks][E]
   int32_t* seg_start = counts + round_up(static_cast<size_t>(nchunks) * E * sizeof(int32_t), 256) / sizeof(int32_t);
   if (nchunks > 0) {
-    sort_count_kernel<<<nchunks, kSortChunk, E * sizeof(int), st>>>(topk_ids, ld, T, topk, E, counts);
+    sort_count_kernel<<<nchunks, kSortChunk, E * sizeof(int), st>>>(topk_ids, ld, T, topk, E, expert_mask, counts);
     if (int rc = check_launch("moe_align_sort (count)")) return rc;
   }
   sort_scan_kernel<<<1, kSortChunk, 2 * E * sizeof(int), st>>>(counts, seg_start, nchunks, T, topk, E, block_m,
@@ -362,10 +384,17 @@ int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, i
   if (int rc = check_launch("moe_align_sort (scan)")) return rc;
   if (nchunks > 0) {
     sort_scatter_kernel<<<nchunks, kSortChunk, static_cast<size_t>(kSortWarps) * E * sizeof(int), st>>>(
-        topk_ids, topk_weights, ld, T, topk, E, counts, seg_start, sorted_ids, sorted_weights);
+        topk_ids, topk_weights, ld, T, topk, E, expert_mask, counts, seg_start, sorted_ids, sorted_weights);
     if (int rc = check_launch("moe_align_sort (scatter)")) return rc;
   }
   return FP8MOE_OK;
+}
+
+int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld, int T, int topk, int E, int block_m,
+                   int32_t* sorted_ids, float* sorted_weights, int32_t* sorted_expert_ids, int32_t* num_valid_ids,
+                   size_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
+  return moe_align_sort_masked(topk_ids, topk_weights, ld, T, topk, E, block_m, nullptr, sorted_ids, sorted_weights,
+                               sorted_expert_ids, num_valid_ids, capacity, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------ S3 quant
@@ -456,6 +485,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (fc2_smooth_scale) return fail(FP8MOE_EUNSUPPORTED, "fc2_smooth_scale must be NULL");
   if (block_m != kBM) return fail(FP8MOE_EUNSUPPORTED, "block_m must be %d (got %d)", kBM, block_m);
   if (T < 0 || E < 1 || topk < 1 || topk > E) return fail(FP8MOE_EINVAL, "bad T, E or topk");
+  if (topk > 32) return fail(FP8MOE_EUNSUPPORTED, "topk must be <= 32 (got %d)", topk);
   if (H < 128 || I < 128 || H % 128 || I % 128)
     return fail(FP8MOE_EUNSUPPORTED, "H and I must be positive multiples of 128 (H=%d, I=%d)", H, I);
   if (static_cast<long long>(T) * topk >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "T*topk too large");
@@ -480,6 +510,8 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   uint8_t* a2 = ws + lay.a2_off;
   float* s2 = reinterpret_cast<float*>(ws + lay.s2_off);
   __nv_bfloat16* ystage = reinterpret_cast<__nv_bfloat16*>(ws + lay.y_off);
+  int* n_present = reinterpret_cast<int*>(ws + lay.flag_off);
+  uint8_t* pair_flag = ws + lay.flag_off + 16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   CUtensorMap m_a8s, m_w1, m_a2, m_w2;
@@ -488,10 +520,14 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (int rc = make_operand_map(&m_a2, a2, capacity, I)) return rc;
   if (int rc = make_operand_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
 
+  // pairs absent from the sorted list (a masked-out expert, a dropped id) keep
+  // flag 0 and add nothing in the combine
+  if (cudaMemsetAsync(n_present, 0, 16 + static_cast<size_t>(T) * topk, st) != cudaSuccess)
+    return check_launch("fused_moe (pair flags)");
   timing_record(0, st);
   moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, sorted_expert_ids,
                                                             num_valid_ids, T, topk, H, static_cast<int>(capacity),
-                                                            a8s, s1s);
+                                                            a8s, s1s, pair_flag, n_present);
   if (int rc = check_launch("fused_moe (gather)")) return rc;
   timing_record(1, st);
 
@@ -541,7 +577,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
 
   const size_t threads = static_cast<size_t>(T) * (H / 8);
   moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
-      ystage, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
+      ystage, pair_flag, n_present, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
   if (int rc = check_launch("fused_moe (combine)")) return rc;
   timing_record(4, st);
   return FP8MOE_OK;

@@ -17,15 +17,22 @@ namespace fp8moe {
 constexpr int kMoeBlockRows = 128;            // rows per sorted block (the GEMM tile's M)
 
 // Copies each sorted slot's token row of a8 [T, H] (and its H/128 scales from
-// a1_scale [H/128, T]) into slot order. Padding slots are skipped: the GEMMs
-// treat rows independently and never store padding rows.
+// a1_scale [H/128, T]) into slot order, sets pair_flag[p] = 1 for every pair p
+// in the list and adds the number of listed pairs to *n_present (the caller
+// zeroes both first). Padding slots are skipped: the GEMMs treat rows
+// independently and never store padding rows.
 constexpr int kGatherWarps = 8;
 __global__ void __launch_bounds__(32 * kGatherWarps)
 moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_scale,
                   const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ sorted_expert_ids,
                   const int32_t* __restrict__ num_valid_ids, int T, int topk, int H, int cap,
-                  uint8_t* __restrict__ a8s, float* __restrict__ s1s) {
+                  uint8_t* __restrict__ a8s, float* __restrict__ s1s, uint8_t* __restrict__ pair_flag,
+                  int* __restrict__ n_present) {
+  __shared__ int cta_present;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) cta_present = 0;
+  __syncthreads();
+  int warp_present = 0;
   const int P = T * topk;
   const int nv = min(max(*num_valid_ids, 0), cap);
   // The gate/up GEMM's tile order needs each expert's blocks to be contiguous, as the
@@ -37,6 +44,8 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
   for (int slot = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); slot < nv; slot += gridDim.x * kGatherWarps) {
     const int sid = sorted_ids[slot];
     if (sid < 0 || sid >= P) continue;
+    if (lane == 0) pair_flag[sid] = 1;
+    ++warp_present;
     const int t = sid / topk;
     const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
     uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
@@ -56,6 +65,9 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
       }
     }
   }
+  if (lane == 0 && warp_present) atomicAdd(&cta_present, warp_present);
+  __syncthreads();
+  if (threadIdx.x == 0 && cta_present) atomicAdd(n_present, cta_present);
   // scales: one lane per slot of a 32-slot group, so each store instruction
   // writes 128 contiguous bytes of a row of s1s
   const int nwarps = gridDim.x * kGatherWarps;
@@ -70,9 +82,13 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
 }
 
 // out[t, :] = bf16( y[t*K + 0] + y[t*K + 1] + ... + y[t*K + K-1] ), fp32 adds in
-// slot order k (the routing weight is already in y). One thread per 8 columns.
+// slot order k over the pairs whose flag is set (the routing weight is already
+// in y; a pair absent from the sorted list has no row). When every pair is
+// listed (*n_present == T*K, one cached load) the flags are not read. One thread
+// per 8 columns.
 __global__ void __launch_bounds__(256)
-moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
+moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, const uint8_t* __restrict__ pair_flag,
+                   const int* __restrict__ n_present, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
   const int cpr = H / 8;
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<size_t>(T) * cpr) return;
@@ -83,7 +99,7 @@ moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, int T, int K, int H
 #pragma unroll
   for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
   // fp32 sum in k order (0.0f + y0 == y0 exactly, so the order is fixed from the first term)
-  for (int k = 0; k < K; ++k) {
+  auto add_row = [&](int k) {
     const uint4 v = *reinterpret_cast<const uint4*>(y + static_cast<size_t>(k) * H);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -92,6 +108,12 @@ moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, int T, int K, int H
       sum[2 * u] += f.x;
       sum[2 * u + 1] += f.y;
     }
+  };
+  if (*n_present == T * K) {
+    for (int k = 0; k < K; ++k) add_row(k);
+  } else {
+    for (int k = 0; k < K; ++k)
+      if (pair_flag[static_cast<size_t>(t) * K + k]) add_row(k);
   }
   __align__(16) __nv_bfloat162 pk[4];
 #pragma unroll

@@ -6,7 +6,11 @@
 // routed_scaling_factor. Scoring (DeepSeek-V3 style): s = sigmoid(logit),
 // b = s + correction_bias; group score = sum of the group's two largest b;
 // ties go to the lower group / expert index; weights are the unbiased s.
+// The logits are fp32 or bf16 (the page's routing test runs over a dtype);
+// bf16 values widen to fp32 exactly, so both take the same fp32 sequence.
 #pragma once
+
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 
@@ -40,6 +44,17 @@ __device__ __forceinline__ float sigmoid_f32_recipe(float x) {
   return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_f32_recipe(-x)));
 }
 
+__device__ __forceinline__ float logit_f32(float v) { return v; }
+__device__ __forceinline__ float logit_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+// four consecutive logits: 16-byte aligned for fp32, 8-byte aligned for bf16
+__device__ __forceinline__ float4 load_logits4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 load_logits4(const __nv_bfloat16* p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 // (value desc, index asc) ordering: does (v1, i1) rank before (v0, i0)?
 __device__ __forceinline__ bool ranks_before(float v1, int i1, float v0, int i0) {
   return v1 > v0 || (v1 == v0 && i1 < i0);
@@ -48,11 +63,11 @@ __device__ __forceinline__ bool ranks_before(float v1, int i1, float v0, int i0)
 // Each lane owns `per_lane` consecutive experts; a lane's experts never span two
 // groups (per_lane divides the group size), so a group is lanes_per_group
 // consecutive lanes. PL > 0 fixes per_lane at compile time (the usual 1, 2, 4,
-// 8, 16); PL == 0 takes it from the argument. vec4: rows and bias allow 16-byte
-// loads of a lane's experts (PL % 4 == 0 only).
-template <int PL>
+// 8, 16); PL == 0 takes it from the argument. vec4: rows and bias allow vector
+// loads of four of a lane's experts (PL % 4 == 0 only). LT: fp32 or bf16 logits.
+template <int PL, typename LT>
 __global__ void __launch_bounds__(32 * kRouteWarps)
-route_kernel(const float* __restrict__ logits, int ld_in, const float* __restrict__ bias,
+route_kernel(const LT* __restrict__ logits, int ld_in, const float* __restrict__ bias,
              float* __restrict__ topk_w, int32_t* __restrict__ topk_ids, int ld_out, int T, int E, int K,
              int G, int TG, int renorm, float factor, int per_lane_arg, int vec4) {
   constexpr int kPL = PL > 0 ? PL : kRouteMaxPerLane;
@@ -65,12 +80,12 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
   const int e0 = lane * per_lane;
 
   float s[kPL], b[kPL];
-  const float* row = logits + static_cast<size_t>(t) * ld_in;
+  const LT* row = logits + static_cast<size_t>(t) * ld_in;
   float x[kPL], bs[kPL];
   if (PL % 4 == 0 && PL > 0 && vec4 && e0 < E) {
 #pragma unroll
     for (int j = 0; j < kPL; j += 4) {
-      const float4 xv = __ldg(reinterpret_cast<const float4*>(row + e0 + j));
+      const float4 xv = load_logits4(row + e0 + j);
       const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + e0 + j));
       x[j] = xv.x; x[j + 1] = xv.y; x[j + 2] = xv.z; x[j + 3] = xv.w;
       bs[j] = bv.x; bs[j + 1] = bv.y; bs[j + 2] = bv.z; bs[j + 3] = bv.w;
@@ -80,7 +95,7 @@ route_kernel(const float* __restrict__ logits, int ld_in, const float* __restric
     for (int j = 0; j < kPL; ++j) {
       const int e = e0 + j;
       const bool in = j < per_lane && e < E;
-      x[j] = in ? __ldg(row + e) : 0.0f;
+      x[j] = in ? logit_f32(__ldg(row + e)) : 0.0f;
       bs[j] = in ? __ldg(bias + e) : 0.0f;
     }
   }

@@ -5,7 +5,9 @@
 // sorted_expert_ids, num_valid_ids). Layout: pair (t, k) is the flat id
 // p = t*topk + k; experts ascending, pairs ascending inside an expert, each
 // segment padded to a multiple of block_m with id T*topk and weight 0; one
-// expert id per block; experts without pairs get no block.
+// expert id per block; experts without pairs get no block. An optional expert
+// mask (the expert_mask argument of the page's asm_moe call: the experts this
+// GPU holds under expert parallelism) drops the pairs of masked-out experts.
 //
 // Three kernels over chunks of kSortChunk consecutive pairs (one CTA each):
 //   1. sort_count_kernel: per-chunk expert histogram -> counts[chunk][E];
@@ -26,25 +28,32 @@ constexpr int kSortChunk = 1024;                 // pairs per CTA = threads per 
 constexpr int kSortWarps = kSortChunk / 32;
 constexpr int kSortMaxExperts = 1024;
 
-__device__ __forceinline__ int read_pair_expert(const int32_t* ids, int ld, int K, int p, int E) {
+// Expert of pair p: kDropInvalid for an id outside [0, E) (flagged by the
+// caller), kDropMasked for an expert that mask (if any) excludes.
+constexpr int kDropInvalid = -1;
+constexpr int kDropMasked = -2;
+__device__ __forceinline__ int read_pair_expert(const int32_t* ids, int ld, int K, int p, int E,
+                                                const int32_t* mask) {
   const int t = p / K, k = p - t * K;
   const int e = ids[static_cast<size_t>(t) * ld + k];
-  return (e >= 0 && e < E) ? e : -1;
+  if (e < 0 || e >= E) return kDropInvalid;
+  return (mask && mask[e] == 0) ? kDropMasked : e;
 }
 
 // 1. counts[c][e] = pairs of chunk c routed to expert e.
 __global__ void __launch_bounds__(kSortChunk)
-sort_count_kernel(const int32_t* __restrict__ ids, int ld, int T, int K, int E, int32_t* __restrict__ counts) {
+sort_count_kernel(const int32_t* __restrict__ ids, int ld, int T, int K, int E, const int32_t* __restrict__ mask,
+                  int32_t* __restrict__ counts) {
   extern __shared__ int sm_cnt[];
   const int P = T * K;
   for (int e = threadIdx.x; e < E; e += kSortChunk) sm_cnt[e] = 0;
   __syncthreads();
   const int p = blockIdx.x * kSortChunk + threadIdx.x;
   if (p < P) {
-    const int e = read_pair_expert(ids, ld, K, p, E);
+    const int e = read_pair_expert(ids, ld, K, p, E, mask);
     if (e >= 0)
       atomicAdd(&sm_cnt[e], 1);
-    else
+    else if (e == kDropInvalid)
       raise_device_error(FP8MOE_DEVERR_EXPERT_ID);
   }
   __syncthreads();
@@ -114,13 +123,13 @@ sort_scan_kernel(int32_t* __restrict__ counts, int32_t* __restrict__ seg_start, 
 // 3. Stable scatter of chunk blockIdx.x.
 __global__ void __launch_bounds__(kSortChunk)
 sort_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, int ld, int T, int K, int E,
-                    const int32_t* __restrict__ before, const int32_t* __restrict__ seg_start,
+                    const int32_t* __restrict__ mask, const int32_t* __restrict__ before, const int32_t* __restrict__ seg_start,
                     int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w) {
   extern __shared__ int warp_cnt[];   // [kSortWarps][E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = T * K;
   const int p = blockIdx.x * kSortChunk + tid;
-  const int e = (p < P) ? read_pair_expert(ids, ld, K, p, E) : -1;
+  const int e = (p < P) ? read_pair_expert(ids, ld, K, p, E, mask) : kDropInvalid;
   float wv = 0.0f;
   if (e >= 0) {
     const int t = p / K, k = p - t * K;
@@ -155,7 +164,7 @@ sort_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w
 // Shared memory: total[E], start[E], warp_cnt[kSortWarps][E].
 __global__ void __launch_bounds__(kSortChunk)
 sort_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, int ld, int T, int K, int E,
-                  int block_m, int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w,
+                  const int32_t* __restrict__ mask, int block_m, int32_t* __restrict__ sorted_ids, float* __restrict__ sorted_w,
                   int32_t* __restrict__ sorted_e, int32_t* __restrict__ num_valid) {
   extern __shared__ int sm_small[];
   int* total = sm_small;
@@ -167,14 +176,14 @@ sort_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, 
   for (int i = tid; i < kSortWarps * E; i += kSortChunk) warp_cnt[i] = 0;
   __syncthreads();
   const int p = tid;
-  int e = -1;
+  int e = kDropInvalid;
   float wv = 0.0f;
   if (p < P) {
-    e = read_pair_expert(ids, ld, K, p, E);
+    e = read_pair_expert(ids, ld, K, p, E, mask);
     if (e >= 0) {
       const int t = p / K, k = p - t * K;
       wv = w[static_cast<size_t>(t) * ld + k];
-    } else {
+    } else if (e == kDropInvalid) {
       raise_device_error(FP8MOE_DEVERR_EXPERT_ID);
     }
   }

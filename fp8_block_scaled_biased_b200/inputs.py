@@ -48,10 +48,21 @@ class MoEConfig:
     x_std: float = 1.0
     w_std: float = 0.02
     seed: int = 0
+    ep_ranks: int = 0           # > 0: the layer as expert-parallel rank ep_rank of ep_ranks sees it
+    ep_rank: int = 0
 
     @property
     def P(self) -> int:
         return self.T * self.K
+
+
+def expert_mask(cfg: MoEConfig):
+    """int32 [E] on the CPU: the experts rank ep_rank holds when E experts are split into
+    ep_ranks contiguous ranges (None when the config is not expert-parallel)."""
+    if cfg.ep_ranks <= 0:
+        return None
+    per = cfg.E // cfg.ep_ranks
+    return (torch.arange(cfg.E) // per == cfg.ep_rank).to(torch.int32)
 
 
 @dataclass(frozen=True)
@@ -76,7 +87,12 @@ GEMM = GemmConfig("gemm_m2048_n4096_k7168", M=2048, N=4096, K=7168)
 # L2) and 512 tokens: small enough for full-set profiler captures.
 PROFILE = MoEConfig("profile_t512_h7168_e32", T=512, H=7168, E=32, G=8, TG=4, K=8, I=2048)
 
-MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, PROFILE)}
+# The prefill batch as expert-parallel rank 0 of 8 computes it: experts 0-31 only
+# (the expert_mask of the page's asm_moe call), a partial output for all 4096 tokens.
+PREFILL_EP8 = MoEConfig("prefill_ep8_rank0_t4096_h7168_e256", T=4096, H=7168, E=256, G=8, TG=4, K=8, I=2048,
+                        ep_ranks=8, ep_rank=0)
+
+MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, PROFILE, PREFILL_EP8)}
 
 
 @dataclass

@@ -63,8 +63,12 @@ class MoELayer:
             B.fp8_per_block_quant(raw2, q=self.w2[e], scales=self.w2_scale[e])
         return self
 
-    def forward(self, logits, bias, x):
-        """logits fp32 [T, E], bias fp32 [E], x bf16 [T, H] (all on the device) -> bf16 [T, H]."""
+    def forward(self, logits, bias, x, expert_mask=None):
+        """logits fp32 or bf16 [T, E], bias fp32 [E], x bf16 [T, H] (all on the device) -> bf16 [T, H].
+
+        expert_mask: optional int32 [E] on the device (nonzero = an expert this GPU holds).
+        The result is then the sum over the kept experts' pairs only, the partial output
+        of one expert-parallel rank."""
         cfg = self.cfg
         T = x.shape[0]
         if T != self.max_tokens:
@@ -77,7 +81,7 @@ class MoELayer:
             self._join.record(self._side)
         B.moe_biased_grouped_topk(logits, bias, self.topk_w, self.topk_ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
         B.moe_align_sort(self.topk_ids, self.topk_w, cfg.E, self.block_m, out=self.sorted,
-                         workspace=self.sort_workspace)
+                         workspace=self.sort_workspace, expert_mask=expert_mask)
         main.wait_event(self._join)
         B.fused_moe_fp8_blockscale_g1u1(self.out, self.a8, self.w1, self.w2, self.sorted, cfg.K, self.a8_scale,
                                         self.w1_scale, self.w2_scale, workspace=self.workspace)

@@ -107,6 +107,21 @@ int moe_biased_grouped_topk(const float* gating_output, int ld_in,
                             float routed_scaling_factor, void* stream);
 
 /*
+ * S1 with bf16 router logits (the page's routing test runs over a `dtype`).
+ * gating_output is bf16 [T, E] (uint16_t bit patterns), row stride ld_in >= E;
+ * everything else as moe_biased_grouped_topk. A bf16 logit widens to fp32
+ * exactly, so the result equals moe_biased_grouped_topk on the widened logits
+ * bit for bit.
+ */
+int moe_biased_grouped_topk_bf16(const uint16_t* gating_output, int ld_in,
+                                 const float* correction_bias,
+                                 float* topk_weights, int32_t* topk_ids,
+                                 int ld_out, int T, int E, int topk,
+                                 int num_expert_group, int topk_group,
+                                 int need_renorm, float routed_scaling_factor,
+                                 void* stream);
+
+/*
  * S2 - MoE align/sort.  (MoE Sorting: moe_sorting(topk_ids, topk_weights, E,
  *      model_dim, dtype) -> sorted_token_ids, sorted_weight_buf,
  *      sorted_expert_ids, num_valid_ids.)
@@ -131,6 +146,24 @@ int moe_align_sort(const int32_t* topk_ids, const float* topk_weights, int ld,
                    int32_t* sorted_expert_ids, int32_t* num_valid_ids,
                    size_t capacity, void* workspace, size_t workspace_bytes,
                    void* stream);
+
+/*
+ * S2 with an expert mask: the expert_mask argument of the page's asm_moe call
+ * (section "MoE Sorting"), the hook for expert parallelism. expert_mask is a
+ * DEVICE int32 [E]; pairs routed to an expert e with expert_mask[e] == 0 are
+ * dropped (no slot, no flag), so the sorted list holds only this GPU's experts.
+ * NULL keeps every expert (= moe_align_sort). Everything else as
+ * moe_align_sort, including the capacity and workspace queries.
+ * fused_moe_fp8_blockscale_g1u1 on the result gives the sum over the kept
+ * experts only: the partial output an expert-parallel rank contributes.
+ */
+int moe_align_sort_masked(const int32_t* topk_ids, const float* topk_weights,
+                          int ld, int T, int topk, int E, int block_m,
+                          const int32_t* expert_mask,
+                          int32_t* sorted_ids, float* sorted_weights,
+                          int32_t* sorted_expert_ids, int32_t* num_valid_ids,
+                          size_t capacity, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /*
  * S3 - dynamic per-token-group FP8 quantisation (1 x group).
@@ -204,8 +237,12 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B,
  *   y_p = blockscale(a2, w2[e]),
  *   out[t] = bf16( sum_{k=0..topk-1} bf16(w_{t,k} * y_{t,k}) ), each weighted
  * row rounded once to bf16 and the topk rows summed in fp32 in k order, which
- * makes the output independent of scheduling (deterministic).
+ * makes the output independent of scheduling (deterministic). A pair absent
+ * from the sorted list (its expert masked out by moe_align_sort_masked, or its
+ * id dropped as out of range) adds nothing; a token with no pair present gets
+ * a zero row.
  * Limits: scale_blk_n == scale_blk_k == 128; H % 128 == 0; I % 128 == 0;
+ * topk <= 32;
  * fc2_smooth_scale must be NULL (the pages do not define it); workspace >=
  * fused_moe_fp8_blockscale_g1u1_workspace(); capacity >= the sort's padded
  * length.

@@ -301,7 +301,8 @@ def biased_grouped_topk(logits: torch.Tensor, bias: torch.Tensor, topk: int,
 # MoE align / sort
 # ---------------------------------------------------------------------------
 
-def align_sort(topk_ids: torch.Tensor, topk_weights: torch.Tensor, num_experts: int, block_m: int):
+def align_sort(topk_ids: torch.Tensor, topk_weights: torch.Tensor, num_experts: int, block_m: int,
+               expert_mask: torch.Tensor | None = None):
     """Group the T*topk token-expert pairs by expert into block_m-padded segments.
 
     From the page's section "MoE Sorting" (moe_sorting returns sorted_token_ids,
@@ -310,7 +311,10 @@ def align_sort(topk_ids: torch.Tensor, topk_weights: torch.Tensor, num_experts: 
     p = t*topk + k; experts in ascending order, each expert's pairs in ascending
     p, each segment padded to a multiple of block_m with the sentinel id T*topk
     and weight 0; experts with no pair get no block; one expert id per block;
-    num_valid_ids = total padded length.
+    num_valid_ids = total padded length. Ids outside [0, num_experts) belong to
+    no expert and are left out. expert_mask (the expert_mask argument of the
+    page's asm_moe call, the experts one GPU holds under expert parallelism):
+    when given, experts e with expert_mask[e] == 0 are left out with their pairs.
 
     Returns (sorted_ids int32 [L], sorted_weights fp32 [L], sorted_expert_ids
     int32 [L/block_m], num_valid_ids int).
@@ -321,6 +325,8 @@ def align_sort(topk_ids: torch.Tensor, topk_weights: torch.Tensor, num_experts: 
     wflat = topk_weights.reshape(-1).to(F32)
     ids_out, w_out, blocks = [], [], []
     for e in range(num_experts):
+        if expert_mask is not None and int(expert_mask[e]) == 0:
+            continue
         pairs = torch.nonzero(flat == e).flatten()          # ascending p
         cnt = pairs.numel()
         if cnt == 0:
@@ -381,13 +387,16 @@ def moe_combine(y_slots: torch.Tensor, topk_weights: torch.Tensor) -> torch.Tens
     return out
 
 
-def moe_layer(a8, a_scale, topk_ids, topk_weights, get_expert, tokens=None, round_bf16=True):
+def moe_layer(a8, a_scale, topk_ids, topk_weights, get_expert, tokens=None, round_bf16=True, expert_mask=None):
     """Fused g1u1 MoE of quantised hidden states a8 [T, H] (scales [T, H/128]).
 
     get_expert(e) -> (w1q [2I, H], w1s [2I/128, H/128], w2q [H, I], w2s [H/128, I/128])
     supplies expert e's quantised weights (so that large layers can be streamed).
     tokens: optional sorted list of token indices to compute (others are skipped);
     the result then has one row per listed token.
+    expert_mask: optional [E]; when given, only pairs whose id e lies in [0, E)
+    with expert_mask[e] != 0 contribute (the others add nothing), which is the
+    partial output of one expert-parallel rank.
     Output: bf16-rounded (fp64 tensor of bf16 values) or unrounded fp64.
     """
     T, K = topk_ids.shape
@@ -396,6 +405,8 @@ def moe_layer(a8, a_scale, topk_ids, topk_weights, get_expert, tokens=None, roun
     H = a8.shape[1]
     y = torch.zeros(len(tok), K, H, dtype=F64)
     for e in torch.unique(ids).tolist():
+        if expert_mask is not None and not (0 <= e < len(expert_mask) and int(expert_mask[e]) != 0):
+            continue
         rows, slots = torch.nonzero(ids == e, as_tuple=True)
         w1q, w1s, w2q, w2s = get_expert(e)
         t = tok[rows]

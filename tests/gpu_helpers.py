@@ -31,8 +31,9 @@ def assert_moe_close(gpu_out, ref):
     return dmax, mre
 
 
-def oracle_moe_rows(cfg, act, tokens, device="cuda"):
-    """Oracle routing on all tokens, then the MoE output of the listed tokens (fp64, unrounded)."""
+def oracle_moe_rows(cfg, act, tokens, device="cuda", expert_mask=None):
+    """Oracle routing on all tokens, then the MoE output of the listed tokens (fp64, unrounded).
+    expert_mask (CPU int32 [E]): only the kept experts' pairs contribute."""
     w, ids = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
     a8, asc = O.quant_1x128(act.x[tokens] if tokens is not None else act.x)
     sub_ids = ids[tokens] if tokens is not None else ids
@@ -44,5 +45,5 @@ def oracle_moe_rows(cfg, act, tokens, device="cuda"):
             cache[e] = oracle_expert(cfg, e, device)
         return cache.pop(e)
 
-    out = O.moe_layer(a8, asc, sub_ids, sub_w, get, round_bf16=False)
+    out = O.moe_layer(a8, asc, sub_ids, sub_w, get, round_bf16=False, expert_mask=expert_mask)
     return out, w, ids

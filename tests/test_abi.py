@@ -129,3 +129,18 @@ def test_binding_fails_loudly_without_library(tmp_path):
             B.load_library(str(tmp_path / "missing.so"))
     finally:
         B._lib = saved
+
+
+def test_bf16_routing_and_masked_sort_reject_bad_arguments(lib):
+    rc, msg = _rc(lib, "moe_biased_grouped_topk_bf16", P, 16, P, P, P, 3, 16, 16, 4, 4, 2, 1, 2.5, None)
+    assert rc == 1 and "ld_out" in msg
+    rc, _ = _rc(lib, "moe_biased_grouped_topk_bf16", P, 1024, P, P, P, 8, 16, 1024, 8, 8, 4, 1, 2.5, None)
+    assert rc == 2
+    rc, _ = _rc(lib, "moe_biased_grouped_topk_bf16", P, 16, P, P, P, 4, 0, 16, 4, 4, 2, 1, 2.5, None)
+    assert rc == 0
+    cap = lib.moe_align_sort_capacity(16, 4, 16, 4)
+    rc, msg = _rc(lib, "moe_align_sort_masked", P, P, 4, 16, 4, 16, 4, P, P, P, P, P, cap - 1, None, 0, None)
+    assert rc == 1 and "capacity" in msg
+    ws = lib.moe_align_sort_workspace(16, 4, 16, 4)
+    rc, msg = _rc(lib, "moe_align_sort_masked", P, P, 4, 16, 4, 16, 4, P, P, P, P, P, cap, P, ws - 1, None)
+    assert rc == 3 and "workspace" in msg

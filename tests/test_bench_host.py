@@ -90,3 +90,21 @@ def test_reference_arm_gemm_line():
     d = _json_lines(r.stdout)[-1]
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["config"]["workload"] == I.GEMM.name
+
+
+def test_layer_work_counts_only_kept_experts_under_a_mask():
+    cfg = I.TINY
+    ids = torch.tensor([[0, 1, 2, 3]] * cfg.T, dtype=torch.int32)
+    mask = torch.tensor([1, 0, 1] + [0] * (cfg.E - 3), dtype=torch.int32)
+    w = bench.layer_work(cfg, ids, mask)
+    P = cfg.T * 2                                   # experts 0 and 2 only
+    assert w["n_experts"] == 2
+    assert w["flops"] == 2 * P * cfg.H * 2 * cfg.I + 2 * P * cfg.I * cfg.H
+
+
+def test_expert_parallel_workload_mask_and_config():
+    cfg = I.PREFILL_EP8
+    m = I.expert_mask(cfg)
+    assert m.dtype == torch.int32 and int(m.sum()) == cfg.E // 8 and bool(m[:32].all())
+    assert I.expert_mask(I.PREFILL) is None and bench.ep_config(I.PREFILL) == {}
+    assert "rank 0 of 8" in bench.ep_config(cfg)["expert_parallel"]

@@ -128,3 +128,31 @@ def test_moe_layer_equivariances_and_zero_input():
     # token subsets give the same rows
     sub = [1, 5, 9]
     assert torch.equal(O.moe_layer(a8, asc, ids, w, get, tokens=sub, round_bf16=False), out[sub])
+
+
+def test_moe_layer_expert_mask_against_dense_evaluation_and_partition():
+    """Expert mask (the page's asm_moe expert_mask): only kept experts' pairs add. Pinned to the
+    dense all-expert evaluation restricted to kept experts, and to the expert-parallel identity:
+    the partial outputs of a partition of the experts sum to the unmasked output."""
+    cfg = I.MoEConfig("pin_mask", T=12, H=256, E=8, G=2, TG=2, K=3, I=128, seed=6)
+    act = I.moe_activations(cfg)
+    w, ids, a8, asc, ex = _layer(cfg, act)
+    get = lambda e: ex[e]
+    mask = torch.tensor([1, 0, 0, 1, 1, 0, 1, 0], dtype=torch.int32)
+    out = O.moe_layer(a8, asc, ids, w, get, round_bf16=False, expert_mask=mask)
+    ys = torch.stack([_dense_ffn(a8, asc, ex[e]) for e in range(cfg.E)])
+    ref = torch.zeros(cfg.T, cfg.H, dtype=torch.float64)
+    for t in range(cfg.T):
+        for k in range(cfg.K):
+            e = ids[t, k].item()
+            if mask[e]:
+                ref[t] += w[t, k].double() * ys[e, t]
+    scale = ref.abs().max().item()
+    d = (out - ref).abs()
+    assert d.max() <= 2e-3 * scale and d.sum() <= 1e-4 * ref.abs().sum()
+    full = O.moe_layer(a8, asc, ids, w, get, round_bf16=False)
+    parts = [O.moe_layer(a8, asc, ids, w, get, round_bf16=False,
+                         expert_mask=(torch.arange(cfg.E) % 4 == r).int()) for r in range(4)]
+    assert torch.allclose(sum(parts), full, rtol=1e-12, atol=1e-12 * full.abs().max().item())
+    none = O.moe_layer(a8, asc, ids, w, get, expert_mask=torch.zeros(cfg.E, dtype=torch.int32))
+    assert (none == 0).all()

@@ -36,3 +36,36 @@ def test_sort_matches_stable_argsort_and_invariants(T, K, E, BM, seed):
 def test_sort_empty_input():
     sid, sw, se, nv = O.align_sort(torch.empty(0, 4, dtype=torch.int32), torch.empty(0, 4), 8, 16)
     assert nv == 0 and sid.numel() == 0 and se.numel() == 0
+
+
+@pytest.mark.parametrize("T,K,E,BM,seed", [(64, 8, 256, 16, 1), (300, 8, 32, 128, 2), (16, 4, 16, 4, 5)])
+def test_masked_sort_is_the_stable_sort_of_the_kept_pairs(T, K, E, BM, seed):
+    """Expert mask (the page's asm_moe expert_mask): the kept pairs in a library stable argsort."""
+    g = torch.Generator().manual_seed(seed)
+    ids = torch.randint(0, E, (T, K), generator=g, dtype=torch.int32)
+    w = torch.rand(T, K, generator=g)
+    mask = (torch.rand(E, generator=g) < 0.4).int()
+    mask[ids[0, 0]] = 1
+    sid, sw, se, nv = O.align_sort(ids, w, E, BM, expert_mask=mask)
+    P = T * K
+    flat = ids.flatten().long()
+    kept = torch.nonzero(mask.bool()[flat]).flatten()
+    order = kept[torch.argsort(flat[kept], stable=True)]
+    valid = sid < P
+    assert torch.equal(sid[valid].long(), order)
+    assert torch.equal(sw[valid], w.flatten()[order])
+    cnt = torch.bincount(flat[kept], minlength=E)
+    assert nv == int(((cnt + BM - 1) // BM * BM).sum())
+    assert set(se.tolist()) <= set(torch.nonzero(mask).flatten().tolist())
+    # an all-ones mask is no mask
+    full = O.align_sort(ids, w, E, BM)
+    ones = O.align_sort(ids, w, E, BM, expert_mask=torch.ones(E, dtype=torch.int32))
+    assert all(torch.equal(a, b) for a, b in zip(full[:3], ones[:3])) and full[3] == ones[3]
+
+
+def test_sort_leaves_out_of_range_ids():
+    ids = torch.tensor([[0, 5], [-1, 1], [7, 0]], dtype=torch.int32)     # E = 4: 5, -1 and 7 belong to no expert
+    w = torch.tensor([[0.1, 0.2], [0.3, 0.4], [0.5, 0.6]])
+    sid, sw, se, nv = O.align_sort(ids, w, 4, 2)
+    assert sid.tolist() == [0, 5, 3, 6] and se.tolist() == [0, 1] and nv == 4
+    assert sw.tolist()[:2] == pytest.approx([0.1, 0.6]) and sw[3] == 0 and sw[2] == pytest.approx(0.4)
