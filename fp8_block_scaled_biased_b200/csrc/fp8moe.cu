@@ -101,7 +101,7 @@ int device_setup(int* sm_count) {
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown>();
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kSortWarps * kSortMaxExperts * static_cast<int>(sizeof(int)));
+                               static_cast<int>(sort_scatter_smem(kSortMaxExperts)));
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(sort_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (kSortWarps + 2) * kSortMaxExperts * static_cast<int>(sizeof(int)));
@@ -342,7 +342,7 @@ size_t moe_align_sort_workspace(int T, int topk, int E, int block_m) {
   if (T < 0 || topk < 1 || E < 1 || block_m < 1) return 0;
   const size_t pairs = static_cast<size_t>(T) * topk;
   const size_t nchunks = (pairs + kSortChunk - 1) / kSortChunk;
-  return round_up(nchunks * E * sizeof(int32_t), 256) + round_up(E * sizeof(int32_t), 256);
+  return round_up(nchunks * E * sizeof(int32_t), 256);
 }
 
 int moe_align_sort_masked(const int32_t* topk_ids, const float* topk_weights, int ld, int T, int topk, int E,
@@ -359,34 +359,26 @@ int moe_align_sort_masked(const int32_t* topk_ids, const float* topk_weights, in
   if (!sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids || (T > 0 && (!topk_ids || !topk_weights)))
     return fail(FP8MOE_EINVAL, "null pointer argument");
   const size_t need = moe_align_sort_workspace(T, topk, E, block_m);
-  if (!workspace || workspace_bytes < need)
+  if (need > 0 && (!workspace || workspace_bytes < need))
     return fail(FP8MOE_EWORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int pairs = T * topk;
   const int nchunks = (pairs + kSortChunk - 1) / kSortChunk;
-  if (nchunks <= 1) {                   // one chunk: count, scan and scatter in a single CTA
+  if (nchunks <= 1) {                   // one chunk: count, offsets and scatter in a single CTA
     sort_small_kernel<<<1, kSortChunk, static_cast<size_t>(kSortWarps + 2) * E * sizeof(int), st>>>(
         topk_ids, topk_weights, ld, T, topk, E, expert_mask, block_m, sorted_ids, sorted_weights, sorted_expert_ids,
         num_valid_ids);
     return check_launch("moe_align_sort (single chunk)");
   }
   int32_t* counts = static_cast<int32_t*>(workspace);                       // [nchunks][E]
-  int32_t* seg_start = counts + round_up(static_cast<size_t>(nchunks) * E * sizeof(int32_t), 256) / sizeof(int32_t);
-  if (nchunks > 0) {
-    sort_count_kernel<<<nchunks, kSortChunk, E * sizeof(int), st>>>(topk_ids, ld, T, topk, E, expert_mask, counts);
-    if (int rc = check_launch("moe_align_sort (count)")) return rc;
-  }
-  sort_scan_kernel<<<1, kSortChunk, 2 * E * sizeof(int), st>>>(counts, seg_start, nchunks, T, topk, E, block_m,
-                                                               sorted_ids, sorted_weights, sorted_expert_ids,
-                                                               num_valid_ids);
-  if (int rc = check_launch("moe_align_sort (scan)")) return rc;
-  if (nchunks > 0) {
-    sort_scatter_kernel<<<nchunks, kSortChunk, static_cast<size_t>(kSortWarps) * E * sizeof(int), st>>>(
-        topk_ids, topk_weights, ld, T, topk, E, expert_mask, counts, seg_start, sorted_ids, sorted_weights);
-    if (int rc = check_launch("moe_align_sort (scatter)")) return rc;
-  }
+  sort_count_kernel<<<nchunks, kSortChunk, E * sizeof(int), st>>>(topk_ids, ld, T, topk, E, expert_mask, counts);
+  if (int rc = check_launch("moe_align_sort (count)")) return rc;
+  sort_scatter_kernel<<<nchunks, kSortChunk, sort_scatter_smem(E), st>>>(
+      topk_ids, topk_weights, ld, T, topk, E, expert_mask, block_m, counts, nchunks, sorted_ids, sorted_weights,
+      sorted_expert_ids, num_valid_ids);
+  if (int rc = check_launch("moe_align_sort (scatter)")) return rc;
   return FP8MOE_OK;
 }
 

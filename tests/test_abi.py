@@ -75,7 +75,7 @@ def test_sort_rejects_bad_arguments(lib):
     rc, _ = _rc(lib, "moe_align_sort", P, P, 4, 16, 4, 2000, 4, P, P, P, P, 10 ** 6, None, 0, None)
     assert rc == 2
     ws = lib.moe_align_sort_workspace(16, 4, 16, 4)
-    assert ws >= 16 * 4                                   # per-chunk histogram + segment starts
+    assert ws >= 16 * 4                                   # per-chunk histograms
     rc, msg = _rc(lib, "moe_align_sort", P, P, 4, 16, 4, 16, 4, P, P, P, P, cap, P, ws - 1, None)
     assert rc == 3 and "workspace" in msg
 
