@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 from fp8_block_scaled_biased_b200 import inputs as I  # noqa: E402
 
 WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED, "profile": I.PROFILE,
-             "prefill_ep8": I.PREFILL_EP8}
+             "prefill_ep8": I.PREFILL_EP8, "prefill_tp8": I.PREFILL_TP8}
 L2_FLUSH_BYTES = 256 << 20
 METRIC = "fused FP8-blockscale MoE layer tokens/s and TFLOPS at 1 B200; % of FP8/HBM roofline"
 EXPERT_W1_BYTES = lambda c: 2 * c.I * c.H + (2 * c.I // 128) * (c.H // 128) * 4   # noqa: E731
@@ -157,13 +157,18 @@ def max_over_ranks(x, world):
 
 
 def ep_config(cfg):
-    """Config keys of an expert-parallel workload: which rank's experts the layer keeps."""
-    if cfg.ep_ranks <= 0:
-        return {}
-    m = I.expert_mask(cfg)
-    kept = torch.nonzero(m).flatten()
-    return {"expert_parallel": f"rank {cfg.ep_rank} of {cfg.ep_ranks}: experts {int(kept[0])}-{int(kept[-1])} "
-                               "(expert_mask), partial output of every token"}
+    """Config keys of an expert- or tensor-parallel workload: which part of the layer it keeps."""
+    out = {}
+    if cfg.ep_ranks > 0:
+        kept = torch.nonzero(I.expert_mask(cfg)).flatten()
+        out["expert_parallel"] = (f"rank {cfg.ep_rank} of {cfg.ep_ranks}: experts {int(kept[0])}-{int(kept[-1])} "
+                                  "(expert_mask), partial output of every token")
+    if cfg.tp_ranks > 0:
+        Is = cfg.I // cfg.tp_ranks
+        out["tensor_parallel"] = (f"rank {cfg.tp_rank} of {cfg.tp_ranks}: intermediate columns "
+                                  f"{cfg.tp_rank * Is}-{(cfg.tp_rank + 1) * Is - 1} of every expert, partial output "
+                                  "of every token")
+    return out
 
 
 PREHEAT_SECONDS = 0.4
@@ -295,6 +300,9 @@ def run_ours(args, world, rank, local):
     cfg = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     layer = MoELayer(cfg, dev).load_synthetic_weights()
+    if cfg.tp_ranks > 0:                            # keep only this rank's shard of the weights
+        layer = layer.tp_shard(cfg.tp_rank, cfg.tp_ranks)
+        torch.cuda.empty_cache()
     act = I.moe_activations(cfg)
     logits, bias, x = act.logits.to(dev), act.bias.to(dev), act.x.to(dev)
     mask = I.expert_mask(cfg)
@@ -307,7 +315,7 @@ def run_ours(args, world, rank, local):
         layer.forward(logits, bias, x, expert_mask=mask_dev)
     torch.cuda.synchronize()
     assert B.device_status() == 0, "device error word set during warm-up"
-    work = layer_work(cfg, layer.topk_ids, mask)
+    work = layer_work(layer.cfg, layer.topk_ids, mask)
 
     # Two graphs of the forward: a plain one for the timed steps, and one holding the
     # fused call's per-kernel event records (the records add gaps between kernels,
@@ -493,7 +501,14 @@ class OracleSample:
         for e in self.experts:
             w1 = I.expert_weight_raw(cfg, "w1", e, device).cpu()
             w2 = I.expert_weight_raw(cfg, "w2", e, device).cpu()
-            self.weights[e] = (*O.quant_128x128(w1), *O.quant_128x128(w2))
+            w1q, w1s, w2q, w2s = (*O.quant_128x128(w1), *O.quant_128x128(w2))
+            if cfg.tp_ranks > 0:                    # the rank's intermediate columns only
+                Is, nb, r = cfg.I // cfg.tp_ranks, cfg.I // cfg.tp_ranks // 128, cfg.tp_rank
+                rows = torch.cat([torch.arange(r * Is, (r + 1) * Is), cfg.I + torch.arange(r * Is, (r + 1) * Is)])
+                brows = torch.cat([torch.arange(r * nb, (r + 1) * nb),
+                                   cfg.I // 128 + torch.arange(r * nb, (r + 1) * nb)])
+                w1q, w1s, w2q, w2s = w1q[rows], w1s[brows], w2q[:, r * Is:(r + 1) * Is], w2s[:, r * nb:(r + 1) * nb]
+            self.weights[e] = (w1q, w1s, w2q, w2s)
         self.n = n_tokens
 
     def step(self):

@@ -50,6 +50,8 @@ class MoEConfig:
     seed: int = 0
     ep_ranks: int = 0           # > 0: the layer as expert-parallel rank ep_rank of ep_ranks sees it
     ep_rank: int = 0
+    tp_ranks: int = 0           # > 0: tensor-parallel shard tp_rank of tp_ranks (over I)
+    tp_rank: int = 0
 
     @property
     def P(self) -> int:
@@ -92,7 +94,12 @@ PROFILE = MoEConfig("profile_t512_h7168_e32", T=512, H=7168, E=32, G=8, TG=4, K=
 PREFILL_EP8 = MoEConfig("prefill_ep8_rank0_t4096_h7168_e256", T=4096, H=7168, E=256, G=8, TG=4, K=8, I=2048,
                         ep_ranks=8, ep_rank=0)
 
-MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, PROFILE, PREFILL_EP8)}
+# The prefill batch on tensor-parallel rank 0 of 8 (the pages' TP8 run): every expert's
+# intermediate columns 0-255, a partial output for all 4096 tokens.
+PREFILL_TP8 = MoEConfig("prefill_tp8_rank0_t4096_h7168_e256", T=4096, H=7168, E=256, G=8, TG=4, K=8, I=2048,
+                        tp_ranks=8, tp_rank=0)
+
+MOE_CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, PROFILE, PREFILL_EP8, PREFILL_TP8)}
 
 
 @dataclass

@@ -9,6 +9,8 @@ then fmoe_fp8_blockscale_g1u1. Every step is a call into the CUDA library.
 """
 from __future__ import annotations
 
+import dataclasses
+
 import torch
 
 from . import binding as B
@@ -62,6 +64,29 @@ class MoELayer:
             raw2 = I.expert_weight_raw(self.cfg, "w2", e, self.device)
             B.fp8_per_block_quant(raw2, q=self.w2[e], scales=self.w2_scale[e])
         return self
+
+    def tp_shard(self, rank: int, nranks: int) -> "MoELayer":
+        """Tensor-parallel shard `rank` of `nranks` (the pages' TP8 deployment): every expert's
+        intermediate columns [rank*I/n, (rank+1)*I/n), i.e. those gate and up rows of w1 and
+        those columns of w2, with their 128x128 block scales, copied into a new layer. Its
+        forward gives that rank's partial output; the ranks' partial outputs sum to the whole
+        layer's, because the 1x128 requantisation groups of the intermediate lie inside a
+        shard (I/n must be a multiple of 128). Routing and the activation quantisation are
+        the same on every rank."""
+        cfg = self.cfg
+        if nranks < 1 or not 0 <= rank < nranks or cfg.I % (128 * nranks):
+            raise ValueError(f"I={cfg.I} cannot be split into {nranks} shards of whole 128-column blocks")
+        Is, I0 = cfg.I // nranks, rank * (cfg.I // nranks)
+        nb, b0, nbI = Is // 128, I0 // 128, cfg.I // 128
+        scfg = dataclasses.replace(cfg, name=f"{cfg.name}_tp{nranks}_rank{rank}", I=Is)
+        shard = MoELayer(scfg, self.device, max_tokens=self.max_tokens)
+        shard.w1[:, :Is].copy_(self.w1[:, I0:I0 + Is])
+        shard.w1[:, Is:].copy_(self.w1[:, cfg.I + I0:cfg.I + I0 + Is])
+        shard.w1_scale[:, :nb].copy_(self.w1_scale[:, b0:b0 + nb])
+        shard.w1_scale[:, nb:].copy_(self.w1_scale[:, nbI + b0:nbI + b0 + nb])
+        shard.w2.copy_(self.w2[:, :, I0:I0 + Is])
+        shard.w2_scale.copy_(self.w2_scale[:, :, b0:b0 + nb])
+        return shard
 
     def forward(self, logits, bias, x, expert_mask=None):
         """logits fp32 or bf16 [T, E], bias fp32 [E], x bf16 [T, H] (all on the device) -> bf16 [T, H].

@@ -108,3 +108,12 @@ def test_expert_parallel_workload_mask_and_config():
     assert m.dtype == torch.int32 and int(m.sum()) == cfg.E // 8 and bool(m[:32].all())
     assert I.expert_mask(I.PREFILL) is None and bench.ep_config(I.PREFILL) == {}
     assert "rank 0 of 8" in bench.ep_config(cfg)["expert_parallel"]
+
+
+def test_tensor_parallel_workload_config_and_oracle_sample():
+    assert "intermediate columns 0-255" in bench.ep_config(I.PREFILL_TP8)["tensor_parallel"]
+    cfg = I.MoEConfig("host_tp2", T=8, H=256, E=4, G=2, TG=1, K=2, I=256, tp_ranks=2, tp_rank=1)
+    r = bench.OracleSample(cfg, 2, device="cpu")
+    assert r.step() > 0
+    w1q, w1s, w2q, w2s = r.weights[r.experts[0]]
+    assert w1q.shape == (256, 256) and w1s.shape == (2, 2) and w2q.shape == (256, 128) and w2s.shape == (2, 1)

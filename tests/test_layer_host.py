@@ -1,0 +1,44 @@
+"""Host-side logic of layer.py on the CPU: the tensor-parallel shard's weight slices."""
+import pytest
+import torch
+
+from fp8_block_scaled_biased_b200 import binding as B
+from fp8_block_scaled_biased_b200 import inputs as I
+from fp8_block_scaled_biased_b200.layer import MoELayer
+
+
+def _random_layer(cfg):
+    layer = MoELayer(cfg, "cpu")
+    g = torch.Generator().manual_seed(3)
+    for t in (layer.w1, layer.w2):
+        t.view(torch.uint8).copy_(torch.randint(0, 256, t.shape, generator=g, dtype=torch.uint8))
+    for t in (layer.w1_scale, layer.w2_scale):
+        t.copy_(torch.rand(t.shape, generator=g))
+    return layer
+
+
+@pytest.mark.parametrize("n", [2, 4])
+def test_tp_shard_takes_the_gate_up_rows_and_down_columns_of_its_slice(n):
+    cfg = I.MoEConfig("host_tp", T=4, H=256, E=3, G=1, TG=1, K=2, I=512)
+    layer = _random_layer(cfg)
+    Is = cfg.I // n
+    for r in range(n):
+        sh = layer.tp_shard(r, n)
+        assert sh.cfg.I == Is and sh.w1.shape == (cfg.E, 2 * Is, cfg.H) and sh.w2.shape == (cfg.E, cfg.H, Is)
+        for e in range(cfg.E):
+            for i in range(Is):                       # row by row: gate row r*Is+i, up row I+r*Is+i
+                assert torch.equal(sh.w1[e, i].view(torch.uint8), layer.w1[e, r * Is + i].view(torch.uint8))
+                assert torch.equal(sh.w1[e, Is + i].view(torch.uint8), layer.w1[e, cfg.I + r * Is + i].view(torch.uint8))
+            assert torch.equal(sh.w2[e].view(torch.uint8), layer.w2[e, :, r * Is:(r + 1) * Is].view(torch.uint8))
+            for j in range(Is // 128):
+                assert torch.equal(sh.w1_scale[e, j], layer.w1_scale[e, (r * Is) // 128 + j])
+                assert torch.equal(sh.w1_scale[e, Is // 128 + j], layer.w1_scale[e, (cfg.I + r * Is) // 128 + j])
+                assert torch.equal(sh.w2_scale[e, :, j], layer.w2_scale[e, :, (r * Is) // 128 + j])
+
+
+def test_tp_shard_rejects_a_split_inside_a_128_block():
+    layer = MoELayer(I.TINY, "cpu")                    # I = 128: one block
+    with pytest.raises(ValueError):
+        layer.tp_shard(0, 2)
+    with pytest.raises(ValueError):
+        layer.tp_shard(1, 1)

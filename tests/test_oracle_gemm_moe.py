@@ -156,3 +156,24 @@ def test_moe_layer_expert_mask_against_dense_evaluation_and_partition():
     assert torch.allclose(sum(parts), full, rtol=1e-12, atol=1e-12 * full.abs().max().item())
     none = O.moe_layer(a8, asc, ids, w, get, expert_mask=torch.zeros(cfg.E, dtype=torch.int32))
     assert (none == 0).all()
+
+
+def test_moe_layer_tensor_parallel_shards_sum_to_the_layer():
+    """TP over I (the pages' TP8 run): each rank holds every expert's I/n intermediate columns
+    (gate and up rows of w1, columns of w2, with their block scales). The 1x128 requantisation
+    groups lie inside a shard, so the ranks' partial outputs sum to the whole layer's output."""
+    cfg = I.MoEConfig("pin_tp", T=9, H=256, E=4, G=2, TG=1, K=2, I=512, seed=8)
+    act = I.moe_activations(cfg)
+    w, ids, a8, asc, ex = _layer(cfg, act)
+    full = O.moe_layer(a8, asc, ids, w, lambda e: ex[e], round_bf16=False)
+    for n in (2, 4):
+        Is, nb = cfg.I // n, cfg.I // n // 128
+
+        def shard(e, r):
+            w1q, w1s, w2q, w2s = ex[e]
+            rows = torch.cat([torch.arange(r * Is, (r + 1) * Is), cfg.I + torch.arange(r * Is, (r + 1) * Is)])
+            brows = torch.cat([torch.arange(r * nb, (r + 1) * nb), cfg.I // 128 + torch.arange(r * nb, (r + 1) * nb)])
+            return (w1q[rows], w1s[brows], w2q[:, r * Is:(r + 1) * Is], w2s[:, r * nb:(r + 1) * nb])
+
+        total = sum(O.moe_layer(a8, asc, ids, w, lambda e, r=r: shard(e, r), round_bf16=False) for r in range(n))
+        assert torch.allclose(total, full, rtol=1e-12, atol=1e-12 * full.abs().max().item())
