@@ -125,6 +125,24 @@ def test_quant_1x128_bit_exact(M, K, col_major):
     assert torch.equal(s_gpu.contiguous().view(torch.int32), s_ref.view(torch.int32))
 
 
+def test_quant_1x128_quotients_near_e4m3_midpoints():
+    """Groups holding elements whose fp32 quotient x / scale lies within 4 ulps of a midpoint
+    between two E4M3 values, or below the E4M3 normal range: the cases in which the kernel
+    takes the exact quotient instead of x times the reciprocal."""
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(16384, 128, generator=g).to(torch.bfloat16)
+    y = (x.float() / (x.float().abs().amax(1, keepdim=True) / 448.0)).abs()
+    below = y.view(torch.int32) & 0xFFFFF
+    near = (((below - 0x80000).abs() <= 4) & (y >= 2.0 ** -6)) | ((y < 2.0 ** -6) & (y > 0))
+    rows = near.any(1)
+    assert int(rows.sum()) > 1000
+    xs = x[rows].contiguous()
+    q, s = B.fp8_per_token_group_quant(xs.to(DEV), 128)
+    q_ref, s_ref = O.quant_1x128(xs)
+    assert torch.equal(u8(q), q_ref)
+    assert torch.equal(s.cpu().view(torch.int32), s_ref.view(torch.int32))
+
+
 def test_quant_strided_rows():
     x = torch.randn(40, 512).to(torch.bfloat16)
     q, s = B.fp8_per_token_group_quant(x.to(DEV)[:, :384], 128)
