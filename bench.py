@@ -214,8 +214,8 @@ def layer_work(cfg, ids, mask=None):
 # figure whose sources have changed since is not reported.
 GATE_UP_TRAFFIC = {
     "prefill_t4096_h7168_e256": {
-        "bytes": 6.891e9,
-        "sha256": "1ca310d1df8d66272ddcd3d752d0aa9cf14867776aad490cd3d70015eba04b4a",
+        "bytes": 6.857e9,
+        "sha256": "ee28cdb3b055b110d66b6e4911ec0404925205dfe68267425eded24aafcce078",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
                    "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean; "
                    "profiles/launches_prefill_t4096.md)",

@@ -40,6 +40,7 @@ _SIGNATURES = {
     "fp8_per_token_group_quant": (_c_int, [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_int, _p]),
     "fp8_per_block_quant": (_c_int, [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _p]),
     "fp8_blockscale_gemm": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _p]),
+    "fp8moe_selftest_gemm_stall": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _p]),
     "fused_moe_fp8_blockscale_g1u1_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "fused_moe_fp8_blockscale_g1u1": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
                                                _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int, _p, _p,
@@ -266,6 +267,16 @@ def fp8_blockscale_gemm(A, B, a_scale, b_scale, out=None):
                                             _row_major(out, "out"), M, N, K, _stream())
     _check("fp8_blockscale_gemm", rc)
     return out
+
+
+def selftest_gemm_stall(A, B, a_scale, b_scale, out, stall_kb):
+    """Failure-handling test hook: the block-scale GEMM with K block stall_kb's scales withheld,
+    so its bounded wait runs out; the caller reads the timeout bit with device_status()."""
+    M, K = A.shape
+    N = B.shape[0]
+    rc = load_library().fp8moe_selftest_gemm_stall(_ptr(A), _ptr(B), _ptr(a_scale), _ptr(b_scale), _ptr(out),
+                                                   _row_major(out, "out"), M, N, K, stall_kb, _stream())
+    _check("fp8moe_selftest_gemm_stall", rc)
 
 
 def fused_moe_workspace_bytes(T, topk, E, H, I, block_m):

@@ -425,8 +425,9 @@ int fp8_per_block_quant(const float* w, int ld_w, int N, int K, int block, uint8
 }
 
 // ------------------------------------------------------------------ S0 GEMM
-int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale, const float* b_scale, uint16_t* C,
-                        int ldc, int M, int N, int K, void* stream) {
+static int blockscale_gemm_impl(const char* name, const uint8_t* A, const uint8_t* B, const float* a_scale,
+                                const float* b_scale, uint16_t* C, int ldc, int M, int N, int K, int stall_kb1,
+                                void* stream) {
   if (M < 1 || N < 1 || K < 1) return fail(FP8MOE_EINVAL, "M, N, K must be >= 1");
   if (K % 16 != 0) return fail(FP8MOE_EUNSUPPORTED, "K must be a multiple of 16 (got %d)", K);
   if (ldc < N) return fail(FP8MOE_EINVAL, "ldc (%d) < N (%d)", ldc, N);
@@ -451,11 +452,24 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale
   a.ldc = ldc;
   a.c_vec = (ldc % 16 == 0) && (reinterpret_cast<uintptr_t>(C) & 31u) == 0;   // 32-byte row stores
   a.b_rows_per_expert = 0;
+  a.stall_kb1 = stall_kb1;
   const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * a.n_tiles;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   blockscale_gemm_kernel<kModeDense><<<grid, kGemmThreads, kGemmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       ma, mb, a);
-  return check_gemm_launch("fp8_blockscale_gemm", blockscale_gemm_kernel<kModeDense>, kGemmThreads, kGemmSmemBytes);
+  return check_gemm_launch(name, blockscale_gemm_kernel<kModeDense>, kGemmThreads, kGemmSmemBytes);
+}
+
+int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale, const float* b_scale, uint16_t* C,
+                        int ldc, int M, int N, int K, void* stream) {
+  return blockscale_gemm_impl("fp8_blockscale_gemm", A, B, a_scale, b_scale, C, ldc, M, N, K, 0, stream);
+}
+
+int fp8moe_selftest_gemm_stall(const uint8_t* A, const uint8_t* B, const float* a_scale, const float* b_scale,
+                               uint16_t* C, int ldc, int M, int N, int K, int stall_kb, void* stream) {
+  if (stall_kb < 0 || stall_kb >= (K + 127) / 128) return fail(FP8MOE_EINVAL, "stall_kb must be a K block index");
+  return blockscale_gemm_impl("fp8moe_selftest_gemm_stall", A, B, a_scale, b_scale, C, ldc, M, N, K, stall_kb + 1,
+                              stream);
 }
 
 // ------------------------------------------------------------------ S4-S7 fused MoE

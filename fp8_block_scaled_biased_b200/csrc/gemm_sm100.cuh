@@ -82,6 +82,10 @@ struct GemmArgs {
   uint8_t* a2;            // up output [M, I] (slot-ordered FP8 intermediate)
   float* s2;              // up output [I/128, M]
   __nv_bfloat16* ystage;  // down output [T*topk, H] (weighted rows by pair id, bf16)
+  // Failure-handling test hook (0 = off): with k + 1, the scale loader withholds
+  // K block k's scales, so the epilogue's bounded wait for them runs out and the
+  // CTA takes its abort path (device error word, TMEM freed, clean exit).
+  int stall_kb1;
 };
 
 struct GemmSmem {
@@ -544,13 +548,15 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         const float* sw_src1 = args.b_scale + (static_cast<size_t>(e) * args.nb_per_expert + nb1) * num_kb;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&s->sempty[sslot], scphase ^ 1u, abort_flag)) { ok = false; break; }
+          if (kb + 1 != args.stall_kb1) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) cp_async_4(&s->sa[sslot][4 * lane + i], sa_src[i] + kb * kstride);
-          if (lane == 0) {
-            cp_async_4(&s->sw[sslot][0], sw_src0 + kb);
-            cp_async_4(&s->sw[sslot][1], sw_src1 + kb);
+            for (int i = 0; i < 4; ++i) cp_async_4(&s->sa[sslot][4 * lane + i], sa_src[i] + kb * kstride);
+            if (lane == 0) {
+              cp_async_4(&s->sw[sslot][0], sw_src0 + kb);
+              cp_async_4(&s->sw[sslot][1], sw_src1 + kb);
+            }
+            cp_async_mbar_arrive(&s->sfull[sslot]);
           }
-          cp_async_mbar_arrive(&s->sfull[sslot]);
           if (++sslot == kScaleSlots) { sslot = 0; scphase ^= 1u; }
         }
       }

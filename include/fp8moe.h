@@ -74,6 +74,17 @@ int fp8moe_device_status(void* stream);
 int fp8moe_timing_enable(int on);
 int fp8moe_timing_last(float* ms);
 
+/* Failure-handling test hook (not part of the pages' API): fp8_blockscale_gemm
+ * on the same arguments, except that in every CTA's tiles the scales of K block
+ * stall_kb are withheld. The epilogue's bounded wait for them runs out (about
+ * 2 s), the CTA sets FP8MOE_DEVERR_TIMEOUT, stops its other warps, frees its
+ * tensor memory and exits; C is left unspecified. fp8moe_device_status() then
+ * reports the bit and the context stays usable. Nothing faults or hangs. */
+int fp8moe_selftest_gemm_stall(const uint8_t* A, const uint8_t* B,
+                               const float* a_scale, const float* b_scale,
+                               uint16_t* C, int ldc, int M, int N, int K,
+                               int stall_kb, void* stream);
+
 /* Block size of the M (token-expert pair) dimension that the fused MoE kernels
  * tile by; moe_align_sort must be called with block_m equal to this. */
 int fp8moe_moe_block_m(void);

@@ -144,3 +144,8 @@ def test_bf16_routing_and_masked_sort_reject_bad_arguments(lib):
     ws = lib.moe_align_sort_workspace(16, 4, 16, 4)
     rc, msg = _rc(lib, "moe_align_sort_masked", P, P, 4, 16, 4, 16, 4, P, P, P, P, P, cap, P, ws - 1, None)
     assert rc == 3 and "workspace" in msg
+
+
+def test_selftest_stall_rejects_a_k_block_out_of_range(lib):
+    rc, msg = _rc(lib, "fp8moe_selftest_gemm_stall", P, P, P, P, P, 256, 128, 256, 256, 2, None)
+    assert rc == 1 and "stall_kb" in msg

@@ -80,6 +80,22 @@ def test_routing_bit_exact_with_strided_outputs(cfg):
     assert (wbuf[:, cfg.K:] == -7.0).all() and (ibuf[:, cfg.K:] == -7).all()
 
 
+@pytest.mark.parametrize("E,G,TG,K", [(256, 8, 4, 8), (64, 8, 3, 6), (16, 1, 1, 4), (24, 4, 2, 5)])
+def test_routing_ties_resolve_like_the_oracle(E, G, TG, K):
+    """Logits and biases on a few levels, so equal biased scores and equal group scores are
+    common: the kernel must break ties toward the lower group and expert index."""
+    g = torch.Generator().manual_seed(E + K)
+    T = 512
+    logits = torch.randint(-2, 3, (T, E), generator=g).float() * 0.5
+    bias = torch.randint(0, 2, (E,), generator=g).float() * 0.25
+    w = torch.empty(T, K, device=DEV)
+    ids = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    B.moe_biased_grouped_topk(logits.to(DEV), bias.to(DEV), w, ids, G, TG, True, 2.5)
+    w_ref, ids_ref = O.biased_grouped_topk(logits, bias, K, G, TG, True, 2.5)
+    assert torch.equal(ids.cpu(), ids_ref)
+    assert torch.equal(w.cpu().view(torch.int32), w_ref.view(torch.int32))
+
+
 # ---------------------------------------------------------------- S2 align/sort
 @pytest.mark.parametrize("cfg,block_m", [(I.TINY, 4), (I.TINY, 128), (I.DECODE, 128), (I.DECODE, 16),
                                          (I.PREFILL, 128), (I.PREFILL, 64), (I.SKEWED, 128)],
@@ -207,6 +223,23 @@ def test_gemm_is_deterministic():
     c1 = B.fp8_blockscale_gemm(qa, qb, sa, sb).clone()
     c2 = B.fp8_blockscale_gemm(qa, qb, sa, sb)
     assert torch.equal(c1, c2)
+
+
+def test_gemm_bounded_wait_runs_out_and_the_context_stays_usable():
+    """Failure handling without a fault: the test hook withholds one K block's scales, the
+    epilogue's bounded wait for them runs out (about 2 s), every CTA stops, frees its tensor
+    memory and flags FP8MOE_DEVERR_TIMEOUT; the next GEMMs run normally."""
+    g = torch.Generator().manual_seed(21)
+    a = torch.randn(256, 512, generator=g).to(torch.bfloat16).to(DEV)
+    b = (torch.randn(512, 512, generator=g) * 0.02).to(DEV)
+    qa, sa = B.fp8_per_token_group_quant(a, 128)
+    qb, sb = B.fp8_per_block_quant(b)
+    c = torch.empty(256, 512, dtype=torch.bfloat16, device=DEV)
+    B.selftest_gemm_stall(qa, qb, sa, sb, c, stall_kb=1)
+    assert B.device_status() & 1                       # FP8MOE_DEVERR_TIMEOUT (read and cleared)
+    assert B.device_status() == 0
+    got, ref = _gemm_case(257, 1000, 1024, seed=3)     # TMEM and the context are intact
+    _assert_gemm_close(got, ref)
 
 
 # ---------------------------------------------------------------- S4-S7 fused MoE
