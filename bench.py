@@ -215,7 +215,7 @@ def layer_work(cfg, ids, mask=None):
 GATE_UP_TRAFFIC = {
     "prefill_t4096_h7168_e256": {
         "bytes": 6.857e9,
-        "sha256": "ee28cdb3b055b110d66b6e4911ec0404925205dfe68267425eded24aafcce078",
+        "sha256": "22bad3149e6e9dc2dcb6fcb925d701f4e6b8b2f2e9d23c2ad816becc2c504417",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
                    "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean; "
                    "profiles/launches_prefill_t4096.md)",
@@ -224,14 +224,23 @@ GATE_UP_TRAFFIC = {
 GEMM_SOURCES = ("fp8_block_scaled_biased_b200/csrc/gemm_sm100.cuh", "fp8_block_scaled_biased_b200/csrc/common.cuh")
 
 
-def gemm_source_sha():
-    """SHA-256 of the GEMM kernel sources with all whitespace removed (layout-only edits keep it)."""
+def source_sha(paths):
+    """SHA-256 of C++ sources with comments and all whitespace removed, so that edits to
+    comments or layout keep it and any change to the code changes it."""
     import hashlib
+    import re
     h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(b"".join(f.read().split()))
+    for path in paths:
+        with open(path, encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)       # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                      # line comments
+        h.update("".join(text.split()).encode())
     return h.hexdigest()
+
+
+def gemm_source_sha():
+    return source_sha(os.path.join(ROOT, rel) for rel in GEMM_SOURCES)
 
 
 def gate_up_traffic(workload, override):

@@ -22,8 +22,9 @@
 //               shape and its rows' pair ids and routing weights into a 2-slot
 //               shared ring for the MMA issuer and the epilogue;
 //   warps 4..11 epilogue: tcgen05.ld the partials, multiply by
-//               a_scale[row, kb] * b_scale[col/128, kb] and add into fp32
-//               registers (the per-128-K promotion), then the mode's output:
+//               a_scale[row, kb] * b_scale[col/128, kb] (the down GEMM also by
+//               the row's routing weight) and add into fp32 registers (the
+//               per-128-K promotion), then the mode's output:
 //               32-byte (whole-sector) stores of each thread's row, or for the
 //               down GEMM's weighted bf16 rows a transpose through a small
 //               shared buffer per warp so that each store writes 8 whole 64-byte
@@ -51,7 +52,7 @@ constexpr int kStages = 4;
 constexpr int kScaleSlots = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 128 + 32 * kEpiWarps;   // warpgroup 0 + two epilogue warpgroups
-constexpr uint32_t kRegsWg0 = 56;                     // producer / MMA / scale-loader warpgroup
+constexpr uint32_t kRegsWg0 = 56;                     // producer / MMA / scale-loader / tile-info warpgroup
 constexpr uint32_t kRegsEpilogue = 224;               // 56 + 2 x 224 == 3 x 168 (launch budget)
 constexpr int kStageA = kBM * kBK;            // bytes
 constexpr int kStageB = kBN * kBK;

@@ -117,3 +117,12 @@ def test_tensor_parallel_workload_config_and_oracle_sample():
     assert r.step() > 0
     w1q, w1s, w2q, w2s = r.weights[r.experts[0]]
     assert w1q.shape == (256, 256) and w1s.shape == (2, 2) and w2q.shape == (256, 128) and w2s.shape == (2, 1)
+
+
+def test_source_hash_ignores_comments_and_layout_only(tmp_path):
+    code = "int f(int a) {\n  return a + 1;  // one more\n}\n/* block\n comment */\n"
+    (tmp_path / "a.cu").write_text(code)
+    (tmp_path / "b.cu").write_text("int f(int a){return a+1;}  // other words\n")
+    (tmp_path / "c.cu").write_text("int f(int a){return a+2;}\n")
+    h = [bench.source_sha([str(tmp_path / n)]) for n in ("a.cu", "b.cu", "c.cu")]
+    assert h[0] == h[1] != h[2]
