@@ -434,7 +434,10 @@ def run_ours(args, world, rank, local):
     e2e_ms = e2e_pipelined(layer, step, logits, x, h_logits, h_x, h_out, args.steps, world)
 
     peaks = load_peaks()
-    fp8_peak_tflops = 2.0 * peaks["bf16_tflops"]           # nominal FP8:BF16 dense ratio 2:1
+    # The timed steps run back to back under the power limit: the tensor peak is the
+    # sustained one (the burst one for the boost-clock context figure); nominal FP8:BF16 2:1.
+    fp8_peak_tflops = 2.0 * peaks["bf16_tflops_sustained"]
+    fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
     hbm = peaks["hbm_gbs"]
     gat_ms, g1_ms, g2_ms, cmb_ms = last_kernel_ms[:4]
     g1_t_bytes = work["gemm1_bytes"] / hbm / 1e9 * 1e3      # ms at peak HBM
@@ -447,8 +450,9 @@ def run_ours(args, world, rank, local):
                     "achieved": work["gemm1_flops"] / (g1_ms * 1e-3) / 1e12, "peak": fp8_peak_tflops, "unit": "TFLOP/s"}
     roofline["frac"] = roofline["achieved"] / roofline["peak"]
     roofline["traffic"], roofline["traffic_source"] = gate_up_traffic(cfg.name, args.traffic)
-    roofline["peak_source"] = peaks["source"] + (" (fp8 = 2 x bf16)" if roofline["bound"] == "tensor" else "")
+    roofline["peak_source"] = peaks["source"] + (" sustained (fp8 = 2 x bf16)" if roofline["bound"] == "tensor" else "")
     t_layer_roof = max(work["flops"] / (fp8_peak_tflops * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
+    t_layer_roof_burst = max(work["flops"] / (fp8_peak_burst * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
 
     tokens = cfg.T * world
     result = {
@@ -473,10 +477,11 @@ def run_ours(args, world, rank, local):
         "layer_roofline": {"ms": t_layer_roof, "frac": t_layer_roof / ms_per_step,
                            "flops": work["flops"], "bytes": work["layer_bytes"],
                            "touched_experts": work["n_experts"], "fp8_peak_tflops": fp8_peak_tflops,
+                           "fp8_peak_source": peaks["source"] + " sustained (fp8 = 2 x bf16)",
                            "hbm_gbs": hbm},
         "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
         "instrumented_ms_per_step": instrumented_ms,
-        "burst": {"ms_per_step": burst_ms_per_step, "layer_roofline_frac": t_layer_roof / burst_ms_per_step,
+        "burst": {"ms_per_step": burst_ms_per_step, "layer_roofline_frac": t_layer_roof_burst / burst_ms_per_step,
                   "method": "median of the same steps each started after 5 ms of idle GPU (boost clock); "
                             "context only, the headline value is the sustained back-to-back run"},
         "kernels_ms": {"moe_gather": gat_ms, "moe_gate_up_gemm": g1_ms, "moe_down_gemm": g2_ms, "moe_combine": cmb_ms,
