@@ -283,22 +283,56 @@ def fused_moe_workspace_bytes(T, topk, E, H, I, block_m):
     return load_library().fused_moe_fp8_blockscale_g1u1_workspace(T, topk, E, H, I, block_m)
 
 
-def fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_pairs: SortedPairs, topk, a1_scale, fc1_scale, fc2_scale,
-                                  scale_blk_n=128, scale_blk_k=128, fc2_smooth_scale=None, workspace=None):
-    """out bf16 [T, H] = fused g1u1 MoE (GEMM1 + SiLU*up + requant + GEMM2 + weighted combine)."""
+def _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale):
+    """Checks shared by both fused MoE entry points; returns (T, H, I, E).
+
+    The library builds its TMA maps from these sizes (w1 as E*2I rows of H, w2 as
+    E*H rows of I), so every tensor must have exactly the shape and dtype the sizes
+    imply and be contiguous; anything else is refused before the call."""
     _cuda(out, torch.bfloat16, "out")
     _cuda(a8, FP8, "a8")
     _cuda(w1, FP8, "w1")
     _cuda(w2, FP8, "w2")
+    for name, t in (("a1_scale", a1_scale), ("fc1_scale", fc1_scale), ("fc2_scale", fc2_scale)):
+        _cuda(t, torch.float32, name)
+    if a8.dim() != 2 or w1.dim() != 3 or w2.dim() != 3:
+        raise ValueError("a8 must be [T, H], w1 [E, 2I, H] and w2 [E, H, I]")
     T, H = a8.shape
-    E, twoI, _ = w1.shape
+    E, twoI, H1 = w1.shape
     I = w2.shape[2]
     if twoI != 2 * I:
         raise ValueError("g1u1 requires w1.shape[1] == 2 * w2.shape[2]")
+    if H1 != H or tuple(w2.shape) != (E, H, I):
+        raise ValueError(f"w1 {tuple(w1.shape)} and w2 {tuple(w2.shape)} do not match a8's H={H}")
+    if tuple(out.shape) != (T, H):
+        raise ValueError(f"out must be [{T}, {H}], got {tuple(out.shape)}")
+    if H % 128 or I % 128:
+        raise ValueError(f"H and I must be multiples of 128 (H={H}, I={I})")
+    expect = {"a1_scale": (H // 128, T), "fc1_scale": (E, 2 * I // 128, H // 128),
+              "fc2_scale": (E, H // 128, I // 128)}
+    for name, t in (("a1_scale", a1_scale), ("fc1_scale", fc1_scale), ("fc2_scale", fc2_scale)):
+        if tuple(t.shape) != expect[name]:
+            raise ValueError(f"{name} must be {expect[name]}, got {tuple(t.shape)}")
     for name, t in (("out", out), ("a8", a8), ("w1", w1), ("w2", w2), ("a1_scale", a1_scale),
                     ("fc1_scale", fc1_scale), ("fc2_scale", fc2_scale)):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    sp = sorted_pairs
+    for name, t, dt in (("sorted_ids", sp.sorted_ids, torch.int32), ("sorted_weights", sp.sorted_weights, torch.float32),
+                        ("sorted_expert_ids", sp.sorted_expert_ids, torch.int32),
+                        ("num_valid_ids", sp.num_valid_ids, torch.int32)):
+        _cuda(t, dt, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if sp.sorted_weights.numel() < sp.capacity or sp.sorted_expert_ids.numel() < sp.capacity // sp.block_m:
+        raise ValueError("sorted_weights / sorted_expert_ids shorter than the sorted list's capacity")
+    return T, H, I, E
+
+
+def fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_pairs: SortedPairs, topk, a1_scale, fc1_scale, fc2_scale,
+                                  scale_blk_n=128, scale_blk_k=128, fc2_smooth_scale=None, workspace=None):
+    """out bf16 [T, H] = fused g1u1 MoE (GEMM1 + SiLU*up + requant + GEMM2 + weighted combine)."""
+    T, H, I, E = _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale)
     sp = sorted_pairs
     lib = load_library()
     need = lib.fused_moe_fp8_blockscale_g1u1_workspace(T, topk, E, H, I, sp.block_m)
@@ -319,13 +353,10 @@ def fused_moe_fp8_blockscale_g1u1_noalloc(out, a8, w1, w2, sorted_pairs: SortedP
 
     For callers that cannot allocate device memory. Problems needing more than
     NOALLOC_SCRATCH_BYTES of scratch are rejected; calls share the scratch, so
-    they must not overlap on the GPU.
+    they must not overlap on the GPU. The arguments are checked exactly as for
+    fused_moe_fp8_blockscale_g1u1.
     """
-    _cuda(out, torch.bfloat16, "out")
-    _cuda(a8, FP8, "a8")
-    T, H = a8.shape
-    E = w1.shape[0]
-    I = w2.shape[2]
+    T, H, I, E = _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale)
     sp = sorted_pairs
     rc = load_library().fused_moe_fp8_blockscale_g1u1_noalloc(
         _ptr(out), _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights),

@@ -593,16 +593,18 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
 // The fused call's scratch for callers that cannot allocate device memory: one
 // fixed array per device, held for the life of the process. Its name is only a
 // host-side handle; the device address comes from cudaGetSymbolAddress, looked
-// up once per device on the first call (with that device current).
+// up on the first successful call on each device (with that device current).
 }  // extern "C"
 
 namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FP8MOE_NOALLOC_SCRATCH_BYTES];
 
+// The looked-up address of the scratch array on each device. A failed lookup
+// (for example one made while the stream was being captured) is not kept: the
+// next call on that device tries again.
 struct NoAllocScratch {
-  std::once_flag once;
+  std::mutex mu;
   void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 NoAllocScratch g_noalloc[kMaxDevices];
 }  // namespace
@@ -628,12 +630,23 @@ int fused_moe_fp8_blockscale_g1u1_noalloc(uint16_t* out, const uint8_t* a8, cons
   if (e != cudaSuccess) return fail(FP8MOE_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(FP8MOE_ECUDA, "device ordinal %d unsupported", dev);
   NoAllocScratch& sc = g_noalloc[dev];
-  std::call_once(sc.once, [&] { sc.err = cudaGetSymbolAddress(&sc.ptr, g_noalloc_scratch); });
-  if (sc.err != cudaSuccess || !sc.ptr)
-    return fail(FP8MOE_ECUDA, "scratch address lookup: %s", cudaGetErrorString(sc.err));
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(sc.mu);
+    if (!sc.ptr) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess || !p) {
+        cudaGetLastError();   // the failed lookup leaves no sticky error behind; the next call retries
+        return fail(FP8MOE_ECUDA, "scratch address lookup: %s", cudaGetErrorString(e));
+      }
+      sc.ptr = p;
+    }
+    scratch = sc.ptr;
+  }
   return fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_ids, sorted_weights, sorted_expert_ids,
                                        num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
-                                       fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, sc.ptr,
+                                       fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, scratch,
                                        FP8MOE_NOALLOC_SCRATCH_BYTES, stream);
 }
 

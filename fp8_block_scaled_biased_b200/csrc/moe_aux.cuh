@@ -18,8 +18,10 @@ constexpr int kMoeBlockRows = 128;            // rows per sorted block (the GEMM
 
 // Copies each sorted slot's token row of a8 [T, H] (and its H/128 scales from
 // a1_scale [H/128, T]) into slot order, sets pair_flag[p] = 1 for every pair p
-// in the list and adds the number of listed pairs to *n_present (the caller
-// zeroes both first). Padding slots are skipped: the GEMMs treat rows
+// in the list and adds the number of distinct listed pairs to *n_present (the
+// caller zeroes both first; pair_flag is 4-byte aligned). A pair id listed twice
+// (not a moe_align_sort result) is counted once, so *n_present == T*topk means
+// every pair is present. Padding slots are skipped: the GEMMs treat rows
 // independently and never store padding rows.
 constexpr int kGatherWarps = 8;
 __global__ void __launch_bounds__(32 * kGatherWarps)
@@ -44,8 +46,12 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
   for (int slot = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); slot < nv; slot += gridDim.x * kGatherWarps) {
     const int sid = sorted_ids[slot];
     if (sid < 0 || sid >= P) continue;
-    if (lane == 0) pair_flag[sid] = 1;
-    ++warp_present;
+    if (lane == 0) {
+      // set the pair's flag byte through its 32-bit word; count the pair only if
+      // this slot set it first
+      const unsigned bit = 1u << (8 * (sid & 3));
+      if ((atomicOr(reinterpret_cast<unsigned*>(pair_flag) + (sid >> 2), bit) & bit) == 0) ++warp_present;
+    }
     const int t = sid / topk;
     const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
     uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
@@ -84,8 +90,8 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
 // out[t, :] = bf16( y[t*K + 0] + y[t*K + 1] + ... + y[t*K + K-1] ), fp32 adds in
 // slot order k over the pairs whose flag is set (the routing weight is already
 // in y; a pair absent from the sorted list has no row). When every pair is
-// listed (*n_present == T*K, one cached load) the flags are not read. One thread
-// per 8 columns.
+// listed (*n_present, the count of distinct listed pairs, equals T*K: one cached
+// load) the flags are not read. One thread per 8 columns.
 __global__ void __launch_bounds__(256)
 moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, const uint8_t* __restrict__ pair_flag,
                    const int* __restrict__ n_present, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
