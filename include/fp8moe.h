@@ -256,7 +256,14 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B,
  * topk <= 32;
  * fc2_smooth_scale must be NULL (the pages do not define it); workspace >=
  * fused_moe_fp8_blockscale_g1u1_workspace(); capacity >= the sort's padded
- * length.
+ * length; workspace 256-byte aligned.
+ * Workspace contents after a call (parts in this order, each starting at the
+ * next multiple of 256 bytes; cap = capacity, P = T*topk): the slot-ordered
+ * activations fp8 [cap, H] and their scales fp32 [H/128, cap]; the re-quantised
+ * intermediate a2 fp8 [cap, I] and its scales fp32 [I/128, cap] (slot s holds
+ * pair sorted_ids[s]; padding slots are not written); the weighted
+ * down-projection rows bf16 [P, H] by pair id; a listed-pair count (16 bytes)
+ * and one flag byte per pair.
  */
 size_t fused_moe_fp8_blockscale_g1u1_workspace(int T, int topk, int E, int H, int I,
                                                 int block_m);
@@ -292,12 +299,17 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8,
  * (fused_moe_fp8_blockscale_g1u1_workspace for the given capacity) is larger
  * is rejected with FP8MOE_EUNSUPPORTED before anything is launched. The first
  * call on a device looks up the array's device address (cudaGetSymbolAddress);
- * make that first call before capturing any stream on that device. All calls
- * on a device share the one array and it keeps whatever the previous call left
- * in it (nothing in it has to start at zero: every byte a call reads, that
- * call has written first), so calls that can overlap on the GPU (different
- * streams without ordering between them) race and corrupt each other: order
- * them on one stream.
+ * make that first call before capturing any stream on that device. A lookup
+ * that fails returns FP8MOE_ECUDA and is tried again by the next call. All
+ * calls on a device share the one array and it keeps whatever the previous
+ * call left in it. The parts that must start at zero (the listed-pair count
+ * and flags) are cleared by every call. The padding rows of the slot-ordered
+ * activations and intermediate are never written: the GEMMs read them (and
+ * their scales), possibly holding an earlier call's data, but rows are
+ * independent and padding rows are never stored, so they cannot affect the
+ * output. Calls that can overlap on the GPU (different streams without
+ * ordering between them) race and corrupt each other: order them on one
+ * stream.
  */
 #define FP8MOE_NOALLOC_SCRATCH_BYTES (64ull << 20)
 int fused_moe_fp8_blockscale_g1u1_noalloc(uint16_t* out, const uint8_t* a8,
