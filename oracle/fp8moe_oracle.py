@@ -356,21 +356,29 @@ def silu(z: torch.Tensor) -> torch.Tensor:
     return z / (1.0 + torch.exp(-z))
 
 
-def expert_ffn(a8_rows, a_scale_rows, w1q, w1s, w2q, w2s):
-    """One expert applied to quantised token rows; returns y [rows, H] in fp64.
+def expert_intermediate(a8_rows, a_scale_rows, w1q, w1s):
+    """The first half of one expert: the re-quantised intermediate (a2 codes [rows, I],
+    scales fp32 [rows, I/128]) that the second GEMM takes.
 
-    From the page's section "Blockscale FP8 MoE Computation" (g1u1: w1 holds
-    gate and up, w2.shape[2] * 2 == w1.shape[1]; activation silu). Readings:
-    w1 rows [0, I) are gate and [I, 2I) are up; GEMM1 stays fp64 (no rounding
-    before the activation); h = silu(gate) * up in fp64, rounded to fp32 and
-    re-quantised per row in 1x128 groups along I by quant_1x128 (the second
-    GEMM's activation quantisation is not printed; it is taken to be the same
-    dynamic recipe as the first); GEMM2 = blockscale_gemm(a2, s2, w2q, w2s).
+    From the page's section "Blockscale FP8 MoE Computation" (g1u1: w1 holds gate
+    and up, w2.shape[2] * 2 == w1.shape[1]; activation silu). Readings: w1 rows
+    [0, I) are gate and [I, 2I) are up; GEMM1 stays fp64 (no rounding before the
+    activation); h = silu(gate) * up in fp64, rounded to fp32 and re-quantised per
+    row in 1x128 groups along I by quant_1x128 (the second GEMM's activation
+    quantisation is not printed; it is taken to be the same dynamic recipe as the
+    first).
     """
-    I = w2q.shape[1]
+    I = w1q.shape[0] // 2
     g1 = blockscale_gemm(a8_rows, a_scale_rows, w1q, w1s)
     h = silu(g1[:, :I]) * g1[:, I:]
-    a2, s2 = quant_1x128(h.to(F32))
+    return quant_1x128(h.to(F32))
+
+
+def expert_ffn(a8_rows, a_scale_rows, w1q, w1s, w2q, w2s):
+    """One expert applied to quantised token rows; returns y [rows, H] in fp64:
+    expert_intermediate, then GEMM2 = blockscale_gemm(a2, s2, w2q, w2s) (same page
+    section)."""
+    a2, s2 = expert_intermediate(a8_rows, a_scale_rows, w1q, w1s)
     return blockscale_gemm(a2, s2, w2q, w2s)
 
 

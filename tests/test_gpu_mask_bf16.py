@@ -8,7 +8,7 @@ from oracle import fp8moe_oracle as O
 from fp8_block_scaled_biased_b200 import binding as B
 from fp8_block_scaled_biased_b200 import inputs as I
 from fp8_block_scaled_biased_b200.layer import MoELayer
-from tests.gpu_helpers import assert_moe_close, oracle_moe_rows
+from tests.gpu_helpers import assert_moe_close, blocks_covered, full_size_tokens, oracle_moe_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -110,14 +110,20 @@ def test_fused_moe_expert_parallel_partials(cfg, nranks):
     assert_moe_close(total, ref_full)
 
 
-def test_fused_moe_expert_mask_full_size_sampled():
+def test_fused_moe_expert_mask_full_size_many_tokens():
+    """Expert-parallel rank 5 of 8 on the prefill layer: 256 seeded tokens, the first and
+    last token and every token of the rank's most-loaded kept expert, chosen from the
+    oracle's routing, against the oracle's partial output."""
     cfg = I.PREFILL
     layer = MoELayer(cfg, DEV).load_synthetic_weights()
     act = I.moe_activations(cfg)
     mask = rank_mask(cfg.E, 5, 8)
     out = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV), expert_mask=mask.to(DEV)).clone()
-    g = torch.Generator().manual_seed(7)
-    tokens = torch.sort(torch.randperm(cfg.T, generator=g)[:6]).values
+    _, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    tokens, roles = full_size_tokens(cfg, ids_ref, 256, seed=7, m64_tail=False, expert_mask=mask)
+    assert int(mask[roles["most_loaded"]]) == 1 and tokens.numel() >= 256
+    hit, nblocks = blocks_covered(ids_ref, tokens, cfg.E, expert_mask=mask)
+    assert hit >= 0.75 * nblocks, (hit, nblocks)
     ref, _, _ = oracle_moe_rows(cfg, act, tokens, expert_mask=mask)
     assert_moe_close(out.cpu()[tokens], ref)
 

@@ -11,7 +11,9 @@ from oracle import fp8moe_oracle as O
 from fp8_block_scaled_biased_b200 import binding as B
 from fp8_block_scaled_biased_b200 import inputs as I
 from fp8_block_scaled_biased_b200.layer import MoELayer
-from tests.gpu_helpers import assert_moe_close, oracle_moe_rows
+from tests.gpu_helpers import (assert_moe_close, blocks_covered, e4m3_ordinal, full_size_tokens,
+                                fused_workspace_intermediate, m64_tail_expert, oracle_expert, oracle_moe_rows,
+                                tokens_of_expert)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device"),
@@ -143,8 +145,8 @@ def test_quant_1x128_bit_exact(M, K, col_major):
 
 def test_quant_1x128_quotients_near_e4m3_midpoints():
     """Groups holding elements whose fp32 quotient x / scale lies within 4 ulps of a midpoint
-    between two E4M3 values, or below the E4M3 normal range: the cases in which the kernel
-    takes the exact quotient instead of x times the reciprocal."""
+    between two E4M3 values, or below the E4M3 normal range: the quotients whose code a
+    division rounded differently (for instance x times a rounded reciprocal) would change."""
     g = torch.Generator().manual_seed(11)
     x = torch.randn(16384, 128, generator=g).to(torch.bfloat16)
     y = (x.float() / (x.float().abs().amax(1, keepdim=True) / 448.0)).abs()
@@ -208,9 +210,10 @@ def test_gemm_small_and_ragged(M, N, K):
     _assert_gemm_close(got, ref)
 
 
-def test_gemm_2048x4096x7168_sampled_rows():
-    rows = torch.cat([torch.arange(0, 2048, 61), torch.tensor([127, 128, 2047])])
-    got, ref = _gemm_case(2048, 4096, 7168, seed=0, sample_rows=rows)
+def test_gemm_2048x4096x7168_every_element():
+    """The standalone GEMM workload (M=2048, N=4096, K=7168) compared in full: all
+    8,388,608 outputs, every one of its 16 x 16 tiles and 56 K blocks."""
+    got, ref = _gemm_case(2048, 4096, 7168, seed=0)
     _assert_gemm_close(got, ref)
 
 
@@ -275,19 +278,112 @@ def big_layer():
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("cfg,n_sample", [(I.DECODE, 6), (I.PREFILL, 4), (I.SKEWED, 8)], ids=lambda v: getattr(v, "name", str(v)))
-def test_fused_moe_full_size_sampled_tokens(big_layer, cfg, n_sample):
+def test_fused_moe_decode_every_token(big_layer):
+    """The decode layer (T=64) compared in full: all 64 tokens, all 512 pairs."""
+    cfg = I.DECODE
     layer = MoELayer(cfg, DEV, weights_from=big_layer)
     act = I.moe_activations(cfg)
     out = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV)).clone()
-    g = torch.Generator().manual_seed(99)
-    tokens = torch.sort(torch.cat([torch.randperm(cfg.T, generator=g)[: n_sample - 1],
-                                   torch.tensor([cfg.T - 1])]).unique()).values
-    ref, w_ref, ids_ref = oracle_moe_rows(cfg, act, tokens)
+    ref, w_ref, ids_ref = oracle_moe_rows(cfg, act, None)
     assert torch.equal(layer.topk_ids.cpu(), ids_ref)
+    assert_moe_close(out, ref)
+    out2 = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    assert torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("cfg", [I.PREFILL, I.SKEWED], ids=lambda c: c.name)
+def test_fused_moe_full_size_many_tokens(big_layer, cfg):
+    """The prefill (T=4096) and skewed (T=16384) layers: 512 seeded tokens and the first and
+    last token; at prefill also every token of the most-loaded expert (1249 pairs, ten row
+    blocks) and of the least-loaded expert with whole row blocks and an M=64 tail. The
+    tokens are chosen from the oracle's routing; their pairs reach nearly every row block.
+    (Every skewed expert carries thousands of pairs: its whole experts are compared pair by
+    pair in the next test.)"""
+    layer = MoELayer(cfg, DEV, weights_from=big_layer)
+    act = I.moe_activations(cfg)
+    out = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV)).clone()
+    _, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    assert torch.equal(layer.topk_ids.cpu(), ids_ref)
+    whole = cfg is I.PREFILL
+    tokens, roles = full_size_tokens(cfg, ids_ref, 512, seed=99, most_loaded=whole, m64_tail=whole)
+    if whole:
+        assert set(roles) == {"most_loaded", "m64_tail"}
+    hit, nblocks = blocks_covered(ids_ref, tokens, cfg.E)
+    assert hit >= 0.95 * nblocks, (hit, nblocks)
+    ref, _, _ = oracle_moe_rows(cfg, act, tokens)
     assert_moe_close(out.cpu()[tokens], ref)
     out2 = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
     assert torch.equal(out, out2)
+
+
+def test_fused_moe_skewed_whole_experts_every_pair(big_layer):
+    """Every pair of two skewed experts: the most-loaded one (12,856 pairs, 101 row blocks)
+    and the least-loaded one whose last block runs as an M=64 tile (6,785 pairs). The expert
+    mask keeps these two alone, so each token's output is the weighted sum of its pairs on
+    them; the oracle computes it for every token they serve, and every other row is zero."""
+    cfg = I.SKEWED
+    layer = MoELayer(cfg, DEV, weights_from=big_layer)
+    act = I.moe_activations(cfg)
+    _, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    e_max = int(torch.bincount(ids_ref.flatten().long(), minlength=cfg.E).argmax())
+    e_tail = m64_tail_expert(ids_ref, cfg.E)
+    assert e_tail is not None and e_tail != e_max
+    mask = torch.zeros(cfg.E, dtype=torch.int32)
+    mask[[e_max, e_tail]] = 1
+    out = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV), expert_mask=mask.to(DEV)).clone()
+    tokens = torch.unique(torch.cat([tokens_of_expert(ids_ref, e_max), tokens_of_expert(ids_ref, e_tail)]))
+    assert tokens.numel() >= 100 * 128
+    others = torch.ones(cfg.T, dtype=torch.bool)
+    others[tokens] = False
+    assert (out[others.to(DEV)] == 0).all()           # tokens without a pair on them: zero rows
+    ref, _, _ = oracle_moe_rows(cfg, act, tokens, expert_mask=mask)
+    assert_moe_close(out.cpu()[tokens], ref)
+
+
+@pytest.mark.parametrize("which", ["mid", "decode"])
+def test_requantised_intermediate_against_the_oracle(big_layer, which):
+    """The gate/up GEMM's epilogue output (SiLU(gate) * up re-quantised 1x128 along I: codes
+    a2 and scales s2 in the workspace) against the oracle's intermediate for every listed
+    pair. The kernel takes SiLU with the fast exponential and division and quantises
+    h * RN(1/scale) where the oracle divides exactly and works in fp64 before the final fp32
+    rounding of h, so: every scale within 2e-5 relative (the fp32 accumulation of GEMM1),
+    at most 0.5% of the codes different, none by more than one E4M3 step."""
+    cfg = MID if which == "mid" else I.DECODE
+    layer = (MoELayer(cfg, DEV).load_synthetic_weights() if which == "mid"
+             else MoELayer(cfg, DEV, weights_from=big_layer))
+    act = I.moe_activations(cfg)
+    layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    torch.cuda.synchronize()
+    sp = layer.sorted
+    cap = sp.capacity
+    a2, s2 = fused_workspace_intermediate(layer.workspace, cap, cfg.T, cfg.K, cfg.H, cfg.I)
+    a2, s2 = a2.cpu(), s2.cpu()
+    nv = int(sp.num_valid_ids.item())
+    sid = sp.sorted_ids[:nv].cpu().long()
+    blk = sp.sorted_expert_ids[: nv // layer.block_m].cpu().long()
+    P = cfg.T * cfg.K
+    a8r, ascr = O.quant_1x128(act.x)
+    diff_codes = total = 0
+    worst_step = 0
+    worst_scale = 0.0
+    for e in torch.unique(blk).tolist():
+        slots = torch.nonzero(blk.repeat_interleave(layer.block_m) == e).flatten()
+        slots = slots[sid[slots] < P]
+        t = sid[slots] // cfg.K
+        w1q, w1s, _, _ = oracle_expert(cfg, e)
+        q_ref, s_ref = O.expert_intermediate(a8r[t], ascr[t], w1q, w1s)
+        s_gpu = s2[:, slots].t()
+        rel = ((s_gpu.double() - s_ref.double()).abs() / s_ref.double().clamp_min(1e-30)).max().item()
+        worst_scale = max(worst_scale, rel)
+        q_gpu = a2[slots]
+        diff = q_gpu != q_ref
+        diff_codes += int(diff.sum())
+        total += diff.numel()
+        if diff.any():
+            worst_step = max(worst_step, int((e4m3_ordinal(q_gpu) - e4m3_ordinal(q_ref)).abs().max()))
+    assert worst_scale <= 2e-5, worst_scale
+    assert worst_step <= 1, worst_step
+    assert diff_codes <= 5e-3 * total, (diff_codes, total)
 
 
 def test_timing_hook_reports_each_fused_kernel():

@@ -8,7 +8,7 @@ from oracle import fp8moe_oracle as O
 from fp8_block_scaled_biased_b200 import binding as B
 from fp8_block_scaled_biased_b200 import inputs as I
 from fp8_block_scaled_biased_b200.layer import MoELayer
-from tests.gpu_helpers import assert_moe_close, oracle_expert, oracle_moe_rows
+from tests.gpu_helpers import assert_moe_close, full_size_tokens, oracle_expert, oracle_moe_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -55,12 +55,16 @@ def test_tp_shards_match_the_oracle_and_sum_to_the_layer(cfg, n):
     assert_moe_close(total, ref)
 
 
-def test_tp8_shard_of_the_prefill_layer_sampled_tokens():
+def test_tp8_shard_of_the_prefill_layer_many_tokens():
+    """Tensor-parallel rank 3 of 8 on the prefill layer: 256 seeded tokens, the first and
+    last token and every token of the most-loaded expert, against the oracle's shard."""
     cfg = I.PREFILL
     layer = MoELayer(cfg, DEV).load_synthetic_weights()
     shard = layer.tp_shard(3, 8)
     del layer
     act = I.moe_activations(cfg)
     out = shard.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV)).clone()
-    tokens = torch.tensor([0, 1001, 2222, 4095])
+    _, ids_ref = O.biased_grouped_topk(act.logits, act.bias, cfg.K, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    tokens, _ = full_size_tokens(cfg, ids_ref, 256, seed=8, m64_tail=False)
+    assert tokens.numel() >= 256
     assert_moe_close(out.cpu()[tokens], oracle_shard_rows(cfg, act, tokens, 3, 8))
