@@ -39,6 +39,11 @@ from fp8_block_scaled_biased_b200 import inputs as I  # noqa: E402
 
 WORKLOADS = {"tiny": I.TINY, "decode": I.DECODE, "prefill": I.PREFILL, "skewed": I.SKEWED, "profile": I.PROFILE,
              "prefill_ep8": I.PREFILL_EP8, "prefill_tp8": I.PREFILL_TP8}
+# The prefill layer split over the torchrun ranks: over I (tensor parallel: one batch of
+# 4096 tokens per step, every rank routes all of it, partial outputs reduced over NCCL) or
+# over E (expert parallel: every rank its own batch of 4096 tokens and E/N experts,
+# dispatch and return all-to-alls over NCCL).
+DIST_WORKLOADS = {"prefill_tp": I.PREFILL, "prefill_ep": I.PREFILL}
 L2_FLUSH_BYTES = 256 << 20
 METRIC = "fused FP8-blockscale MoE layer tokens/s and TFLOPS at 1 B200; % of FP8/HBM roofline"
 EXPERT_W1_BYTES = lambda c: 2 * c.I * c.H + (2 * c.I // 128) * (c.H // 128) * 4   # noqa: E731
@@ -217,8 +222,7 @@ GATE_UP_TRAFFIC = {
         "bytes": 6.857e9,
         "sha256": "22bad3149e6e9dc2dcb6fcb925d701f4e6b8b2f2e9d23c2ad816becc2c504417",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
-                   "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean; "
-                   "profiles/launches_prefill_t4096.md)",
+                   "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph` (2 launches, mean)",
     },
 }
 GEMM_SOURCES = ("fp8_block_scaled_biased_b200/csrc/gemm_sm100.cuh", "fp8_block_scaled_biased_b200/csrc/common.cuh")
@@ -302,21 +306,21 @@ def e2e_pipelined(layer, step, logits, x, h_logits, h_x, h_out, steps, world):
     return max_over_ranks(start.elapsed_time(end), world) / steps
 
 
-def run_ours(args, world, rank, local):
-    from fp8_block_scaled_biased_b200 import binding as B
-    from fp8_block_scaled_biased_b200.layer import MoELayer
+NOMINAL_HBM_GBS = 8000.0      # the ~8 TB/s HBM3e figure of the B200 spec sheet (context beside the measured peak)
 
-    cfg = WORKLOADS[args.workload]
+
+def measure_layer(args, world, local, cfg, layer, flush, headline=True):
+    """Times `args.steps` forwards of `layer` on its workload's seeded inputs (CUDA graph,
+    L2 flushed between steps, after a preheat) and returns the bench result: headline keys,
+    roofline of the dominant kernel, per-kernel times averaged over an instrumented run,
+    and (headline only) the boost-clock context figure and the end-to-end figures."""
+    from fp8_block_scaled_biased_b200 import binding as B
+
     dev = torch.device("cuda", local)
-    layer = MoELayer(cfg, dev).load_synthetic_weights()
-    if cfg.tp_ranks > 0:                            # keep only this rank's shard of the weights
-        layer = layer.tp_shard(cfg.tp_rank, cfg.tp_ranks)
-        torch.cuda.empty_cache()
     act = I.moe_activations(cfg)
     logits, bias, x = act.logits.to(dev), act.bias.to(dev), act.x.to(dev)
     mask = I.expert_mask(cfg)
     mask_dev = mask.to(dev) if mask is not None else None
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     # warm-up (also the first, eager pass through every entry point)
@@ -377,16 +381,109 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     barrier(world)
-    # The same number of steps again, straight after, with the per-kernel event
-    # records: the fused call's events then hold the last step's kernel durations.
+    # The same number of steps again, straight after, with the per-kernel event records.
+    # The fused call's events hold one call's kernel durations, so each step is read
+    # (a host wait of a few tens of microseconds) before the next one starts.
     if graph_timed is None:
         B.timing_enable(True)
-    t_starts, t_ends = run_steps(step_timed, args.steps)
-    torch.cuda.synchronize()
+    per_kernel = []
+    instrumented = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        step_timed()
+        t1.record(stream)
+        per_kernel.append(B.timing_last())
+        torch.cuda.synchronize()
+        instrumented.append(t0.elapsed_time(t1))
     clocks = sampler.stop()
-    last_kernel_ms = B.timing_last()
     B.timing_enable(False)
-    instrumented_ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(t_starts, t_ends))
+    instrumented_ms = statistics.mean(instrumented)
+    kmean = [statistics.mean(k[j] for k in per_kernel) for j in range(4)]
+    kmin = [min(k[j] for k in per_kernel) for j in range(4)]
+    kmax = [max(k[j] for k in per_kernel) for j in range(4)]
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    status = B.device_status()
+    if status:
+        raise RuntimeError(f"device error word {status} after the timed steps")
+
+    peaks = load_peaks()
+    # The timed steps run back to back under the power limit: the tensor peak is the
+    # sustained one (the burst one for the boost-clock context figure); nominal FP8:BF16 2:1.
+    fp8_peak_tflops = 2.0 * peaks["bf16_tflops_sustained"]
+    fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
+    gat_ms, g1_ms, g2_ms, cmb_ms = kmean
+    g1_t_bytes = work["gemm1_bytes"] / hbm / 1e9 * 1e3      # ms at peak HBM
+    g1_t_flops = work["gemm1_flops"] / (fp8_peak_tflops * 1e12) * 1e3
+    if g1_t_bytes >= g1_t_flops:
+        achieved = work["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9
+        roofline = {"kernel": "moe_gate_up_gemm", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS}
+    else:
+        achieved = work["gemm1_flops"] / (g1_ms * 1e-3) / 1e12
+        roofline = {"kernel": "moe_gate_up_gemm", "bound": "tensor", "achieved": achieved,
+                    "peak": fp8_peak_tflops, "unit": "TFLOP/s", "frac": achieved / fp8_peak_tflops}
+    roofline["traffic"], roofline["traffic_source"] = gate_up_traffic(cfg.name, args.traffic if headline else None)
+    roofline["algorithmic"] = work["gemm1_bytes"] if roofline["bound"] == "hbm" else work["gemm1_flops"]
+    roofline["launch_ms"] = g1_ms
+    roofline["peak_source"] = peaks["source"] + (" sustained (fp8 = 2 x bf16)" if roofline["bound"] == "tensor" else "")
+    t_layer_roof = max(work["flops"] / (fp8_peak_tflops * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
+    t_layer_roof_burst = max(work["flops"] / (fp8_peak_burst * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
+    t_layer_roof_nominal = max(work["flops"] / (fp8_peak_tflops * 1e12), work["layer_bytes"] / (NOMINAL_HBM_GBS * 1e9)) * 1e3
+    mhz = clocks.get("sm_mhz")
+    cycles = (lambda ms: ms * 1e-3 * mhz * 1e6) if mhz else (lambda ms: None)
+
+    tokens = cfg.T * world
+    result = {
+        "metric": METRIC,
+        "value": tokens / (ms_per_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8_e4m3fn x fp8_e4m3fn -> fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded; random-init weights quantised to FP8 in 128x128 blocks)",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "groups": cfg.G,
+                   "topk_group": cfg.TG, "topk": cfg.K, "I": cfg.I, "block_m": layer.block_m,
+                   "parallelism": f"dp{world} (replicated layer, token batches per GPU)",
+                   "l2": "flushed between steps (256 MB write); touched expert weights exceed L2 anyway",
+                   "cuda_graph": graph is not None, **ep_config(cfg)},
+        "tflops": work["flops"] * world / (ms_per_step * 1e-3) / 1e12,
+        "layer_roofline": {"ms": t_layer_roof, "frac": t_layer_roof / ms_per_step,
+                           "frac_vs_nominal_8tbs": t_layer_roof_nominal / ms_per_step,
+                           "flops": work["flops"], "bytes": work["layer_bytes"],
+                           "touched_experts": work["n_experts"], "fp8_peak_tflops": fp8_peak_tflops,
+                           "fp8_peak_source": peaks["source"] + " sustained (fp8 = 2 x bf16)",
+                           "hbm_gbs": hbm, "hbm_source": peaks["source"]},
+        "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
+        "instrumented_ms_per_step": instrumented_ms,
+        "kernels_ms": {"moe_gather": gat_ms, "moe_gate_up_gemm": g1_ms, "moe_down_gemm": g2_ms, "moe_combine": cmb_ms,
+                       "route_sort_quant": instrumented_ms - sum(kmean),
+                       "min": dict(zip(("moe_gather", "moe_gate_up_gemm", "moe_down_gemm", "moe_combine"), kmin)),
+                       "max": dict(zip(("moe_gather", "moe_gate_up_gemm", "moe_down_gemm", "moe_combine"), kmax)),
+                       "source": f"mean over the {args.steps} steps of a second run of the timed steps with the "
+                                 "fused call's kernel events recorded; route_sort_quant = instrumented mean step - "
+                                 "the four"},
+        "kernels_mcycles": {"moe_gate_up_gemm": cycles(g1_ms) and cycles(g1_ms) / 1e6,
+                            "moe_down_gemm": cycles(g2_ms) and cycles(g2_ms) / 1e6,
+                            "sm_mhz": mhz, "source": "kernel ms x median sampled SM clock"},
+        "roofline": roofline,
+        "gpu_launches": args.steps * layer.launches_per_forward,
+        "clocks": clocks,
+        "wall_s_timed": wall,
+    }
+    if not headline:
+        del graph, graph_timed
+        return result
+
     # Context only: the same steps each started from an idle GPU (5 ms of host sleep
     # before each), i.e. at the boost clock of a layer run alone, not under sustained load.
     burst_ms = []
@@ -401,12 +498,10 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         burst_ms.append(b0.elapsed_time(b1))
     burst_ms_per_step = max_over_ranks(statistics.median(burst_ms), world)
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms), world)
-    ms_per_step = total_ms / args.steps
-    status = B.device_status()
-    if status:
-        raise RuntimeError(f"device error word {status} after the timed steps")
+    result["burst"] = {"ms_per_step": burst_ms_per_step,
+                       "layer_roofline_frac": t_layer_roof_burst / burst_ms_per_step,
+                       "method": "median of the same steps each started after 5 ms of idle GPU (boost clock); "
+                                 "context only, the headline value is the sustained back-to-back run"}
 
     # End to end through the public API with host buffers. Serial: per step, the pinned H2D
     # copies of the inputs, the forward and the D2H copy of the output on one stream.
@@ -432,77 +527,134 @@ def run_ours(args, world, rank, local):
     # H2D and step i-1's D2H run on their own copy streams while step i computes. Every step
     # still moves its own inputs and output across PCIe; the time is that of all steps.
     e2e_ms = e2e_pipelined(layer, step, logits, x, h_logits, h_x, h_out, args.steps, world)
+    result["e2e"] = {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                     "h2d_bytes_per_step": act.logits.numel() * 4 + act.x.numel() * 2,
+                     "d2h_bytes_per_step": cfg.T * cfg.H * 2, "ms_per_step": e2e_ms,
+                     "method": "pinned host buffers through layer.forward; two-deep pipeline: step i+1's H2D and "
+                               "step i-1's D2H overlap step i's forward on separate copy streams; no L2 flush "
+                               "between these steps (each step reads its touched experts' weights, more than L2)",
+                     "serial": {"value": tokens / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}}
+    del graph, graph_timed
+    return result
 
-    peaks = load_peaks()
-    # The timed steps run back to back under the power limit: the tensor peak is the
-    # sustained one (the burst one for the boost-clock context figure); nominal FP8:BF16 2:1.
-    fp8_peak_tflops = 2.0 * peaks["bf16_tflops_sustained"]
-    fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
-    hbm = peaks["hbm_gbs"]
-    gat_ms, g1_ms, g2_ms, cmb_ms = last_kernel_ms[:4]
-    g1_t_bytes = work["gemm1_bytes"] / hbm / 1e9 * 1e3      # ms at peak HBM
-    g1_t_flops = work["gemm1_flops"] / (fp8_peak_tflops * 1e12) * 1e3
-    if g1_t_bytes >= g1_t_flops:
-        roofline = {"kernel": "moe_gate_up_gemm", "bound": "hbm", "achieved": work["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9,
-                    "peak": hbm, "unit": "GB/s"}
+
+# The other workloads of the same layer timed by the default run, next to the prefill
+# headline: the decode and skewed batches (same expert weights) and the standalone GEMM.
+EXTRA_WORKLOADS = ("decode", "skewed", "gemm")
+EXTRA_KEYS = ("value", "unit", "ms_per_step", "steps", "warmup", "tflops", "step_ms", "layer_roofline", "roofline",
+              "kernels_ms", "kernels_mcycles", "clocks", "config", "gpu_launches", "l2_warm")
+
+
+def run_distributed(args, world, rank, local):
+    """prefill_tp / prefill_ep: the layer split over the ranks (eager steps: the step holds
+    NCCL collectives and, for expert parallelism, a host read of the all-to-all counts)."""
+    from fp8_block_scaled_biased_b200 import binding as B
+    from fp8_block_scaled_biased_b200 import distributed as D
+    from fp8_block_scaled_biased_b200.layer import MoELayer
+
+    cfg = DIST_WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    act = I.moe_activations(cfg)
+    logits, bias, x = act.logits.to(dev), act.bias.to(dev), act.x.to(dev)
+    if args.workload == "prefill_tp":
+        full = MoELayer(cfg, dev).load_synthetic_weights()
+        model = D.TensorParallelMoE(full)
+        del full
+        torch.cuda.empty_cache()
+        routing_layer = model.shard
     else:
-        roofline = {"kernel": "moe_gate_up_gemm", "bound": "tensor",
-                    "achieved": work["gemm1_flops"] / (g1_ms * 1e-3) / 1e12, "peak": fp8_peak_tflops, "unit": "TFLOP/s"}
-    roofline["frac"] = roofline["achieved"] / roofline["peak"]
-    roofline["traffic"], roofline["traffic_source"] = gate_up_traffic(cfg.name, args.traffic)
-    roofline["peak_source"] = peaks["source"] + (" sustained (fp8 = 2 x bf16)" if roofline["bound"] == "tensor" else "")
-    t_layer_roof = max(work["flops"] / (fp8_peak_tflops * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
-    t_layer_roof_burst = max(work["flops"] / (fp8_peak_burst * 1e12), work["layer_bytes"] / (hbm * 1e9)) * 1e3
-
-    tokens = cfg.T * world
-    result = {
-        "metric": METRIC,
-        "value": tokens / (ms_per_step * 1e-3),
-        "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": ms_per_step,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+        e0, e1 = D.ep_expert_range(cfg.E, rank, world)
+        model = D.ExpertParallelMoE(cfg, D.ExpertShard(cfg, e0, e1, dev).load_synthetic_weights())
+        routing_layer = MoELayer(cfg, dev)        # routing only, for the work count
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        out = model.forward(logits, bias, x)
+    torch.cuda.synchronize()
+    assert B.device_status() == 0, "device error word set during warm-up"
+    B.moe_biased_grouped_topk(logits, bias, routing_layer.topk_w, routing_layer.topk_ids, cfg.G, cfg.TG, cfg.renorm,
+                              cfg.scale)
+    work = layer_work(cfg, routing_layer.topk_ids)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    barrier(world)
+    torch.cuda.synchronize()
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        st[i].record(stream)
+        out = model.forward(logits, bias, x)
+        en[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(st, en)]
+    ms_per_step = max_over_ranks(sum(step_ms), world) / args.steps
+    if B.device_status():
+        raise RuntimeError("device error word set during the timed steps")
+    peaks = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    hbm = peaks["hbm_gbs"]
+    tp = args.workload == "prefill_tp"
+    batches = 1 if tp else world                   # token batches processed per step by the whole job
+    flops = work["flops"] * batches
+    wbytes = work["layer_bytes"] - (cfg.T * cfg.E * 4 + cfg.E * 4 + 4 * cfg.T * cfg.H)
+    act_bytes = (cfg.T * cfg.E * 4 + cfg.E * 4 + 4 * cfg.T * cfg.H) * (world if tp else batches)
+    t_roof = max(flops / world / (fp8_peak * 1e12), (wbytes + act_bytes) / world / (hbm * 1e9)) * 1e3
+    tokens = cfg.T * batches
+    del out
+    return {
+        "metric": METRIC, "value": tokens / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if tp else "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3fn x fp8_e4m3fn -> fp32 accumulate, bf16 out",
         "data": "synthetic (seeded; random-init weights quantised to FP8 in 128x128 blocks)",
-        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "groups": cfg.G,
-                   "topk_group": cfg.TG, "topk": cfg.K, "I": cfg.I, "block_m": layer.block_m,
-                   "parallelism": f"dp{world} (replicated layer, token batches per GPU)",
-                   "l2": "flushed between steps (256 MB write); touched expert weights exceed L2 anyway",
-                   "cuda_graph": graph is not None, **ep_config(cfg)},
-        "tflops": work["flops"] * world / (ms_per_step * 1e-3) / 1e12,
-        "layer_roofline": {"ms": t_layer_roof, "frac": t_layer_roof / ms_per_step,
-                           "flops": work["flops"], "bytes": work["layer_bytes"],
-                           "touched_experts": work["n_experts"], "fp8_peak_tflops": fp8_peak_tflops,
-                           "fp8_peak_source": peaks["source"] + " sustained (fp8 = 2 x bf16)",
-                           "hbm_gbs": hbm},
+        "config": {"workload": f"{cfg.name}_{'tp' if tp else 'ep'}{world}", "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                   "topk": cfg.K, "I": cfg.I,
+                   "parallelism": (f"tp{world}: intermediate columns split over the ranks, one batch of {cfg.T} "
+                                   "tokens per step, partial outputs summed by an fp32 NCCL reduce-scatter and a "
+                                   "bf16 all-gather") if tp else
+                                  (f"ep{world}: experts split over the ranks, each rank its own batch of {cfg.T} "
+                                   "tokens, dispatch and return all-to-alls over NCCL"),
+                   "l2": "flushed between steps (256 MB write)", "cuda_graph": False},
+        "tflops": flops / (ms_per_step * 1e-3) / 1e12,
+        "layer_roofline": {"ms": t_roof, "frac": t_roof / ms_per_step, "flops": flops,
+                           "bytes": wbytes + act_bytes, "touched_experts": work["n_experts"],
+                           "note": "whole-job work spread evenly over the ranks; collective time not in the bound"},
         "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
-        "instrumented_ms_per_step": instrumented_ms,
-        "burst": {"ms_per_step": burst_ms_per_step, "layer_roofline_frac": t_layer_roof_burst / burst_ms_per_step,
-                  "method": "median of the same steps each started after 5 ms of idle GPU (boost clock); "
-                            "context only, the headline value is the sustained back-to-back run"},
-        "kernels_ms": {"moe_gather": gat_ms, "moe_gate_up_gemm": g1_ms, "moe_down_gemm": g2_ms, "moe_combine": cmb_ms,
-                       "route_sort_quant": instrumented_ms - gat_ms - g1_ms - g2_ms - cmb_ms,
-                       "source": "the last step of a second run of the timed steps with the fused call's kernel "
-                                 "events recorded; route_sort_quant = instrumented mean step - the four"},
-        "roofline": roofline,
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": act.logits.numel() * 4 + act.x.numel() * 2,
-                "d2h_bytes_per_step": cfg.T * cfg.H * 2, "ms_per_step": e2e_ms,
-                "method": "pinned host buffers through layer.forward; two-deep pipeline: step i+1's H2D and "
-                          "step i-1's D2H overlap step i's forward on separate copy streams; no L2 flush "
-                          "between these steps (each step reads its touched experts' weights, more than L2)",
-                "serial": {"value": tokens / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}},
-        "gpu_launches": args.steps * layer.launches_per_forward,
-        "clocks": clocks,
-        "wall_s_timed": wall,
+        "gpu_launches": None, "clocks": clocks,
     }
+
+
+def run_ours(args, world, rank, local):
+    from fp8_block_scaled_biased_b200.layer import MoELayer
+
+    if args.workload in DIST_WORKLOADS:
+        return run_distributed(args, world, rank, local)
+    cfg = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    layer = MoELayer(cfg, dev).load_synthetic_weights()
+    if cfg.tp_ranks > 0:                            # keep only this rank's shard of the weights
+        layer = layer.tp_shard(cfg.tp_rank, cfg.tp_ranks)
+        torch.cuda.empty_cache()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    result = measure_layer(args, world, local, cfg, layer, flush, headline=True)
+    if args.workload == "prefill" and world == 1 and not args.no_workloads:
+        extras = {}
+        for name in EXTRA_WORKLOADS:
+            if name == "gemm":
+                r = run_gemm(args, world, rank, local, cpu=False)
+            else:
+                other = MoELayer(WORKLOADS[name], dev, weights_from=layer)
+                r = measure_layer(args, world, local, WORKLOADS[name], other, flush, headline=False)
+                del other
+                torch.cuda.empty_cache()
+            extras[name] = {k: r[k] for k in EXTRA_KEYS if k in r}
+        result["workloads"] = extras
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample_tokens, device=dev)
-    del graph
     return result
 
 
@@ -564,8 +716,9 @@ def cpu_baseline(cfg, n_tokens, device="cuda", min_seconds=10.0):
                       f"before timing), {len(times)} passes in {sum(times):.1f} s"}
 
 
-def run_gemm(args, world, rank, local):
-    """The standalone block-scale GEMM (C = A . B^T with 1x128 / 128x128 FP8 scales), A pre-quantised."""
+def run_gemm(args, world, rank, local, cpu=True):
+    """The standalone block-scale GEMM (C = A . B^T with 1x128 / 128x128 FP8 scales), A pre-quantised.
+    cpu=False leaves out the oracle's CPU baseline."""
     from fp8_block_scaled_biased_b200 import binding as B
 
     cfg = I.GEMM
@@ -643,7 +796,7 @@ def run_gemm(args, world, rank, local):
         "gpu_launches": args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import fp8moe_oracle as O
         rows = torch.arange(0, cfg.M, cfg.M // 8)
         qa_h, sa_h = O.quant_1x128(a[rows].cpu())
@@ -689,7 +842,7 @@ def run_reference_gemm(args, world):
 def run_reference(args, world, rank):
     if args.workload == "gemm":
         return run_reference_gemm(args, world)
-    cfg = WORKLOADS[args.workload]
+    cfg = WORKLOADS[args.workload] if args.workload in WORKLOADS else DIST_WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     runner = OracleSample(cfg, args.ref_sample_tokens, device=dev)
     for _ in range(args.warmup):
@@ -719,11 +872,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["gemm"], default="prefill",
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DIST_WORKLOADS) + ["gemm"], default="prefill",
                     help="MoE layer workload, or gemm: the standalone block-scale GEMM (M=2048, N=4096, K=7168)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="prefill only: leave out the decode, skewed and GEMM workloads timed beside the headline")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8,
                     help="tokens of the workload the oracle runs for cpu_baseline")
     ap.add_argument("--ref-sample-tokens", type=int, default=1,
