@@ -1,0 +1,244 @@
+"""Multi-GPU forms of the FP8 block-scaled MoE layer, one process per GPU over
+torch.distributed (NCCL between GPUs; gloo for the rank logic on the CPU).
+
+"Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang" runs the layer at
+TP8 (section "Performance Reproduction for AITER-Optimized in SGLang", --tp 8),
+summing the ranks' outputs with the custom all-reduce of section "Other
+Operators", and gives asm_moe an expert_mask (section "Blockscale FP8 MoE
+Computation"), the hook of expert parallelism. Two forms are built here:
+
+Tensor parallelism over I (TensorParallelMoE). Every rank routes every token and
+runs its shard of each expert's intermediate columns (MoELayer.tp_shard); the
+ranks' bf16 partial outputs are summed by tp_reduce: an fp32 reduce-scatter (each
+rank sums one slice of the tokens over all ranks) and a bf16 all-gather of the
+rounded slices.
+
+Expert parallelism over E (ExpertParallelMoE). Rank r holds experts
+[r*E/n, (r+1)*E/n) and its own batch of tokens. It routes and quantises its
+tokens, then one all-to-all sends every (token, owner rank) pair that has work
+there: the token's FP8 row, its 1x128 scales, and its top-k ids (as the owner's
+local ids; pairs of other ranks carry a sentinel id that the owner's sort drops)
+and weights, packed in one byte row. The owner sorts what it received with an
+expert mask and runs the fused MoE on its experts; a second all-to-all returns
+each received row's partial output (the bf16 sum over that rank's pairs), and the
+origin adds, per token, the partial rows in ascending rank order in fp32 and
+rounds to bf16 once. The result is deterministic for a given rank count.
+
+The compute is the library's kernels (routing, quantisation, sort, fused MoE);
+the collectives are NCCL's; what lies between them here is index bookkeeping and
+byte packing on the device (torch indexing), with the local compute passed in as
+a callable so that the rank logic runs unchanged on the CPU with the oracle in
+its place.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+import torch.distributed as dist
+
+from . import binding as B
+from . import inputs as I
+
+
+def _world(group):
+    return dist.get_world_size(group) if dist.is_initialized() else 1
+
+
+def _rank(group):
+    return dist.get_rank(group) if dist.is_initialized() else 0
+
+
+# ---------------------------------------------------------------------------------- tensor parallel
+
+def tp_reduce(partial: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum over the group's ranks of each rank's partial output [T, H] (bf16), returned
+    on every rank as bf16 [T, H]: the tokens are split into one slice per rank, each slice
+    summed over the ranks in fp32 (reduce-scatter) and rounded to bf16 once, then the
+    slices gathered (all-gather). With one rank the partial is the output."""
+    n = _world(group)
+    if n == 1:
+        return partial
+    T, H = partial.shape
+    Tp = -(-T // n) * n
+    full = torch.zeros(Tp, H, dtype=torch.float32, device=partial.device)
+    full[:T].copy_(partial)
+    piece = torch.empty(Tp // n, H, dtype=torch.float32, device=partial.device)
+    dist.reduce_scatter_tensor(piece, full, op=dist.ReduceOp.SUM, group=group)
+    out = torch.empty(Tp, H, dtype=torch.bfloat16, device=partial.device)
+    dist.all_gather_into_tensor(out, piece.to(torch.bfloat16), group=group)
+    return out[:T]
+
+
+class TensorParallelMoE:
+    """One rank of the layer split over I: its shard (rank, n) of every expert, the whole
+    routing, and tp_reduce of the partial outputs."""
+
+    def __init__(self, layer, group=None):
+        """layer: the whole MoELayer (its shard is copied out) or an already-sharded one
+        whose cfg.tp_ranks / tp_rank match the group."""
+        self.group = group
+        n, r = _world(group), _rank(group)
+        if layer.cfg.tp_ranks == n and layer.cfg.tp_rank == r:
+            self.shard = layer
+        else:
+            self.shard = layer.tp_shard(r, n) if n > 1 else layer
+
+    def forward(self, logits, bias, x):
+        partial = self.shard.forward(logits, bias, x)
+        return tp_reduce(partial, self.group)
+
+
+# ---------------------------------------------------------------------------------- expert parallel
+
+def ep_expert_range(E: int, rank: int, n: int):
+    """Experts [e0, e1) that rank `rank` of `n` holds (contiguous ranges; E % n == 0)."""
+    if n < 1 or E % n:
+        raise ValueError(f"E={E} experts cannot be split evenly over {n} ranks")
+    per = E // n
+    return rank * per, (rank + 1) * per
+
+
+@dataclasses.dataclass
+class EpPlan:
+    """Where a rank's tokens went: for each destination rank d, the tokens (ascending)
+    that have at least one pair on d's experts, in the order their rows were sent."""
+    tokens: list          # per destination: int64 [n_d] token indices
+    send_counts: list     # per destination: n_d
+    recv_counts: list     # per source: rows received from it
+    T: int
+    H: int
+
+
+def _row_bytes(H, K):
+    return H + 4 * (H // 128) + 4 * K + 4 * K
+
+
+def ep_dispatch(a8, a8_scale, topk_ids, topk_weights, E, group=None):
+    """Sends each (token, owner rank) pair with work to the owner. a8 fp8 [T, H],
+    a8_scale fp32 [T, H/128] (row-major), topk_ids int32 [T, K], topk_weights fp32 [T, K].
+
+    Returns (received, plan): received = (a8 fp8 [m, H], scales fp32 [m, H/128], local ids
+    int32 [m, K], weights fp32 [m, K]) for the m rows this rank received, sources in rank
+    order; a pair of another rank carries the local id E/n (one past this rank's experts)."""
+    n, r = _world(group), _rank(group)
+    T, H = a8.shape
+    K = topk_ids.shape[1]
+    per = E // n
+    dev = a8.device
+    owner = topk_ids.long() // per                                   # [T, K]
+    has = torch.zeros(T, n, dtype=torch.bool, device=dev)
+    has.scatter_(1, owner.clamp(0, n - 1), True)
+    tokens = [torch.nonzero(has[:, d]).flatten() for d in range(n)]
+    send_counts = [int(t.numel()) for t in tokens]
+    idx = torch.cat(tokens) if tokens else torch.empty(0, dtype=torch.long, device=dev)
+    dest = torch.repeat_interleave(torch.arange(n, device=dev), torch.tensor(send_counts, device=dev))
+    ids = topk_ids[idx].long()
+    local = torch.where(ids // per == dest[:, None], ids - dest[:, None] * per, torch.full_like(ids, per))
+    rb = _row_bytes(H, K)
+    send = torch.empty(idx.numel(), rb, dtype=torch.uint8, device=dev)
+    o1, o2, o3 = H, H + 4 * (H // 128), H + 4 * (H // 128) + 4 * K
+    send[:, :o1] = a8.view(torch.uint8)[idx]
+    send[:, o1:o2] = a8_scale[idx].contiguous().view(torch.uint8)
+    send[:, o2:o3] = local.to(torch.int32).contiguous().view(torch.uint8)
+    send[:, o3:] = topk_weights[idx].contiguous().view(torch.uint8)
+    counts = torch.tensor(send_counts, dtype=torch.int64, device=dev)
+    recv_c = torch.empty_like(counts)
+    if n > 1:
+        dist.all_to_all_single(recv_c, counts, group=group)
+    else:
+        recv_c.copy_(counts)
+    recv_counts = [int(c) for c in recv_c.tolist()]
+    recv = torch.empty(sum(recv_counts), rb, dtype=torch.uint8, device=dev)
+    if n > 1:
+        dist.all_to_all_single(recv, send, recv_counts, send_counts, group=group)
+    else:
+        recv.copy_(send)
+    m = recv.shape[0]
+    r_a8 = recv[:, :o1].contiguous().view(a8.dtype)
+    r_sc = recv[:, o1:o2].contiguous().view(torch.float32).view(m, H // 128)
+    r_ids = recv[:, o2:o3].contiguous().view(torch.int32).view(m, K)
+    r_w = recv[:, o3:].contiguous().view(torch.float32).view(m, K)
+    return (r_a8, r_sc, r_ids, r_w), EpPlan(tokens, send_counts, recv_counts, T, H)
+
+
+def ep_combine(partials: torch.Tensor, plan: EpPlan, group=None) -> torch.Tensor:
+    """Returns each received row's partial output (bf16 [m, H], rows in the order received)
+    to its origin and sums, per token, the rows from all ranks in ascending rank order in
+    fp32, rounded to bf16 once. A token with no pair anywhere gets a zero row."""
+    n = _world(group)
+    H = plan.H
+    back = torch.empty(sum(plan.send_counts), H, dtype=partials.dtype, device=partials.device)
+    if n > 1:
+        dist.all_to_all_single(back, partials.contiguous(), plan.send_counts, plan.recv_counts, group=group)
+    else:
+        back.copy_(partials)
+    acc = torch.zeros(plan.T, H, dtype=torch.float32, device=partials.device)
+    off = 0
+    for d in range(n):
+        c = plan.send_counts[d]
+        if c:
+            # each token appears at most once per source rank: no two adds hit one row here
+            acc.index_add_(0, plan.tokens[d], back[off:off + c].float())
+        off += c
+    return acc.to(torch.bfloat16)
+
+
+class ExpertShard:
+    """The experts [e0, e1) of a layer, as one expert-parallel rank holds them: w1
+    [n_e, 2I, H], w2 [n_e, H, I] and their 128x128 block scales, on the device."""
+
+    def __init__(self, cfg: I.MoEConfig, e0: int, e1: int, device="cuda"):
+        self.cfg, self.e0, self.e1 = cfg, e0, e1
+        ne, H, Im = e1 - e0, cfg.H, cfg.I
+        self.w1 = torch.empty(ne, 2 * Im, H, dtype=B.FP8, device=device)
+        self.w1_scale = torch.empty(ne, 2 * Im // 128, H // 128, dtype=torch.float32, device=device)
+        self.w2 = torch.empty(ne, H, Im, dtype=B.FP8, device=device)
+        self.w2_scale = torch.empty(ne, H // 128, Im // 128, dtype=torch.float32, device=device)
+        self.block_m = B.moe_block_m()
+        # sort over the rank's experts plus one sentinel expert (other ranks' pairs), masked out
+        self.sort_mask = torch.ones(ne + 1, dtype=torch.int32, device=device)
+        self.sort_mask[ne] = 0
+
+    def load_synthetic_weights(self):
+        """Draw and quantise the raw weights of global experts e0..e1-1 (as MoELayer does)."""
+        for i, e in enumerate(range(self.e0, self.e1)):
+            B.fp8_per_block_quant(I.expert_weight_raw(self.cfg, "w1", e, self.w1.device), q=self.w1[i],
+                                  scales=self.w1_scale[i])
+            B.fp8_per_block_quant(I.expert_weight_raw(self.cfg, "w2", e, self.w2.device), q=self.w2[i],
+                                  scales=self.w2_scale[i])
+        return self
+
+    def __call__(self, a8, scales, ids, weights):
+        """The fused MoE over received rows: a8 fp8 [m, H], scales fp32 [m, H/128], local ids
+        int32 [m, K] (sentinel n_e = another rank's pair), weights fp32 [m, K] -> bf16 [m, H]."""
+        m, H = a8.shape
+        K = ids.shape[1]
+        ne = self.e1 - self.e0
+        out = torch.empty(m, H, dtype=torch.bfloat16, device=a8.device)
+        if m == 0:
+            return out
+        sp = B.moe_align_sort(ids, weights, ne + 1, self.block_m, expert_mask=self.sort_mask)
+        B.fused_moe_fp8_blockscale_g1u1(out, a8, self.w1, self.w2, sp, K, scales.t().contiguous(), self.w1_scale,
+                                        self.w2_scale)
+        return out
+
+
+class ExpertParallelMoE:
+    """One expert-parallel rank: its experts (an ExpertShard or any callable with its
+    signature), the whole routing of its own tokens, and the dispatch/return all-to-alls."""
+
+    def __init__(self, cfg: I.MoEConfig, local_experts, group=None):
+        self.cfg, self.local, self.group = cfg, local_experts, group
+        ep_expert_range(cfg.E, _rank(group), _world(group))
+
+    def forward(self, logits, bias, x):
+        cfg = self.cfg
+        T = x.shape[0]
+        w = torch.empty(T, cfg.K, dtype=torch.float32, device=x.device)
+        ids = torch.empty(T, cfg.K, dtype=torch.int32, device=x.device)
+        B.moe_biased_grouped_topk(logits, bias, w, ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+        a8, a8_scale = B.fp8_per_token_group_quant(x, 128, column_major_scales=False)
+        received, plan = ep_dispatch(a8, a8_scale, ids, w, cfg.E, self.group)
+        partial = self.local(*received)
+        return ep_combine(partial, plan, self.group)
