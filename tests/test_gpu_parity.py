@@ -381,6 +381,8 @@ def test_requantised_intermediate_against_the_oracle(big_layer, which):
         total += diff.numel()
         if diff.any():
             worst_step = max(worst_step, int((e4m3_ordinal(q_gpu) - e4m3_ordinal(q_ref)).abs().max()))
+    print(f"{cfg.name}: scales within {worst_scale:.2e} relative, {diff_codes} of {total} codes differ "
+          f"({diff_codes / total:.2e}), by at most {worst_step} step")
     assert worst_scale <= 2e-5, worst_scale
     assert worst_step <= 1, worst_step
     assert diff_codes <= 5e-3 * total, (diff_codes, total)
