@@ -279,7 +279,13 @@ def selftest_gemm_stall(A, B, a_scale, b_scale, out, stall_kb):
     _check("fp8moe_selftest_gemm_stall", rc)
 
 
-def fused_moe_workspace_bytes(T, topk, E, H, I, block_m):
+def fused_moe_workspace_bytes(T, topk, E, H, I, block_m, capacity=None):
+    """Workspace bytes of the fused call. capacity: the sorted list's capacity when it is larger
+    than moe_align_sort_capacity(T, topk, E, block_m) (a list sorted over more experts than
+    the weights hold, e.g. with a masked-out sentinel expert); the query is then made for the
+    expert count whose capacity covers it."""
+    if capacity is not None and block_m > 1:
+        E = max(E, -(-(int(capacity) - T * topk) // (block_m - 1)))
     return load_library().fused_moe_fp8_blockscale_g1u1_workspace(T, topk, E, H, I, block_m)
 
 
@@ -335,8 +341,8 @@ def fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_pairs: SortedPairs, to
     T, H, I, E = _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale)
     sp = sorted_pairs
     lib = load_library()
-    need = lib.fused_moe_fp8_blockscale_g1u1_workspace(T, topk, E, H, I, sp.block_m)
     if workspace is None:
+        need = fused_moe_workspace_bytes(T, topk, E, H, I, sp.block_m, capacity=sp.capacity)
         workspace = torch.empty(need, dtype=torch.uint8, device=a8.device)
     rc = lib.fused_moe_fp8_blockscale_g1u1(
         _ptr(out), _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights),

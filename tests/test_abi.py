@@ -149,3 +149,14 @@ def test_bf16_routing_and_masked_sort_reject_bad_arguments(lib):
 def test_selftest_stall_rejects_a_k_block_out_of_range(lib):
     rc, msg = _rc(lib, "fp8moe_selftest_gemm_stall", P, P, P, P, P, 256, 128, 256, 256, 2, None)
     assert rc == 1 and "stall_kb" in msg
+
+
+def test_workspace_bytes_cover_a_sorted_list_over_more_experts(lib):
+    """A list sorted over E+1 experts (a masked-out sentinel expert, as the expert-parallel
+    owner sorts) has a larger capacity than the weights' E implies: the binding sizes the
+    fused call's workspace for that capacity."""
+    T, K, E, H, I, bm = 256, 4, 8, 1024, 512, 128
+    cap = lib.moe_align_sort_capacity(T, K, E + 1, bm)
+    assert B.fused_moe_workspace_bytes(T, K, E, H, I, bm, capacity=cap) == \
+        lib.fused_moe_fp8_blockscale_g1u1_workspace(T, K, E + 1, H, I, bm)
+    assert B.fused_moe_workspace_bytes(T, K, E, H, I, bm) < B.fused_moe_workspace_bytes(T, K, E, H, I, bm, capacity=cap)
