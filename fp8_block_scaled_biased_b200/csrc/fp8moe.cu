@@ -531,10 +531,15 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (cudaMemsetAsync(n_present, 0, 16 + static_cast<size_t>(T) * topk, st) != cudaSuccess)
     return check_launch("fused_moe (pair flags)");
   timing_record(0, st);
-  moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, a1_scale, sorted_ids, sorted_expert_ids,
-                                                            num_valid_ids, T, topk, H, static_cast<int>(capacity),
-                                                            a8s, s1s, pair_flag, n_present);
+  // pair -> slot map of the gather, kept in the pair-row region (P * 4 <= P * H * 2
+  // bytes) that the down GEMM writes only later
+  int* inv = reinterpret_cast<int*>(ystage);
+  moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a1_scale, sorted_ids, sorted_expert_ids, num_valid_ids,
+                                                            T, topk, H, static_cast<int>(capacity), s1s, pair_flag,
+                                                            n_present, inv);
   if (int rc = check_launch("fused_moe (gather)")) return rc;
+  moe_gather_rows_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, T, topk, H, pair_flag, inv, a8s);
+  if (int rc = check_launch("fused_moe (gather rows)")) return rc;
   timing_record(1, st);
 
   GemmArgs up{};

@@ -3,9 +3,10 @@
 // "Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang", section
 // "Blockscale FP8 MoE Computation": the fused MoE reads the sorted token-expert
 // slots (moe_sorting) and writes the top-k weighted sum per token (moe_buf).
-// moe_gather_kernel puts each slot's FP8 activation row and scales into slot
-// order for the gate/up GEMM's TMA loads; moe_combine_kernel sums a token's
-// topk weighted down-projection rows in a fixed order.
+// moe_gather_kernel and moe_gather_rows_kernel put each slot's FP8 activation
+// row and scales into slot order for the gate/up GEMM's TMA loads;
+// moe_combine_kernel sums a token's topk weighted down-projection rows in a
+// fixed order.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -16,66 +17,41 @@ namespace fp8moe {
 
 constexpr int kMoeBlockRows = 128;            // rows per sorted block (the GEMM tile's M)
 
-// Copies each sorted slot's token row of a8 [T, H] (and its H/128 scales from
-// a1_scale [H/128, T]) into slot order, sets pair_flag[p] = 1 for every pair p
-// in the list and adds the number of distinct listed pairs to *n_present (the
-// caller zeroes both first; pair_flag is 4-byte aligned). A pair id listed twice
-// (not a moe_align_sort result) is counted once, so *n_present == T*topk means
-// every pair is present. Padding slots are skipped: the GEMMs treat rows
-// independently and never store padding rows.
 constexpr int kGatherWarps = 8;
+// Slot-ordered pass over the sorted list: sets pair_flag[p] = 1 for every listed
+// pair p and adds the number of distinct listed pairs to *n_present (the caller
+// zeroes both first; pair_flag is 4-byte aligned; a pair id listed twice, which
+// moe_align_sort never produces, is counted once, so *n_present == T*topk means
+// every pair is present), writes the pair -> slot map inv[p] (valid where the
+// flag is set) and copies each slot's H/128 scales from a1_scale [H/128, T] into
+// slot order. Padding slots are skipped: the GEMMs treat rows independently and
+// never store padding rows.
 __global__ void __launch_bounds__(32 * kGatherWarps)
-moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_scale,
-                  const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ sorted_expert_ids,
-                  const int32_t* __restrict__ num_valid_ids, int T, int topk, int H, int cap,
-                  uint8_t* __restrict__ a8s, float* __restrict__ s1s, uint8_t* __restrict__ pair_flag,
-                  int* __restrict__ n_present) {
+moe_gather_kernel(const float* __restrict__ a1_scale, const int32_t* __restrict__ sorted_ids,
+                  const int32_t* __restrict__ sorted_expert_ids, const int32_t* __restrict__ num_valid_ids, int T,
+                  int topk, int H, int cap, float* __restrict__ s1s, uint8_t* __restrict__ pair_flag,
+                  int* __restrict__ n_present, int* __restrict__ inv) {
   __shared__ int cta_present;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) cta_present = 0;
   __syncthreads();
-  int warp_present = 0;
+  int present = 0;
   const int P = T * topk;
   const int nv = min(max(*num_valid_ids, 0), cap);
-  // The gate/up GEMM's tile order needs each expert's blocks to be contiguous, as the
-  // sort's ascending expert order makes them: flag a decreasing pair of block ids.
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b + 1 < nv / kMoeBlockRows; b += gridDim.x * blockDim.x)
     if (sorted_expert_ids[b] > sorted_expert_ids[b + 1]) raise_device_error(FP8MOE_DEVERR_BLOCK_ORDER);
   const int KB = H / 128;
-  const int vec_per_row = H / 16;
-  for (int slot = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); slot < nv; slot += gridDim.x * kGatherWarps) {
+  for (int slot = blockIdx.x * blockDim.x + threadIdx.x; slot < nv; slot += gridDim.x * blockDim.x) {
     const int sid = sorted_ids[slot];
     if (sid < 0 || sid >= P) continue;
-    if (lane == 0) {
-      // set the pair's flag byte through its 32-bit word; count the pair only if
-      // this slot set it first
-      const unsigned bit = 1u << (8 * (sid & 3));
-      if ((atomicOr(reinterpret_cast<unsigned*>(pair_flag) + (sid >> 2), bit) & bit) == 0) ++warp_present;
-    }
-    const int t = sid / topk;
-    const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
-    uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
-    // issue a batch of loads before their stores, so the row costs one round trip per batch
-    constexpr int kBatch = 16;
-    for (int v0 = 0; v0 < vec_per_row; v0 += 32 * kBatch) {
-      uint4 buf[kBatch];
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int v = v0 + i * 32 + lane;
-        if (v < vec_per_row) buf[i] = src[v];
-      }
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int v = v0 + i * 32 + lane;
-        if (v < vec_per_row) dst[v] = buf[i];
-      }
-    }
+    const unsigned bit = 1u << (8 * (sid & 3));
+    if ((atomicOr(reinterpret_cast<unsigned*>(pair_flag) + (sid >> 2), bit) & bit) == 0) ++present;
+    inv[sid] = slot;
   }
-  if (lane == 0 && warp_present) atomicAdd(&cta_present, warp_present);
+  present = __reduce_add_sync(0xffffffffu, present);
+  if (lane == 0 && present) atomicAdd(&cta_present, present);
   __syncthreads();
   if (threadIdx.x == 0 && cta_present) atomicAdd(n_present, cta_present);
-  // scales: one lane per slot of a 32-slot group, so each store instruction
-  // writes 128 contiguous bytes of a row of s1s
   const int nwarps = gridDim.x * kGatherWarps;
   for (int s0 = (blockIdx.x * kGatherWarps + (threadIdx.x >> 5)) * 32; s0 < nv; s0 += nwarps * 32) {
     const int slot = s0 + lane;
@@ -83,7 +59,47 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
     if (sid < 0 || sid >= P) continue;
     const int t = sid / topk;
     for (int kb = 0; kb < KB; ++kb)
-      s1s[static_cast<size_t>(kb) * cap + slot] = __ldg(a1_scale + static_cast<size_t>(kb) * T + t);
+      __stcs(&s1s[static_cast<size_t>(kb) * cap + slot], __ldg(a1_scale + static_cast<size_t>(kb) * T + t));
+  }
+}
+
+// Token-ordered pass: each token's FP8 row of a8 [T, H] is read once and written
+// to the slot of each of its listed pairs (one warp per token). Going by token
+// rather than by slot keeps a8 from being re-read topk times from memory once
+// the slot-ordered writes have pushed it out of L2. Stores are marked
+// evict-first.
+__global__ void __launch_bounds__(32 * kGatherWarps)
+moe_gather_rows_kernel(const uint8_t* __restrict__ a8, int T, int topk, int H,
+                       const uint8_t* __restrict__ pair_flag, const int* __restrict__ inv,
+                       uint8_t* __restrict__ a8s) {
+  const int lane = threadIdx.x & 31;
+  const int vec_per_row = H / 16;
+  for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += gridDim.x * kGatherWarps) {
+    int slot_k = -1;
+    if (lane < topk) {
+      const int p = t * topk + lane;
+      if (pair_flag[p]) slot_k = inv[p];
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
+    constexpr int kBatch = 16;
+    for (int v0 = 0; v0 < vec_per_row; v0 += 32 * kBatch) {
+      uint4 buf[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < vec_per_row) buf[i] = __ldg(src + v);
+      }
+      for (int k = 0; k < topk; ++k) {
+        const int slot = __shfl_sync(0xffffffffu, slot_k, k);
+        if (slot < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          const int v = v0 + i * 32 + lane;
+          if (v < vec_per_row) __stcs(dst + v, buf[i]);
+        }
+      }
+    }
   }
 }
 
@@ -91,7 +107,8 @@ moe_gather_kernel(const uint8_t* __restrict__ a8, const float* __restrict__ a1_s
 // slot order k over the pairs whose flag is set (the routing weight is already
 // in y; a pair absent from the sorted list has no row). When every pair is
 // listed (*n_present, the count of distinct listed pairs, equals T*K: one cached
-// load) the flags are not read. One thread per 8 columns.
+// load) the flags are not read. One thread per 8 columns; the rows are read once,
+// with evict-first loads.
 __global__ void __launch_bounds__(256)
 moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, const uint8_t* __restrict__ pair_flag,
                    const int* __restrict__ n_present, int T, int K, int H, __nv_bfloat16* __restrict__ out) {
@@ -106,7 +123,7 @@ moe_combine_kernel(const __nv_bfloat16* __restrict__ ystage, const uint8_t* __re
   for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
   // fp32 sum in k order (0.0f + y0 == y0 exactly, so the order is fixed from the first term)
   auto add_row = [&](int k) {
-    const uint4 v = *reinterpret_cast<const uint4*>(y + static_cast<size_t>(k) * H);
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(y + static_cast<size_t>(k) * H));
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {

@@ -115,6 +115,7 @@ class MoELayer:
     @property
     def launches_per_forward(self):
         """Kernels one forward launches: route, sort (count and scatter; one kernel when the
-        T*topk pairs fit one 1024-pair chunk), quant, gather, gate/up GEMM, down GEMM, combine."""
+        T*topk pairs fit one 1024-pair chunk), quant, gather (slot pass and row pass), gate/up
+        GEMM, down GEMM, combine."""
         sort_kernels = 1 if self.max_tokens * self.cfg.K <= 1024 else 2
-        return 6 + sort_kernels
+        return 7 + sort_kernels

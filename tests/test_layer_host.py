@@ -45,6 +45,6 @@ def test_tp_shard_rejects_a_split_inside_a_128_block():
 
 
 def test_launches_per_forward_counts_the_sort_kernels():
-    assert MoELayer(I.TINY, "cpu").launches_per_forward == 7            # 64 pairs: one sort kernel
+    assert MoELayer(I.TINY, "cpu").launches_per_forward == 8            # 64 pairs: one sort kernel
     big = I.MoEConfig("host_big", T=200, H=256, E=16, G=4, TG=2, K=8, I=128)
-    assert MoELayer(big, "cpu").launches_per_forward == 8               # 1600 pairs: count + scatter
+    assert MoELayer(big, "cpu").launches_per_forward == 9               # 1600 pairs: count + scatter
