@@ -48,6 +48,10 @@ _SIGNATURES = {
     "fused_moe_fp8_blockscale_g1u1_noalloc": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int,
                                                        _c_int, _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int,
                                                        _p, _p]),
+    "fused_moe_fp8_blockscale_g1u1_tiled": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
+                                                     _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int, _p, _p,
+                                                     _c_size, _p]),
+    "fp8_tile_weights": (_c_int, [_p, _c_int, _c_int, _c_int, _p, _p]),
 }
 EXPORTED = tuple(_SIGNATURES)
 
@@ -251,6 +255,40 @@ def fp8_per_block_quant(w, block=128, q=None, scales=None):
     return q, scales
 
 
+def fp8_tile_weights(w, out=None):
+    """Re-pack fp8 expert matrices w [E, N, K] (or one matrix [N, K]) into the tiled layout
+    [E, N/128, K/128, 128, 128]: every 128 x 128 block 16 KB of consecutive bytes."""
+    _cuda(w, FP8, "w")
+    if not w.is_contiguous():
+        raise ValueError("w must be contiguous")
+    w3 = w if w.dim() == 3 else w.unsqueeze(0)
+    E, N, K = w3.shape
+    if N % 128 or K % 128:
+        raise ValueError(f"N and K must be multiples of 128 (N={N}, K={K})")
+    if out is None:
+        out = torch.empty(E, N // 128, K // 128, 128, 128, dtype=FP8, device=w.device)
+    _cuda(out, FP8, "out")
+    if out.numel() != w.numel() or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor with as many elements as w")
+    rc = load_library().fp8_tile_weights(_ptr(w), E, N, K, _ptr(out), _stream())
+    _check("fp8_tile_weights", rc)
+    return out
+
+
+def is_tiled(w) -> bool:
+    """True for expert weights in the tiled layout ([E, N/128, K/128, 128, 128])."""
+    return w.dim() == 5 and tuple(w.shape[3:]) == (128, 128)
+
+
+def _expert_matrix_shape(w):
+    """(E, N, K) of expert weights, row-major [E, N, K] or tiled [E, N/128, K/128, 128, 128]."""
+    if is_tiled(w):
+        return w.shape[0], w.shape[1] * 128, w.shape[2] * 128
+    if w.dim() != 3:
+        raise ValueError("expert weights must be [E, N, K] or tiled [E, N/128, K/128, 128, 128]")
+    return tuple(w.shape)
+
+
 def fp8_blockscale_gemm(A, B, a_scale, b_scale, out=None):
     """C bf16 [M, N] = block-scaled A fp8 [M, K] x B fp8 [N, K]^T."""
     _cuda(A, FP8, "A")
@@ -301,14 +339,16 @@ def _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, 
     _cuda(w2, FP8, "w2")
     for name, t in (("a1_scale", a1_scale), ("fc1_scale", fc1_scale), ("fc2_scale", fc2_scale)):
         _cuda(t, torch.float32, name)
-    if a8.dim() != 2 or w1.dim() != 3 or w2.dim() != 3:
-        raise ValueError("a8 must be [T, H], w1 [E, 2I, H] and w2 [E, H, I]")
+    if a8.dim() != 2:
+        raise ValueError("a8 must be [T, H]")
+    if is_tiled(w1) != is_tiled(w2):
+        raise ValueError("w1 and w2 must both be row-major or both tiled")
     T, H = a8.shape
-    E, twoI, H1 = w1.shape
-    I = w2.shape[2]
+    E, twoI, H1 = _expert_matrix_shape(w1)
+    E2, H2, I = _expert_matrix_shape(w2)
     if twoI != 2 * I:
-        raise ValueError("g1u1 requires w1.shape[1] == 2 * w2.shape[2]")
-    if H1 != H or tuple(w2.shape) != (E, H, I):
+        raise ValueError("g1u1 requires 2I rows of w1 for I columns of w2")
+    if H1 != H or (E2, H2) != (E, H):
         raise ValueError(f"w1 {tuple(w1.shape)} and w2 {tuple(w2.shape)} do not match a8's H={H}")
     if tuple(out.shape) != (T, H):
         raise ValueError(f"out must be [{T}, {H}], got {tuple(out.shape)}")
@@ -337,19 +377,22 @@ def _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, 
 
 def fused_moe_fp8_blockscale_g1u1(out, a8, w1, w2, sorted_pairs: SortedPairs, topk, a1_scale, fc1_scale, fc2_scale,
                                   scale_blk_n=128, scale_blk_k=128, fc2_smooth_scale=None, workspace=None):
-    """out bf16 [T, H] = fused g1u1 MoE (GEMM1 + SiLU*up + requant + GEMM2 + weighted combine)."""
+    """out bf16 [T, H] = fused g1u1 MoE (GEMM1 + SiLU*up + requant + GEMM2 + weighted combine).
+    w1, w2 row-major ([E, 2I, H], [E, H, I]) or both tiled (fp8_tile_weights): the tiled
+    ones take fused_moe_fp8_blockscale_g1u1_tiled."""
     T, H, I, E = _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale)
     sp = sorted_pairs
     lib = load_library()
     if workspace is None:
         need = fused_moe_workspace_bytes(T, topk, E, H, I, sp.block_m, capacity=sp.capacity)
         workspace = torch.empty(need, dtype=torch.uint8, device=a8.device)
-    rc = lib.fused_moe_fp8_blockscale_g1u1(
+    name = "fused_moe_fp8_blockscale_g1u1_tiled" if is_tiled(w1) else "fused_moe_fp8_blockscale_g1u1"
+    rc = getattr(lib, name)(
         _ptr(out), _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights),
         _ptr(sp.sorted_expert_ids), _ptr(sp.num_valid_ids), T, H, I, E, topk, sp.block_m, sp.capacity,
         _ptr(a1_scale), _ptr(fc1_scale), _ptr(fc2_scale), scale_blk_n, scale_blk_k, _ptr(fc2_smooth_scale),
         _ptr(workspace), workspace.numel(), _stream())
-    _check("fused_moe_fp8_blockscale_g1u1", rc)
+    _check(name, rc)
     return out
 
 
@@ -363,6 +406,8 @@ def fused_moe_fp8_blockscale_g1u1_noalloc(out, a8, w1, w2, sorted_pairs: SortedP
     fused_moe_fp8_blockscale_g1u1.
     """
     T, H, I, E = _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale)
+    if is_tiled(w1):
+        raise ValueError("the no-allocation entry point takes row-major weights")
     sp = sorted_pairs
     rc = load_library().fused_moe_fp8_blockscale_g1u1_noalloc(
         _ptr(out), _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights),

@@ -73,9 +73,9 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[kMaxDevices];
 
-template <int MODE>
+template <int MODE, bool TILED_B = false>
 cudaError_t enable_gemm_smem() {
-  return cudaFuncSetAttribute(blockscale_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(blockscale_gemm_kernel<MODE, TILED_B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(kGemmSmemBytes));
 }
 
@@ -99,6 +99,8 @@ int device_setup(int* sm_count) {
     if (r == cudaSuccess) r = enable_gemm_smem<kModeDense>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeUp>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown>();
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeUp, true>();
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, true>();
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sort_scatter_smem(kSortMaxExperts)));
@@ -155,6 +157,25 @@ int make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, con
 int make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
   return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, cols, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Map over weights in the tiled layout (fp8_tile_weights): 128 x 128-byte blocks,
+// each 16 KB of consecutive bytes, ordered (row block, K block). Viewed as a 3-D
+// tensor {128 bytes, 128 rows, block}; a box is one block; 128-byte swizzle.
+int make_tiled_weight_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8MOE_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[3] = {128, 128, (rows / 128) * (cols / 128)};
+  const cuuint64_t strides[2] = {128, 128 * 128};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FP8MOE_ECUDA, "cuTensorMapEncodeTiled failed (%d) for tiled weights [%llu x %llu]", static_cast<int>(r),
+                static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols));
+  return FP8MOE_OK;
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -478,13 +499,16 @@ size_t fused_moe_fp8_blockscale_g1u1_workspace(int T, int topk, int E, int H, in
   return moe_workspace_layout(moe_align_sort_capacity(T, topk, E, block_m), T, topk, H, I).total;
 }
 
-int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_t* w1, const uint8_t* w2,
-                                  const int32_t* sorted_ids, const float* sorted_weights,
-                                  const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H, int I,
-                                  int E, int topk, int block_m, size_t capacity, const float* a1_scale,
-                                  const float* fc1_scale, const float* fc2_scale, int scale_blk_n, int scale_blk_k,
-                                  const float* fc2_smooth_scale, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+}  // extern "C"
+
+// The fused MoE call on row-major (tiled == false) or tiled (fp8_tile_weights) weights.
+static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uint8_t* a8, const uint8_t* w1,
+                          const uint8_t* w2, const int32_t* sorted_ids, const float* sorted_weights,
+                          const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H, int I, int E,
+                          int topk, int block_m, size_t capacity, const float* a1_scale, const float* fc1_scale,
+                          const float* fc2_scale, int scale_blk_n, int scale_blk_k, const float* fc2_smooth_scale,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  (void)name;
   if (scale_blk_n != 128 || scale_blk_k != 128)
     return fail(FP8MOE_EUNSUPPORTED, "only (128, 128) scale blocks are supported (got %d, %d)", scale_blk_n,
                 scale_blk_k);
@@ -522,9 +546,14 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
 
   CUtensorMap m_a8s, m_w1, m_a2, m_w2;
   if (int rc = make_operand_map(&m_a8s, a8s, capacity, H)) return rc;
-  if (int rc = make_operand_map(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H)) return rc;
   if (int rc = make_operand_map(&m_a2, a2, capacity, I)) return rc;
-  if (int rc = make_operand_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
+  if (tiled) {
+    if (int rc = make_tiled_weight_map(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H)) return rc;
+    if (int rc = make_tiled_weight_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
+  } else {
+    if (int rc = make_operand_map(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H)) return rc;
+    if (int rc = make_operand_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
+  }
 
   // pairs absent from the sorted list (a masked-out expert, a dropped id) keep
   // flag 0 and add nothing in the combine
@@ -563,7 +592,10 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   up.a2 = a2;
   up.s2 = s2;
   up.ystage = ystage;
-  blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, up);
+  if (tiled)
+    blockscale_gemm_kernel<kModeMoeUp, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, up);
+  else
+    blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, up);
   if (int rc = check_gemm_launch("fused_moe (gate/up GEMM)", blockscale_gemm_kernel<kModeMoeUp>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
@@ -580,7 +612,10 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   dn.nb_valid = H / 128;
   dn.b_rows_per_expert = H;
   dn.s2 = nullptr;
-  blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
+  if (tiled)
+    blockscale_gemm_kernel<kModeMoeDown, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
+  else
+    blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
   if (int rc = check_gemm_launch("fused_moe (down GEMM)", blockscale_gemm_kernel<kModeMoeDown>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
@@ -592,6 +627,50 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
   if (int rc = check_launch("fused_moe (combine)")) return rc;
   timing_record(4, st);
   return FP8MOE_OK;
+}
+
+extern "C" {
+
+int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_t* w1, const uint8_t* w2,
+                                  const int32_t* sorted_ids, const float* sorted_weights,
+                                  const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H, int I,
+                                  int E, int topk, int block_m, size_t capacity, const float* a1_scale,
+                                  const float* fc1_scale, const float* fc2_scale, int scale_blk_n, int scale_blk_k,
+                                  const float* fc2_smooth_scale, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1", false, out, a8, w1, w2, sorted_ids, sorted_weights,
+                        sorted_expert_ids, num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
+                        fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, workspace, workspace_bytes, stream);
+}
+
+int fused_moe_fp8_blockscale_g1u1_tiled(uint16_t* out, const uint8_t* a8, const uint8_t* w1, const uint8_t* w2,
+                                        const int32_t* sorted_ids, const float* sorted_weights,
+                                        const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H,
+                                        int I, int E, int topk, int block_m, size_t capacity, const float* a1_scale,
+                                        const float* fc1_scale, const float* fc2_scale, int scale_blk_n,
+                                        int scale_blk_k, const float* fc2_smooth_scale, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1_tiled", true, out, a8, w1, w2, sorted_ids, sorted_weights,
+                        sorted_expert_ids, num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
+                        fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------------------------ weight re-pack
+int fp8_tile_weights(const uint8_t* w, int E, int N, int K, uint8_t* out, void* stream) {
+  if (E < 1 || E > 65535) return fail(FP8MOE_EINVAL, "E must be in [1, 65535] (got %d)", E);
+  if (N < 128 || K < 128 || N % 128 || K % 128)
+    return fail(FP8MOE_EUNSUPPORTED, "N and K must be positive multiples of 128 (N=%d, K=%d)", N, K);
+  if (N / 128 > 65535 || K / 128 > 65535) return fail(FP8MOE_EUNSUPPORTED, "N or K too large");
+  if (!w || !out) return fail(FP8MOE_EINVAL, "null pointer argument");
+  if (!aligned16(w) || !aligned16(out)) return fail(FP8MOE_EINVAL, "w and out must be 16-byte aligned");
+  const size_t bytes = static_cast<size_t>(E) * N * K;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(w), b = reinterpret_cast<uintptr_t>(out);
+  if (a < b + bytes && b < a + bytes) return fail(FP8MOE_EINVAL, "w and out overlap");
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const dim3 grid(K / 128, N / 128, E);
+  tile_weights_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(w, N, K, out);
+  return check_launch("fp8_tile_weights");
 }
 
 // ------------------------------------------------------------------ no-allocation variant

@@ -32,6 +32,10 @@
 // In the MoE modes the rows are the sorted token-expert slots: A is the
 // slot-ordered activation matrix (gathered by moe_gather_kernel for GEMM1, the
 // re-quantised intermediate for GEMM2), one expert per 128-row block.
+// The MoE GEMMs read the weights either row-major ([E * rows, K]: a box is 128 rows
+// x 128 bytes, the rows a full K apart) or tiled (each 128 x 128 block stored as 16
+// KB of consecutive bytes, blocks ordered (row block, K block): a box is one block,
+// read through a 3-D tensor map), chosen by the template flag TILED_B.
 // All waits are bounded; on expiry the CTA flags FP8MOE_DEVERR_TIMEOUT, sets a
 // shared abort flag so the other roles stop, frees TMEM and exits.
 #pragma once
@@ -432,7 +436,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
   if (!ok) abort_all(s);
 }
 
-template <int MODE>
+template <int MODE, bool TILED_B = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const GemmArgs args) {
@@ -506,8 +510,14 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             uint8_t* sb_tile = tiles_b + stage * kStageB;
             mbar_arrive_expect_tx(&s->full[stage], kStageA + kStageB);
             tma_load_2d(sa_tile, &tmA, &s->full[stage], kb * kBK, mb * kBM);
-            tma_load_2d(sb_tile, &tmB, &s->full[stage], kb * kBK, brow0);
-            tma_load_2d(sb_tile + kStageB / 2, &tmB, &s->full[stage], kb * kBK, brow1);
+            if constexpr (TILED_B) {
+              // block (row block r, K block kb) is box (0, 0, r * num_kb + kb)
+              tma_load_3d(sb_tile, &tmB, &s->full[stage], 0, 0, (brow0 / 128) * num_kb + kb);
+              tma_load_3d(sb_tile + kStageB / 2, &tmB, &s->full[stage], 0, 0, (brow1 / 128) * num_kb + kb);
+            } else {
+              tma_load_2d(sb_tile, &tmB, &s->full[stage], kb * kBK, brow0);
+              tma_load_2d(sb_tile + kStageB / 2, &tmB, &s->full[stage], kb * kBK, brow1);
+            }
           }
           __syncwarp();
           if (++stage == kStages) { stage = 0; sphase ^= 1u; }

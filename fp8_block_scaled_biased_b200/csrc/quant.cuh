@@ -127,4 +127,23 @@ quant_128x128_kernel(const float* __restrict__ w, int ld_w, int N, int K, uint8_
   }
 }
 
+// Weight re-pack into the tiled layout the MoE GEMMs can read with one contiguous
+// 16 KB box per 128 x 128 block: w [E, N, K] row-major -> out [E, N/128, K/128,
+// 128, 128] (block (e, nb, kb) holds rows nb*128.. and columns kb*128.. of expert
+// e's matrix, row-major inside the block). One CTA per block, 16-byte copies.
+__global__ void __launch_bounds__(256)
+tile_weights_kernel(const uint8_t* __restrict__ w, int N, int K, uint8_t* __restrict__ out) {
+  const int kb = blockIdx.x, nb = blockIdx.y, e = blockIdx.z;
+  const int NB = gridDim.y, KB = gridDim.x;
+  const uint8_t* src = w + (static_cast<size_t>(e) * N + static_cast<size_t>(nb) * 128) * K + static_cast<size_t>(kb) * 128;
+  uint8_t* dst = out + ((static_cast<size_t>(e) * NB + nb) * KB + kb) * (128 * 128);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = i * 256 + threadIdx.x;   // 16-byte piece: row idx / 8, column piece idx % 8
+    const int r = idx >> 3, c = (idx & 7) * 16;
+    *reinterpret_cast<uint4*>(dst + r * 128 + c) =
+        __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(r) * K + c));
+  }
+}
+
 }  // namespace fp8moe

@@ -185,15 +185,20 @@ def ep_combine(partials: torch.Tensor, plan: EpPlan, group=None) -> torch.Tensor
 
 
 class ExpertShard:
-    """The experts [e0, e1) of a layer, as one expert-parallel rank holds them: w1
-    [n_e, 2I, H], w2 [n_e, H, I] and their 128x128 block scales, on the device."""
+    """The experts [e0, e1) of a layer, as one expert-parallel rank holds them: w1 and w2
+    (tiled as fp8_tile_weights writes them, or row-major [n_e, 2I, H], [n_e, H, I]) and
+    their 128x128 block scales, on the device."""
 
-    def __init__(self, cfg: I.MoEConfig, e0: int, e1: int, device="cuda"):
-        self.cfg, self.e0, self.e1 = cfg, e0, e1
+    def __init__(self, cfg: I.MoEConfig, e0: int, e1: int, device="cuda", tiled: bool = True):
+        self.cfg, self.e0, self.e1, self.tiled = cfg, e0, e1, tiled
         ne, H, Im = e1 - e0, cfg.H, cfg.I
-        self.w1 = torch.empty(ne, 2 * Im, H, dtype=B.FP8, device=device)
+        if tiled:
+            self.w1 = torch.empty(ne, 2 * Im // 128, H // 128, 128, 128, dtype=B.FP8, device=device)
+            self.w2 = torch.empty(ne, H // 128, Im // 128, 128, 128, dtype=B.FP8, device=device)
+        else:
+            self.w1 = torch.empty(ne, 2 * Im, H, dtype=B.FP8, device=device)
+            self.w2 = torch.empty(ne, H, Im, dtype=B.FP8, device=device)
         self.w1_scale = torch.empty(ne, 2 * Im // 128, H // 128, dtype=torch.float32, device=device)
-        self.w2 = torch.empty(ne, H, Im, dtype=B.FP8, device=device)
         self.w2_scale = torch.empty(ne, H // 128, Im // 128, dtype=torch.float32, device=device)
         self.block_m = B.moe_block_m()
         # sort over the rank's experts plus one sentinel expert (other ranks' pairs), masked out
@@ -202,11 +207,18 @@ class ExpertShard:
 
     def load_synthetic_weights(self):
         """Draw and quantise the raw weights of global experts e0..e1-1 (as MoELayer does)."""
+        dev = self.w1.device
+        cfg = self.cfg
+        stage1 = torch.empty(2 * cfg.I, cfg.H, dtype=B.FP8, device=dev) if self.tiled else None
+        stage2 = torch.empty(cfg.H, cfg.I, dtype=B.FP8, device=dev) if self.tiled else None
         for i, e in enumerate(range(self.e0, self.e1)):
-            B.fp8_per_block_quant(I.expert_weight_raw(self.cfg, "w1", e, self.w1.device), q=self.w1[i],
+            B.fp8_per_block_quant(I.expert_weight_raw(cfg, "w1", e, dev), q=stage1 if self.tiled else self.w1[i],
                                   scales=self.w1_scale[i])
-            B.fp8_per_block_quant(I.expert_weight_raw(self.cfg, "w2", e, self.w2.device), q=self.w2[i],
+            B.fp8_per_block_quant(I.expert_weight_raw(cfg, "w2", e, dev), q=stage2 if self.tiled else self.w2[i],
                                   scales=self.w2_scale[i])
+            if self.tiled:
+                B.fp8_tile_weights(stage1, out=self.w1[i])
+                B.fp8_tile_weights(stage2, out=self.w2[i])
         return self
 
     def __call__(self, a8, scales, ids, weights):

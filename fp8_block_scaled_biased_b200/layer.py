@@ -18,8 +18,13 @@ from . import inputs as I
 
 
 class MoELayer:
-    def __init__(self, cfg: I.MoEConfig, device="cuda", max_tokens: int | None = None, weights_from=None):
-        """weights_from: another MoELayer of the same layer shape whose device weights are shared."""
+    def __init__(self, cfg: I.MoEConfig, device="cuda", max_tokens: int | None = None, weights_from=None,
+                 tiled: bool = True):
+        """weights_from: another MoELayer of the same layer shape whose device weights (and
+        layout) are shared. tiled: keep w1 and w2 in the tiled layout of fp8_tile_weights
+        ([E, N/128, K/128, 128, 128], every 128 x 128 block 16 KB of consecutive bytes), which
+        the GEMMs read with one contiguous load per block; False keeps them row-major
+        ([E, 2I, H], [E, H, I]), the layout the pages' fused call takes."""
         self.cfg = cfg
         self.device = torch.device(device)
         self.max_tokens = max_tokens or cfg.T
@@ -29,11 +34,17 @@ class MoELayer:
             o = weights_from
             if (o.cfg.E, o.cfg.H, o.cfg.I) != (E, H, Im):
                 raise ValueError("weights_from has a different layer shape")
+            self.tiled = o.tiled
             self.w1, self.w1_scale, self.w2, self.w2_scale = o.w1, o.w1_scale, o.w2, o.w2_scale
         else:
-            self.w1 = torch.empty(E, 2 * Im, H, dtype=B.FP8, device=dev)
+            self.tiled = tiled
+            if tiled:
+                self.w1 = torch.empty(E, 2 * Im // 128, H // 128, 128, 128, dtype=B.FP8, device=dev)
+                self.w2 = torch.empty(E, H // 128, Im // 128, 128, 128, dtype=B.FP8, device=dev)
+            else:
+                self.w1 = torch.empty(E, 2 * Im, H, dtype=B.FP8, device=dev)
+                self.w2 = torch.empty(E, H, Im, dtype=B.FP8, device=dev)
             self.w1_scale = torch.empty(E, 2 * Im // 128, H // 128, dtype=torch.float32, device=dev)
-            self.w2 = torch.empty(E, H, Im, dtype=B.FP8, device=dev)
             self.w2_scale = torch.empty(E, H // 128, Im // 128, dtype=torch.float32, device=dev)
         self.block_m = B.moe_block_m()
         self._alloc(self.max_tokens)
@@ -56,13 +67,24 @@ class MoELayer:
         ws = B.fused_moe_workspace_bytes(T, cfg.K, cfg.E, cfg.H, cfg.I, self.block_m)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
 
-    def load_synthetic_weights(self):
-        """Draw each expert's raw fp32 weights on the device and quantise them in 128x128 blocks."""
-        for e in range(self.cfg.E):
-            raw1 = I.expert_weight_raw(self.cfg, "w1", e, self.device)
-            B.fp8_per_block_quant(raw1, q=self.w1[e], scales=self.w1_scale[e])
-            raw2 = I.expert_weight_raw(self.cfg, "w2", e, self.device)
-            B.fp8_per_block_quant(raw2, q=self.w2[e], scales=self.w2_scale[e])
+    def load_synthetic_weights(self, expert_offset: int = 0):
+        """Draw each expert's raw fp32 weights on the device, quantise them in 128x128 blocks
+        and, for a tiled layer, re-pack them (fp8_tile_weights). Slot i holds global expert
+        expert_offset + i (an expert-parallel rank's experts start past 0)."""
+        cfg = self.cfg
+        stage1 = stage2 = None
+        if self.tiled:
+            stage1 = torch.empty(2 * cfg.I, cfg.H, dtype=B.FP8, device=self.device)
+            stage2 = torch.empty(cfg.H, cfg.I, dtype=B.FP8, device=self.device)
+        for i in range(self.w1.shape[0]):
+            e = expert_offset + i
+            raw1 = I.expert_weight_raw(cfg, "w1", e, self.device)
+            B.fp8_per_block_quant(raw1, q=stage1 if self.tiled else self.w1[i], scales=self.w1_scale[i])
+            raw2 = I.expert_weight_raw(cfg, "w2", e, self.device)
+            B.fp8_per_block_quant(raw2, q=stage2 if self.tiled else self.w2[i], scales=self.w2_scale[i])
+            if self.tiled:
+                B.fp8_tile_weights(stage1, out=self.w1[i])
+                B.fp8_tile_weights(stage2, out=self.w2[i])
         return self
 
     def tp_shard(self, rank: int, nranks: int) -> "MoELayer":
@@ -78,13 +100,18 @@ class MoELayer:
             raise ValueError(f"I={cfg.I} cannot be split into {nranks} shards of whole 128-column blocks")
         Is, I0 = cfg.I // nranks, rank * (cfg.I // nranks)
         nb, b0, nbI = Is // 128, I0 // 128, cfg.I // 128
-        scfg = dataclasses.replace(cfg, name=f"{cfg.name}_tp{nranks}_rank{rank}", I=Is)
-        shard = MoELayer(scfg, self.device, max_tokens=self.max_tokens)
-        shard.w1[:, :Is].copy_(self.w1[:, I0:I0 + Is])
-        shard.w1[:, Is:].copy_(self.w1[:, cfg.I + I0:cfg.I + I0 + Is])
+        scfg = dataclasses.replace(cfg, name=f"{cfg.name}_tp{nranks}_rank{rank}", I=Is, tp_ranks=nranks, tp_rank=rank)
+        shard = MoELayer(scfg, self.device, max_tokens=self.max_tokens, tiled=self.tiled)
+        if self.tiled:                   # whole 128-blocks: gate/up row blocks of w1, K blocks of w2
+            shard.w1[:, :nb].copy_(self.w1[:, b0:b0 + nb])
+            shard.w1[:, nb:].copy_(self.w1[:, nbI + b0:nbI + b0 + nb])
+            shard.w2.copy_(self.w2[:, :, b0:b0 + nb])
+        else:
+            shard.w1[:, :Is].copy_(self.w1[:, I0:I0 + Is])
+            shard.w1[:, Is:].copy_(self.w1[:, cfg.I + I0:cfg.I + I0 + Is])
+            shard.w2.copy_(self.w2[:, :, I0:I0 + Is])
         shard.w1_scale[:, :nb].copy_(self.w1_scale[:, b0:b0 + nb])
         shard.w1_scale[:, nb:].copy_(self.w1_scale[:, nbI + b0:nbI + b0 + nb])
-        shard.w2.copy_(self.w2[:, :, I0:I0 + Is])
         shard.w2_scale.copy_(self.w2_scale[:, :, b0:b0 + nb])
         return shard
 

@@ -209,6 +209,24 @@ int fp8_per_block_quant(const float* w, int ld_w, int N, int K, int block,
                         uint8_t* q, float* scales, void* stream);
 
 /*
+ * Weight preparation - re-pack into the tiled layout. (The B200 counterpart of the
+ * pages' offline weight pre-shuffle: the MoE section passes w1 and w2 through
+ * shuffle_weight(w, (16, 16)) before asm_moe, and the linear section notes a
+ * shuffled-weight variant, both in "Blockscale FP8 MoE Computation" and "General
+ * Linear Layer". The pages print that layout only for AMD's kernels; this one is
+ * this library's own.)
+ *
+ * w    fp8 [E, N, K] row-major (E expert matrices), 16-byte aligned
+ * out  fp8 [E, N/128, K/128, 128, 128]: block (e, nb, kb) holds rows
+ *      nb*128 .. nb*128+127 and columns kb*128 .. kb*128+127 of matrix e,
+ *      row-major inside the block, so each 128 x 128 block is 16 KB of
+ *      consecutive bytes (16-byte aligned, not overlapping w). The block scales
+ *      are unchanged ([E, N/128, K/128] in either layout).
+ * Limits: N and K positive multiples of 128, E <= 65535.
+ */
+int fp8_tile_weights(const uint8_t* w, int E, int N, int K, uint8_t* out, void* stream);
+
+/*
  * S0 - FP8 block-scale GEMM.  (General Linear Layer:
  *      gemm_a8w8_blockscale(XQ, WQ, x_scale, w_scale, dtype) -> Y.)
  *
@@ -280,6 +298,27 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8,
                                   int scale_blk_k, const float* fc2_smooth_scale,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream);
+
+/*
+ * S4-S7 on tiled weights: fused_moe_fp8_blockscale_g1u1 with w1 and w2 in the
+ * layout fp8_tile_weights writes (w1 tiled as [E, 2I/128, H/128, 128, 128], w2 as
+ * [E, H/128, I/128, 128, 128]); every other argument, the workspace and the result
+ * (bit for bit) as fused_moe_fp8_blockscale_g1u1. Each 128 x 128 weight block is
+ * then one contiguous 16 KB read instead of 128 reads of 128 bytes a row apart.
+ */
+int fused_moe_fp8_blockscale_g1u1_tiled(uint16_t* out, const uint8_t* a8,
+                                        const uint8_t* w1, const uint8_t* w2,
+                                        const int32_t* sorted_ids,
+                                        const float* sorted_weights,
+                                        const int32_t* sorted_expert_ids,
+                                        const int32_t* num_valid_ids,
+                                        int T, int H, int I, int E, int topk,
+                                        int block_m, size_t capacity,
+                                        const float* a1_scale, const float* fc1_scale,
+                                        const float* fc2_scale, int scale_blk_n,
+                                        int scale_blk_k, const float* fc2_smooth_scale,
+                                        void* workspace, size_t workspace_bytes,
+                                        void* stream);
 
 /*
  * Fused g1u1 MoE without any device allocation by the caller.

@@ -270,6 +270,32 @@ def test_fused_moe_full_small_layers(cfg):
     assert torch.equal(out, out2)                      # deterministic combine
 
 
+@pytest.mark.parametrize("E,N,K", [(1, 128, 128), (3, 384, 256), (2, 4096, 7168), (2, 7168, 2048)])
+def test_tile_weights_layout(E, N, K):
+    """fp8_tile_weights against the tiled layout's definition: block (e, nb, kb) holds rows
+    nb*128.. and columns kb*128.. of matrix e, row-major inside the block."""
+    g = torch.Generator().manual_seed(E * N + K)
+    w = torch.randint(0, 256, (E, N, K), generator=g, dtype=torch.uint8)
+    t = B.fp8_tile_weights(w.to(DEV).view(B.FP8))
+    ref = w.view(E, N // 128, 128, K // 128, 128).permute(0, 1, 3, 2, 4).contiguous()
+    assert torch.equal(t.view(torch.uint8).cpu(), ref)
+    with pytest.raises(ValueError):
+        B.fp8_tile_weights(torch.empty(1, 200, 128, dtype=B.FP8, device=DEV))
+
+
+@pytest.mark.parametrize("cfg", [MID, SKEW_SMALL, ODD_ONE, ODD_E24, FEW_EXPERTS], ids=lambda c: c.name)
+def test_fused_moe_tiled_weights_equal_row_major_bit_for_bit(cfg):
+    """The fused call on tiled weights computes exactly what it computes on row-major ones:
+    only the order in which the weight bytes sit in memory differs."""
+    act = I.moe_activations(cfg)
+    args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    rm = MoELayer(cfg, DEV, tiled=False).load_synthetic_weights()
+    tl = MoELayer(cfg, DEV, tiled=True).load_synthetic_weights()
+    assert tl.tiled and tl.w1.dim() == 5
+    out_rm = rm.forward(*args).clone()
+    assert torch.equal(tl.forward(*args), out_rm)
+
+
 @pytest.fixture(scope="module")
 def big_layer():
     layer = MoELayer(I.DECODE, DEV).load_synthetic_weights()

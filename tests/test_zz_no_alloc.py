@@ -34,7 +34,7 @@ MULTI_BLOCK = I.MoEConfig("noalloc_t1024_h1024_e8", T=1024, H=1024, E=8, G=2, TG
 
 @pytest.mark.parametrize("cfg", [ONE_BLOCK, MULTI_BLOCK], ids=lambda c: c.name)
 def test_noalloc_equals_workspace_entry_point_on_two_calls(cfg):
-    layer = MoELayer(cfg, "cuda").load_synthetic_weights()
+    layer = MoELayer(cfg, "cuda", tiled=False).load_synthetic_weights()       # the call takes row-major weights
     act = I.moe_activations(cfg)
     ref = layer.forward(act.logits.cuda(), act.bias.cuda(), act.x.cuda()).clone()
     need = B.load_library().fused_moe_fp8_blockscale_g1u1_workspace(cfg.T, cfg.K, cfg.E, cfg.H, cfg.I,
@@ -73,7 +73,7 @@ def test_noalloc_binding_refuses_mismatched_or_strided_weights():
     """The binding checks the no-allocation call's tensors as it checks the workspace call's:
     the library sizes its tensor maps from these shapes, so a mismatch must never reach it."""
     cfg = ONE_BLOCK
-    layer = MoELayer(cfg, "cuda")
+    layer = MoELayer(cfg, "cuda", tiled=False)
     act = I.moe_activations(cfg)
     a8, a1 = B.fp8_per_token_group_quant(act.x.cuda(), 128, column_major_scales=True)
     sp = B.alloc_sorted(cfg.T, cfg.K, cfg.E, layer.block_m, "cuda")
