@@ -64,40 +64,44 @@ moe_gather_kernel(const float* __restrict__ a1_scale, const int32_t* __restrict_
 }
 
 // Token-ordered pass: each token's FP8 row of a8 [T, H] is read once and written
-// to the slot of each of its listed pairs (one warp per token). Going by token
-// rather than by slot keeps a8 from being re-read topk times from memory once
-// the slot-ordered writes have pushed it out of L2. Stores are marked
+// to the slot of each of its listed pairs. Going by token rather than by slot
+// keeps a8 from being re-read topk times from memory once the slot-ordered
+// writes have pushed it out of L2. A warp takes one 2 KB chunk of one token's row
+// (so that a small batch still spreads over the GPU); stores are marked
 // evict-first.
+constexpr int kRowChunkVec = 4;               // 16-byte vectors per lane per chunk
 __global__ void __launch_bounds__(32 * kGatherWarps)
 moe_gather_rows_kernel(const uint8_t* __restrict__ a8, int T, int topk, int H,
                        const uint8_t* __restrict__ pair_flag, const int* __restrict__ inv,
                        uint8_t* __restrict__ a8s) {
   const int lane = threadIdx.x & 31;
   const int vec_per_row = H / 16;
-  for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += gridDim.x * kGatherWarps) {
+  const int chunks = (vec_per_row + 32 * kRowChunkVec - 1) / (32 * kRowChunkVec);
+  const long long units = static_cast<long long>(T) * chunks;
+  for (long long u = static_cast<long long>(blockIdx.x) * kGatherWarps + (threadIdx.x >> 5); u < units;
+       u += static_cast<long long>(gridDim.x) * kGatherWarps) {
+    const int t = static_cast<int>(u / chunks);
+    const int v0 = static_cast<int>(u % chunks) * 32 * kRowChunkVec;
     int slot_k = -1;
     if (lane < topk) {
       const int p = t * topk + lane;
       if (pair_flag[p]) slot_k = inv[p];
     }
     const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
-    constexpr int kBatch = 16;
-    for (int v0 = 0; v0 < vec_per_row; v0 += 32 * kBatch) {
-      uint4 buf[kBatch];
+    uint4 buf[kRowChunkVec];
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
+    for (int i = 0; i < kRowChunkVec; ++i) {
+      const int v = v0 + i * 32 + lane;
+      if (v < vec_per_row) buf[i] = __ldg(src + v);
+    }
+    for (int k = 0; k < topk; ++k) {
+      const int slot = __shfl_sync(0xffffffffu, slot_k, k);
+      if (slot < 0) continue;
+      uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
+#pragma unroll
+      for (int i = 0; i < kRowChunkVec; ++i) {
         const int v = v0 + i * 32 + lane;
-        if (v < vec_per_row) buf[i] = __ldg(src + v);
-      }
-      for (int k = 0; k < topk; ++k) {
-        const int slot = __shfl_sync(0xffffffffu, slot_k, k);
-        if (slot < 0) continue;
-        uint4* dst = reinterpret_cast<uint4*>(a8s + static_cast<size_t>(slot) * H);
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const int v = v0 + i * 32 + lane;
-          if (v < vec_per_row) __stcs(dst + v, buf[i]);
-        }
+        if (v < vec_per_row) __stcs(dst + v, buf[i]);
       }
     }
   }
