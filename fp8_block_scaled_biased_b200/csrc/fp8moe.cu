@@ -178,6 +178,12 @@ int make_tiled_weight_map(CUtensorMap* map, const void* base, uint64_t rows, uin
   return FP8MOE_OK;
 }
 
+// The same with a 64-row box (the first half of an M=64 tile's A rows).
+int make_operand_map_64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, cols, 128, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Scratch of the fused MoE call: the slot-ordered FP8 activations and their
@@ -477,7 +483,7 @@ static int blockscale_gemm_impl(const char* name, const uint8_t* A, const uint8_
   const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * a.n_tiles;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   blockscale_gemm_kernel<kModeDense><<<grid, kGemmThreads, kGemmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      ma, mb, a);
+      ma, mb, ma, a);
   return check_gemm_launch(name, blockscale_gemm_kernel<kModeDense>, kGemmThreads, kGemmSmemBytes);
 }
 
@@ -547,6 +553,9 @@ static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uin
   CUtensorMap m_a8s, m_w1, m_a2, m_w2;
   if (int rc = make_operand_map(&m_a8s, a8s, capacity, H)) return rc;
   if (int rc = make_operand_map(&m_a2, a2, capacity, I)) return rc;
+  CUtensorMap m_a8s64, m_a264;
+  if (int rc = make_operand_map_64(&m_a8s64, a8s, capacity, H)) return rc;
+  if (int rc = make_operand_map_64(&m_a264, a2, capacity, I)) return rc;
   if (tiled) {
     if (int rc = make_tiled_weight_map(&m_w1, w1, static_cast<uint64_t>(E) * 2 * I, H)) return rc;
     if (int rc = make_tiled_weight_map(&m_w2, w2, static_cast<uint64_t>(E) * H, I)) return rc;
@@ -593,9 +602,9 @@ static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uin
   up.s2 = s2;
   up.ystage = ystage;
   if (tiled)
-    blockscale_gemm_kernel<kModeMoeUp, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, up);
+    blockscale_gemm_kernel<kModeMoeUp, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, m_a8s64, up);
   else
-    blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, up);
+    blockscale_gemm_kernel<kModeMoeUp><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a8s, m_w1, m_a8s64, up);
   if (int rc = check_gemm_launch("fused_moe (gate/up GEMM)", blockscale_gemm_kernel<kModeMoeUp>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;
@@ -613,9 +622,9 @@ static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uin
   dn.b_rows_per_expert = H;
   dn.s2 = nullptr;
   if (tiled)
-    blockscale_gemm_kernel<kModeMoeDown, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
+    blockscale_gemm_kernel<kModeMoeDown, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, m_a264, dn);
   else
-    blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, dn);
+    blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, m_a264, dn);
   if (int rc = check_gemm_launch("fused_moe (down GEMM)", blockscale_gemm_kernel<kModeMoeDown>, kGemmThreads,
                                  kGemmSmemBytes))
     return rc;

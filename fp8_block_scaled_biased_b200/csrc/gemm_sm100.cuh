@@ -36,6 +36,8 @@
 // x 128 bytes, the rows a full K apart) or tiled (each 128 x 128 block stored as 16
 // KB of consecutive bytes, blocks ordered (row block, K block): a box is one block,
 // read through a 3-D tensor map), chosen by the template flag TILED_B.
+// A MoE tile that runs M=64 MMAs (its second 64 slots are padding) loads only its
+// first 64 A rows (tmA64, a 64-row box), which spares shared-memory and L2 traffic.
 // All waits are bounded; on expiry the CTA flags FP8MOE_DEVERR_TIMEOUT, sets a
 // shared abort flag so the other roles stop, frees TMEM and exits.
 #pragma once
@@ -439,7 +441,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
 template <int MODE, bool TILED_B = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const GemmArgs args) {
+                       const __grid_constant__ CUtensorMap tmA64, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* tiles = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -470,6 +472,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     s->abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
+    if (MODE != kModeDense) prefetch_tensormap(&tmA64);
     prefetch_tensormap(&tmB);
   }
   if (warp == 1) {
@@ -500,6 +503,13 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         int mb, nt;
         tile_coords<MODE>(args, tile, m_blocks, mb, nt);
         const int e = (MODE == kModeDense) ? 0 : moe_expert(args, mb);
+        // a MoE tile whose slot kBM/2 is padding runs M=64 MMAs: load its first 64 A rows only
+        bool a64 = false;
+        if (MODE != kModeDense) {
+          const int id_half = args.sorted_ids[mb * kBM + kBM / 2];
+          a64 = id_half < 0 || id_half >= P;
+        }
+        const uint32_t a_bytes = a64 ? kStageA / 2 : kStageA;
         const int brow0 = (MODE == kModeMoeUp) ? e * args.b_rows_per_expert + nt * 128
                                                : e * args.b_rows_per_expert + nt * kBN;
         const int brow1 = (MODE == kModeMoeUp) ? brow0 + args.N : brow0 + 128;
@@ -508,8 +518,8 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           if (lane == 0) {
             uint8_t* sa_tile = tiles_a + stage * kStageA;
             uint8_t* sb_tile = tiles_b + stage * kStageB;
-            mbar_arrive_expect_tx(&s->full[stage], kStageA + kStageB);
-            tma_load_2d(sa_tile, &tmA, &s->full[stage], kb * kBK, mb * kBM);
+            mbar_arrive_expect_tx(&s->full[stage], a_bytes + kStageB);
+            tma_load_2d(sa_tile, a64 ? &tmA64 : &tmA, &s->full[stage], kb * kBK, mb * kBM);
             if constexpr (TILED_B) {
               // block (row block r, K block kb) is box (0, 0, r * num_kb + kb)
               tma_load_3d(sb_tile, &tmB, &s->full[stage], 0, 0, (brow0 / 128) * num_kb + kb);
