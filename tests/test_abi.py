@@ -160,3 +160,24 @@ def test_workspace_bytes_cover_a_sorted_list_over_more_experts(lib):
     assert B.fused_moe_workspace_bytes(T, K, E, H, I, bm, capacity=cap) == \
         lib.fused_moe_fp8_blockscale_g1u1_workspace(T, K, E + 1, H, I, bm)
     assert B.fused_moe_workspace_bytes(T, K, E, H, I, bm) < B.fused_moe_workspace_bytes(T, K, E, H, I, bm, capacity=cap)
+
+
+def test_tile_weights_and_tiled_fused_call_reject_bad_arguments(lib):
+    rc, msg = _rc(lib, "fp8_tile_weights", P, 2, 200, 128, ctypes.c_void_p(1 << 20), None)
+    assert rc == 2 and "multiples of 128" in msg                       # N not a multiple of 128
+    rc, _ = _rc(lib, "fp8_tile_weights", P, 0, 128, 128, ctypes.c_void_p(1 << 20), None)
+    assert rc == 1                                                     # no experts
+    rc, msg = _rc(lib, "fp8_tile_weights", P, 1, 128, 128, P, None)
+    assert rc == 1 and "overlap" in msg                                # in place is refused
+    rc, _ = _rc(lib, "fp8_tile_weights", ctypes.c_void_p(24), 1, 128, 128, ctypes.c_void_p(1 << 20), None)
+    assert rc == 1                                                     # w not 16-byte aligned
+    T, K, E, H, I = 16, 4, 16, 256, 128
+    cap = lib.moe_align_sort_capacity(T, K, E, 128)
+    ws = lib.fused_moe_fp8_blockscale_g1u1_workspace(T, K, E, H, I, 128)
+    args = [P] * 8 + [T, H, I, E, K, 128, cap, P, P, P, 128, 128, None, ctypes.c_void_p(256), ws, None]
+    a = list(args)
+    a[18] = 64                                                         # scale_blk_n
+    assert _rc(lib, "fused_moe_fp8_blockscale_g1u1_tiled", *a)[0] == 2
+    a = list(args)
+    a[22] = ws - 1                                                     # workspace too small
+    assert _rc(lib, "fused_moe_fp8_blockscale_g1u1_tiled", *a)[0] == 3
