@@ -220,8 +220,8 @@ def layer_work(cfg, ids, mask=None):
 # figure whose sources have changed since is not reported.
 GATE_UP_TRAFFIC = {
     "prefill_t4096_h7168_e256": {
-        "bytes": 6.835e9,
-        "sha256": "92eb4d672dca8e8c17daceb59748ff218b234d718ac3046361f63e3a464445bc",
+        "bytes": 6.810e9,
+        "sha256": "1b410dc9b6f77136e0368a93c182c91921b7c5aa3243d082a167790710085253",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
                    "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph --no-workloads` "
                    "(2 launches, mean; tiled weights)",
