@@ -563,20 +563,19 @@ def run_distributed(args, world, rank, local):
         model = D.TensorParallelMoE(full)
         del full
         torch.cuda.empty_cache()
-        routing_layer = model.shard
     else:
         e0, e1 = D.ep_expert_range(cfg.E, rank, world)
         model = D.ExpertParallelMoE(cfg, D.ExpertShard(cfg, e0, e1, dev).load_synthetic_weights())
-        routing_layer = MoELayer(cfg, dev)        # routing only, for the work count
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         out = model.forward(logits, bias, x)
     torch.cuda.synchronize()
     assert B.device_status() == 0, "device error word set during warm-up"
-    B.moe_biased_grouped_topk(logits, bias, routing_layer.topk_w, routing_layer.topk_ids, cfg.G, cfg.TG, cfg.renorm,
-                              cfg.scale)
-    work = layer_work(cfg, routing_layer.topk_ids)
+    topk_w = torch.empty(cfg.T, cfg.K, dtype=torch.float32, device=dev)      # the routing, for the work count
+    topk_ids = torch.empty(cfg.T, cfg.K, dtype=torch.int32, device=dev)
+    B.moe_biased_grouped_topk(logits, bias, topk_w, topk_ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+    work = layer_work(cfg, topk_ids)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.05)
