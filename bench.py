@@ -1,7 +1,7 @@
 """Benchmark of the fused FP8 block-scaled MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed|tiny|profile]
-                    [--impl ours|reference]
+                    [--tokens T] [--impl ours|reference]
 
 One step = one forward of the whole layer on the device: biased grouped top-k
 routing -> align/sort -> 1x128 activation quantisation -> fused g1u1 MoE
@@ -23,8 +23,10 @@ computation) on the host cores on a bounded token sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -634,12 +636,21 @@ def run_distributed(args, world, rank, local):
     }
 
 
+def workload_config(args):
+    """The MoE workload's configuration; with --tokens T, the same recipe (shapes, routing,
+    value distributions, seed) at T tokens: one point of a batch-size sweep."""
+    cfg = WORKLOADS[args.workload] if args.workload in WORKLOADS else DIST_WORKLOADS[args.workload]
+    if args.tokens is None:
+        return cfg
+    return dataclasses.replace(cfg, name=re.sub(r"_t\d+_", f"_t{args.tokens}_", cfg.name, count=1), T=args.tokens)
+
+
 def run_ours(args, world, rank, local):
     from fp8_block_scaled_biased_b200.layer import MoELayer
 
     if args.workload in DIST_WORKLOADS:
         return run_distributed(args, world, rank, local)
-    cfg = WORKLOADS[args.workload]
+    cfg = workload_config(args)
     dev = torch.device("cuda", local)
     layer = MoELayer(cfg, dev).load_synthetic_weights()
     if cfg.tp_ranks > 0:                            # keep only this rank's shard of the weights
@@ -647,7 +658,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.empty_cache()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     result = measure_layer(args, world, local, cfg, layer, flush, headline=True)
-    if args.workload == "prefill" and world == 1 and not args.no_workloads:
+    if args.workload == "prefill" and world == 1 and not args.no_workloads and args.tokens is None:
         extras = {}
         for name in EXTRA_WORKLOADS:
             if name == "gemm":
@@ -848,7 +859,7 @@ def run_reference_gemm(args, world):
 def run_reference(args, world, rank):
     if args.workload == "gemm":
         return run_reference_gemm(args, world)
-    cfg = WORKLOADS[args.workload] if args.workload in WORKLOADS else DIST_WORKLOADS[args.workload]
+    cfg = workload_config(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     runner = OracleSample(cfg, args.ref_sample_tokens, device=dev)
     for _ in range(args.warmup):
@@ -880,6 +891,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DIST_WORKLOADS) + ["gemm"], default="prefill",
                     help="MoE layer workload, or gemm: the standalone block-scale GEMM (M=2048, N=4096, K=7168)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the MoE workload's recipe at this many tokens (a batch-size sweep point; the "
+                         "workloads timed beside the prefill headline are then left out)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -894,6 +908,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
+    if args.tokens is not None and (args.tokens < 1 or args.workload not in WORKLOADS):
+        ap.error("--tokens takes a positive count and a single-GPU MoE workload")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -126,3 +126,23 @@ def test_source_hash_ignores_comments_and_layout_only(tmp_path):
     (tmp_path / "c.cu").write_text("int f(int a){return a+2;}\n")
     h = [bench.source_sha([str(tmp_path / n)]) for n in ("a.cu", "b.cu", "c.cu")]
     assert h[0] == h[1] != h[2]
+
+
+def test_tokens_option_keeps_the_recipe_at_another_batch_size():
+    """--tokens T is a batch-size sweep point: the workload's recipe (shapes, routing, seed)
+    at T tokens, named as such; the reference arm runs it too."""
+    import argparse
+    cfg = bench.workload_config(argparse.Namespace(workload="prefill", tokens=16))
+    assert cfg.T == 16 and cfg.name == "prefill_t16_h7168_e256"
+    assert (cfg.H, cfg.E, cfg.G, cfg.TG, cfg.K, cfg.I, cfg.seed) == (I.PREFILL.H, I.PREFILL.E, I.PREFILL.G,
+                                                                    I.PREFILL.TG, I.PREFILL.K, I.PREFILL.I,
+                                                                    I.PREFILL.seed)
+    assert bench.workload_config(argparse.Namespace(workload="decode", tokens=None)) is I.DECODE
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--tokens", "3",
+                        "--steps", "1", "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    (d,) = _json_lines(r.stdout)
+    assert d["config"]["workload"] == "tiny_t3_h256_e16" and d["config"]["T"] == 3
+    bad = subprocess.run([sys.executable, "bench.py", "--workload", "gemm", "--tokens", "3"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=600)
+    assert bad.returncode != 0 and "--tokens" in bad.stderr

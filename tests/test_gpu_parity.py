@@ -4,6 +4,8 @@ Bit-exact for routing ids/weights, the sort, and FP8 codes and scales; the
 stated tolerance for the GEMM and the fused MoE output. Inputs come from the
 seeded generator; each side quantises raw numbers with its own code.
 """
+import dataclasses
+
 import pytest
 import torch
 
@@ -433,6 +435,36 @@ def test_timing_hook_reports_each_fused_kernel():
         B.timing_enable(False)
     assert len(ms) == 4 and all(m > 0 for m in ms), ms
     assert sum(ms) <= start.elapsed_time(end) * 1.05 + 0.01
+
+
+@pytest.mark.parametrize("cfg", [ODD_ONE, MID, SKEW_SMALL], ids=lambda c: c.name)
+def test_graph_replays_follow_their_inputs(cfg):
+    """The layer's forward captured in a CUDA graph (as the bench replays it: quantisation on
+    a side stream joined before the fused call) gives on every replay exactly the eager
+    forward's output for the inputs then in its buffers. Two input sets with different
+    routings alternate between replays, so a kernel that read a buffer before its producer
+    wrote it, or a sorted list left from the previous replay, would show the other set's
+    values."""
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    sets = []
+    for seed in (cfg.seed, cfg.seed + 100):
+        act = I.moe_activations(dataclasses.replace(cfg, seed=seed))
+        args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+        sets.append((args, layer.forward(*args).clone()))
+    assert not torch.equal(sets[0][1], sets[1][1])
+    bufs = tuple(t.clone() for t in sets[0][0])
+    layer.forward(*bufs)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        out = layer.forward(*bufs)
+    for i in range(16):
+        args, want = sets[i % 2]
+        for b, a in zip(bufs, args):
+            b.copy_(a)
+        graph.replay()
+        assert torch.equal(out, want), f"replay {i}"
+    del graph
 
 
 def test_fused_moe_zero_tokens_is_a_no_op():
