@@ -562,7 +562,7 @@ def run_distributed(args, world, rank, local):
     logits, bias, x = act.logits.to(dev), act.bias.to(dev), act.x.to(dev)
     if args.workload == "prefill_tp":
         full = MoELayer(cfg, dev).load_synthetic_weights()
-        model = D.TensorParallelMoE(full)
+        model = D.TensorParallelMoE(full, reduce=args.tp_reduce)
         del full
         torch.cuda.empty_cache()
     else:
@@ -622,8 +622,9 @@ def run_distributed(args, world, rank, local):
         "config": {"workload": f"{cfg.name}_{'tp' if tp else 'ep'}{world}", "T": cfg.T, "H": cfg.H, "E": cfg.E,
                    "topk": cfg.K, "I": cfg.I,
                    "parallelism": (f"tp{world}: intermediate columns split over the ranks, one batch of {cfg.T} "
-                                   "tokens per step, partial outputs summed by an fp32 NCCL reduce-scatter and a "
-                                   "bf16 all-gather") if tp else
+                                   "tokens per step, partial outputs summed " +
+                                   ("by the combine fused with the all-reduce over peer memory" if args.tp_reduce ==
+                                    "peer" else "by an fp32 NCCL reduce-scatter and a bf16 all-gather")) if tp else
                                   (f"ep{world}: experts split over the ranks, each rank its own batch of {cfg.T} "
                                    "tokens, dispatch and return all-to-alls over NCCL"),
                    "l2": "flushed between steps (256 MB write)", "cuda_graph": False},
@@ -894,6 +895,9 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the MoE workload's recipe at this many tokens (a batch-size sweep point; the "
                          "workloads timed beside the prefill headline are then left out)")
+    ap.add_argument("--tp-reduce", choices=["peer", "nccl"], default="peer",
+                    help="prefill_tp: sum the ranks' partials with the combine fused with the all-reduce over "
+                         "peer memory (peer) or with NCCL's reduce-scatter and all-gather (nccl)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -52,10 +52,21 @@ _SIGNATURES = {
                                                      _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int, _p, _p,
                                                      _c_size, _p]),
     "fp8_tile_weights": (_c_int, [_p, _c_int, _c_int, _c_int, _p, _p]),
+    "fused_moe_fp8_blockscale_g1u1_pairs": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
+                                                     _c_int, _c_int, _c_size, _p, _p, _p, _c_int, _c_int, _p,
+                                                     _c_int, _p, _c_size, _p]),
+    "moe_tp_recv_bytes": (_c_size, [_c_int, _c_int, _c_int]),
+    "moe_combine_allreduce": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p,
+                                       ctypes.c_uint64, _p]),
+    "moe_combine_allreduce_emulated": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p,
+                                                ctypes.c_uint64, _p]),
 }
 EXPORTED = tuple(_SIGNATURES)
 
 NOALLOC_SCRATCH_BYTES = 64 << 20   # FP8MOE_NOALLOC_SCRATCH_BYTES in include/fp8moe.h
+TP_MAX_RANKS = 8                   # FP8MOE_TP_MAX_RANKS
+TP_FLAG_WORDS = 16                 # FP8MOE_TP_FLAG_WORDS (64-bit words per rank)
+TP_BARRIER_WORDS = 2               # FP8MOE_TP_BARRIER_WORDS
 SCALE_ROW_MAJOR = 0
 SCALE_COL_MAJOR = 1
 FP8 = torch.float8_e4m3fn
@@ -328,12 +339,14 @@ def fused_moe_workspace_bytes(T, topk, E, H, I, block_m, capacity=None):
 
 
 def _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale):
-    """Checks shared by both fused MoE entry points; returns (T, H, I, E).
+    """Checks shared by the fused MoE entry points; returns (T, H, I, E). out is None for
+    the call without a combine.
 
     The library builds its TMA maps from these sizes (w1 as E*2I rows of H, w2 as
     E*H rows of I), so every tensor must have exactly the shape and dtype the sizes
     imply and be contiguous; anything else is refused before the call."""
-    _cuda(out, torch.bfloat16, "out")
+    if out is not None:
+        _cuda(out, torch.bfloat16, "out")
     _cuda(a8, FP8, "a8")
     _cuda(w1, FP8, "w1")
     _cuda(w2, FP8, "w2")
@@ -350,7 +363,7 @@ def _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, 
         raise ValueError("g1u1 requires 2I rows of w1 for I columns of w2")
     if H1 != H or (E2, H2) != (E, H):
         raise ValueError(f"w1 {tuple(w1.shape)} and w2 {tuple(w2.shape)} do not match a8's H={H}")
-    if tuple(out.shape) != (T, H):
+    if out is not None and tuple(out.shape) != (T, H):
         raise ValueError(f"out must be [{T}, {H}], got {tuple(out.shape)}")
     if H % 128 or I % 128:
         raise ValueError(f"H and I must be multiples of 128 (H={H}, I={I})")
@@ -361,7 +374,7 @@ def _fused_moe_shapes(out, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, 
             raise ValueError(f"{name} must be {expect[name]}, got {tuple(t.shape)}")
     for name, t in (("out", out), ("a8", a8), ("w1", w1), ("w2", w2), ("a1_scale", a1_scale),
                     ("fc1_scale", fc1_scale), ("fc2_scale", fc2_scale)):
-        if not t.is_contiguous():
+        if t is not None and not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
     sp = sorted_pairs
     for name, t, dt in (("sorted_ids", sp.sorted_ids, torch.int32), ("sorted_weights", sp.sorted_weights, torch.float32),
@@ -416,3 +429,76 @@ def fused_moe_fp8_blockscale_g1u1_noalloc(out, a8, w1, w2, sorted_pairs: SortedP
         _stream())
     _check("fused_moe_fp8_blockscale_g1u1_noalloc", rc)
     return out
+
+
+# ---------------------------------------------------------------- tensor-parallel combine + all-reduce
+def fused_moe_fp8_blockscale_g1u1_pairs(a8, w1, w2, sorted_pairs: SortedPairs, topk, a1_scale, fc1_scale, fc2_scale,
+                                        workspace=None, scale_blk_n=128, scale_blk_k=128, fc2_smooth_scale=None):
+    """The fused call without its combine (one tensor-parallel rank's share of I): the
+    weighted pair rows and pair flags are left in the returned workspace for
+    moe_combine_allreduce. Arguments and checks as fused_moe_fp8_blockscale_g1u1, minus out."""
+    T, H, I, E = _fused_moe_shapes(None, a8, w1, w2, sorted_pairs, topk, a1_scale, fc1_scale, fc2_scale)
+    sp = sorted_pairs
+    if workspace is None:
+        need = fused_moe_workspace_bytes(T, topk, E, H, I, sp.block_m, capacity=sp.capacity)
+        workspace = torch.empty(need, dtype=torch.uint8, device=a8.device)
+    rc = load_library().fused_moe_fp8_blockscale_g1u1_pairs(
+        _ptr(a8), _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids), _ptr(sp.sorted_weights), _ptr(sp.sorted_expert_ids),
+        _ptr(sp.num_valid_ids), T, H, I, E, topk, sp.block_m, sp.capacity, _ptr(a1_scale), _ptr(fc1_scale),
+        _ptr(fc2_scale), scale_blk_n, scale_blk_k, _ptr(fc2_smooth_scale), 1 if is_tiled(w1) else 0,
+        _ptr(workspace), workspace.numel(), _stream())
+    _check("fused_moe_fp8_blockscale_g1u1_pairs", rc)
+    return workspace
+
+
+def moe_tp_recv_bytes(T, H, nranks):
+    """Bytes of one rank's receive buffer for moe_combine_allreduce."""
+    return load_library().moe_tp_recv_bytes(T, H, nranks)
+
+
+def _addresses(items, name):
+    """A ctypes array of device addresses from tensors or plain integer addresses."""
+    addrs = [t if isinstance(t, int) else t.data_ptr() for t in items]
+    if any(a == 0 for a in addrs):
+        raise ValueError(f"{name}: null address")
+    return (ctypes.c_void_p * len(addrs))(*addrs)
+
+
+def moe_combine_allreduce(workspace, capacity, T, topk, H, I, rank, recv, out, flags, barrier, epoch):
+    """One tensor-parallel rank's fused combine + all-reduce (include/fp8moe.h). recv, out,
+    flags: one device address (or tensor) per rank, as this GPU addresses that rank's buffer;
+    barrier: int64 [TP_BARRIER_WORDS] on this GPU; epoch: larger than every earlier call's."""
+    _cuda(workspace, torch.uint8, "workspace")
+    _cuda(barrier, torch.int64, "barrier")
+    n = len(recv)
+    if not (len(out) == len(flags) == n) or not 1 <= n <= TP_MAX_RANKS:
+        raise ValueError("recv, out and flags need one entry per rank (at most TP_MAX_RANKS)")
+    if barrier.numel() < TP_BARRIER_WORDS:
+        raise ValueError("barrier too small")
+    rc = load_library().moe_combine_allreduce(
+        _ptr(workspace), capacity, T, topk, H, I, n, rank, _addresses(recv, "recv"), _addresses(out, "out"),
+        _addresses(flags, "flags"), _ptr(barrier), epoch, _stream())
+    _check("moe_combine_allreduce", rc)
+
+
+def moe_combine_allreduce_emulated(workspaces, capacity, T, topk, H, I, recv, out, flags, barriers, epoch):
+    """Every rank of moe_combine_allreduce on this GPU in one launch (the rank protocol on one
+    device). Per rank r: workspaces[r] (its pairs call's workspace), recv[r] bf16 [n, Ts, H],
+    out[r] bf16 [T, H], flags[r] int64 [TP_FLAG_WORDS], barriers[r] int64 [TP_BARRIER_WORDS]."""
+    n = len(workspaces)
+    if not (len(recv) == len(out) == len(flags) == len(barriers) == n) or not 1 <= n <= TP_MAX_RANKS:
+        raise ValueError("one workspace, recv, out, flags and barrier per rank (at most TP_MAX_RANKS)")
+    Ts = -(-T // n)
+    for r in range(n):
+        _cuda(workspaces[r], torch.uint8, "workspaces")
+        _cuda(recv[r], torch.bfloat16, "recv")
+        _cuda(out[r], torch.bfloat16, "out")
+        _cuda(flags[r], torch.int64, "flags")
+        _cuda(barriers[r], torch.int64, "barriers")
+        if recv[r].numel() < n * Ts * H or out[r].numel() < T * H or flags[r].numel() < TP_FLAG_WORDS \
+                or barriers[r].numel() < TP_BARRIER_WORDS:
+            raise ValueError(f"rank {r}: a buffer is smaller than the call needs")
+    rc = load_library().moe_combine_allreduce_emulated(
+        _addresses(workspaces, "workspaces"), capacity, T, topk, H, I, n, _addresses(recv, "recv"),
+        _addresses(out, "out"), _addresses(flags, "flags"), _addresses(barriers, "barriers"), epoch, _stream())
+    _check("moe_combine_allreduce_emulated", rc)

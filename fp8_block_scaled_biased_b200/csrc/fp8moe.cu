@@ -17,6 +17,7 @@
 #include "quant.cuh"
 #include "route.cuh"
 #include "sort.cuh"
+#include "tp_reduce.cuh"
 
 static_assert(fp8moe::kMoeBlockRows == fp8moe::kBM, "sorted blocks are GEMM tiles");
 
@@ -507,8 +508,11 @@ size_t fused_moe_fp8_blockscale_g1u1_workspace(int T, int topk, int E, int H, in
 
 }  // extern "C"
 
-// The fused MoE call on row-major (tiled == false) or tiled (fp8_tile_weights) weights.
-static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uint8_t* a8, const uint8_t* w1,
+// The fused MoE call on row-major (tiled == false) or tiled (fp8_tile_weights) weights;
+// with combine == false it stops after the down GEMM (the weighted pair rows and the
+// pair flags stay in the workspace) and out is not used.
+static int fused_moe_impl(const char* name, bool tiled, bool combine, uint16_t* out, const uint8_t* a8,
+                          const uint8_t* w1,
                           const uint8_t* w2, const int32_t* sorted_ids, const float* sorted_weights,
                           const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H, int I, int E,
                           int topk, int block_m, size_t capacity, const float* a1_scale, const float* fc1_scale,
@@ -529,7 +533,7 @@ static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uin
     return fail(FP8MOE_EINVAL, "capacity %zu below the sort's bound %zu", capacity,
                 moe_align_sort_capacity(T, topk, E, block_m));
   if (T == 0) return FP8MOE_OK;
-  if (!out || !a8 || !w1 || !w2 || !sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids ||
+  if ((combine && !out) || !a8 || !w1 || !w2 || !sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids ||
       !a1_scale || !fc1_scale || !fc2_scale)
     return fail(FP8MOE_EINVAL, "null pointer argument");
   if (!aligned16(a8) || !aligned16(w1) || !aligned16(w2) || !aligned16(sorted_ids) || !aligned16(out))
@@ -629,6 +633,7 @@ static int fused_moe_impl(const char* name, bool tiled, uint16_t* out, const uin
                                  kGemmSmemBytes))
     return rc;
   timing_record(3, st);
+  if (!combine) return FP8MOE_OK;
 
   const size_t threads = static_cast<size_t>(T) * (H / 8);
   moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
@@ -647,7 +652,7 @@ int fused_moe_fp8_blockscale_g1u1(uint16_t* out, const uint8_t* a8, const uint8_
                                   const float* fc1_scale, const float* fc2_scale, int scale_blk_n, int scale_blk_k,
                                   const float* fc2_smooth_scale, void* workspace, size_t workspace_bytes,
                                   void* stream) {
-  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1", false, out, a8, w1, w2, sorted_ids, sorted_weights,
+  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1", false, true, out, a8, w1, w2, sorted_ids, sorted_weights,
                         sorted_expert_ids, num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
                         fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, workspace, workspace_bytes, stream);
 }
@@ -659,7 +664,7 @@ int fused_moe_fp8_blockscale_g1u1_tiled(uint16_t* out, const uint8_t* a8, const 
                                         const float* fc1_scale, const float* fc2_scale, int scale_blk_n,
                                         int scale_blk_k, const float* fc2_smooth_scale, void* workspace,
                                         size_t workspace_bytes, void* stream) {
-  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1_tiled", true, out, a8, w1, w2, sorted_ids, sorted_weights,
+  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1_tiled", true, true, out, a8, w1, w2, sorted_ids, sorted_weights,
                         sorted_expert_ids, num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
                         fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, workspace, workspace_bytes, stream);
 }
@@ -741,6 +746,129 @@ int fused_moe_fp8_blockscale_g1u1_noalloc(uint16_t* out, const uint8_t* a8, cons
                                        num_valid_ids, T, H, I, E, topk, block_m, capacity, a1_scale, fc1_scale,
                                        fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, scratch,
                                        FP8MOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// ------------------------------------------------------------------ tensor-parallel combine + all-reduce
+int fused_moe_fp8_blockscale_g1u1_pairs(const uint8_t* a8, const uint8_t* w1, const uint8_t* w2,
+                                        const int32_t* sorted_ids, const float* sorted_weights,
+                                        const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H,
+                                        int I, int E, int topk, int block_m, size_t capacity, const float* a1_scale,
+                                        const float* fc1_scale, const float* fc2_scale, int scale_blk_n,
+                                        int scale_blk_k, const float* fc2_smooth_scale, int weights_tiled,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1_pairs", weights_tiled != 0, false, nullptr, a8, w1, w2,
+                        sorted_ids, sorted_weights, sorted_expert_ids, num_valid_ids, T, H, I, E, topk, block_m,
+                        capacity, a1_scale, fc1_scale, fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale,
+                        workspace, workspace_bytes, stream);
+}
+
+size_t moe_tp_recv_bytes(int T, int H, int nranks) {
+  if (T < 0 || H < 0 || nranks < 1 || nranks > FP8MOE_TP_MAX_RANKS) return 0;
+  const size_t Ts = (static_cast<size_t>(T) + nranks - 1) / nranks;
+  return static_cast<size_t>(nranks) * Ts * H * sizeof(__nv_bfloat16);
+}
+
+}  // extern "C"
+
+static_assert(FP8MOE_TP_MAX_RANKS == kTpMaxRanks && FP8MOE_TP_FLAG_WORDS == kTpFlagWords, "header and kernel agree");
+
+// Checks shared by the one-rank and the emulated launches: fills `a` (the peer
+// buffers, and the workspace buffers of the nlocal ranks launched here) and
+// *ctas (CTAs per rank: all of the launch must be resident at once).
+static int tp_setup(const char* name, int nranks, int T, int topk, int H, int I, size_t capacity,
+                    const void* const* workspaces, const int* ranks, int nlocal, void* const* recv,
+                    void* const* out, uint64_t* const* flags, uint64_t* const* barriers, uint64_t epoch,
+                    TpArgs* a, int* ctas) {
+  if (nranks < 1 || nranks > kTpMaxRanks) return fail(FP8MOE_EINVAL, "%s: nranks must be in [1, %d]", name, kTpMaxRanks);
+  if (T < 1 || topk < 1 || topk > 32) return fail(FP8MOE_EINVAL, "%s: T >= 1 and topk in [1, 32] required", name);
+  if (H < 128 || H % 128 || I < 128 || I % 128)
+    return fail(FP8MOE_EUNSUPPORTED, "%s: H and I must be positive multiples of 128", name);
+  if (static_cast<long long>(T) * topk >= (1ll << 31) || static_cast<long long>(T) * (H / 8) >= (1ll << 40))
+    return fail(FP8MOE_EUNSUPPORTED, "%s: T too large", name);
+  if (epoch == 0) return fail(FP8MOE_EINVAL, "%s: epoch must be >= 1", name);
+  if (!recv || !out || !flags) return fail(FP8MOE_EINVAL, "%s: null pointer argument", name);
+  *a = TpArgs{};
+  for (int p = 0; p < nranks; ++p) {
+    if (!recv[p] || !out[p] || !flags[p]) return fail(FP8MOE_EINVAL, "%s: null buffer of rank %d", name, p);
+    if (!aligned16(recv[p]) || !aligned16(out[p]) || (reinterpret_cast<uintptr_t>(flags[p]) & 7u))
+      return fail(FP8MOE_EINVAL, "%s: rank %d's buffers must be 16-byte (flags 8-byte) aligned", name, p);
+    a->recv[p] = static_cast<__nv_bfloat16*>(recv[p]);
+    a->out[p] = static_cast<__nv_bfloat16*>(out[p]);
+    a->flags[p] = reinterpret_cast<unsigned long long*>(flags[p]);
+  }
+  const MoeWorkspace lay = moe_workspace_layout(capacity, T, topk, H, I);
+  for (int i = 0; i < nlocal; ++i) {
+    const int r = ranks[i];
+    if (!workspaces[i] || !barriers[i]) return fail(FP8MOE_EINVAL, "%s: null workspace or barrier", name);
+    if (reinterpret_cast<uintptr_t>(workspaces[i]) & 255u)
+      return fail(FP8MOE_EINVAL, "%s: workspace must be 256-byte aligned", name);
+    if (reinterpret_cast<uintptr_t>(barriers[i]) & 7u) return fail(FP8MOE_EINVAL, "%s: barrier must be 8-byte aligned", name);
+    const uint8_t* ws = static_cast<const uint8_t*>(workspaces[i]);
+    a->ystage[r] = reinterpret_cast<const __nv_bfloat16*>(ws + lay.y_off);
+    a->n_present[r] = reinterpret_cast<const int*>(ws + lay.flag_off);
+    a->pair_flag[r] = ws + lay.flag_off + 16;
+    a->barrier[r] = reinterpret_cast<unsigned long long*>(barriers[i]);
+  }
+  a->nranks = nranks;
+  a->T = T;
+  a->K = topk;
+  a->H = H;
+  a->epoch = epoch;
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tp_combine_allreduce_kernel, kTpThreads, 0) !=
+          cudaSuccess || per_sm < 1)
+    return fail(FP8MOE_ECUDA, "%s: occupancy query failed", name);
+  const long long resident = static_cast<long long>(per_sm) * sms / nlocal;
+  const long long need = (static_cast<long long>(T) * (H / 8) + kTpThreads - 1) / kTpThreads;
+  *ctas = static_cast<int>(std::min(resident, need));
+  if (*ctas < 1) return fail(FP8MOE_EUNSUPPORTED, "%s: %d ranks do not fit one GPU", name, nlocal);
+  return FP8MOE_OK;
+}
+
+static int tp_launch(const char* name, const TpArgs& a, int rank_first, int ctas, int nlocal, void* stream) {
+  void* args[] = {const_cast<TpArgs*>(&a), &rank_first, &ctas};
+  const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(tp_combine_allreduce_kernel),
+                                                    dim3(ctas * nlocal), dim3(kTpThreads), args, 0,
+                                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FP8MOE_ECUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+  }
+  return check_launch(name);
+}
+
+extern "C" {
+
+int moe_combine_allreduce(const void* workspace, size_t capacity, int T, int topk, int H, int I, int nranks,
+                          int rank, void* const* recv, void* const* out, uint64_t* const* flags, uint64_t* barrier,
+                          uint64_t epoch, void* stream) {
+  if (nranks < 1 || rank < 0 || rank >= nranks) return fail(FP8MOE_EINVAL, "moe_combine_allreduce: bad rank");
+  TpArgs a;
+  int ctas = 0;
+  const void* ws[1] = {workspace};
+  uint64_t* bars[1] = {barrier};
+  const int ranks[1] = {rank};
+  if (int rc = tp_setup("moe_combine_allreduce", nranks, T, topk, H, I, capacity, ws, ranks, 1, recv, out, flags,
+                        bars, epoch, &a, &ctas))
+    return rc;
+  return tp_launch("moe_combine_allreduce", a, rank, ctas, 1, stream);
+}
+
+int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacity, int T, int topk, int H, int I,
+                                   int nranks, void* const* recv, void* const* out, uint64_t* const* flags,
+                                   uint64_t* const* barriers, uint64_t epoch, void* stream) {
+  if (!workspaces || !barriers) return fail(FP8MOE_EINVAL, "moe_combine_allreduce_emulated: null pointer argument");
+  if (nranks < 1 || nranks > kTpMaxRanks) return fail(FP8MOE_EINVAL, "moe_combine_allreduce_emulated: bad nranks");
+  TpArgs a;
+  int ctas = 0;
+  int ranks[kTpMaxRanks];
+  for (int r = 0; r < nranks; ++r) ranks[r] = r;
+  if (int rc = tp_setup("moe_combine_allreduce_emulated", nranks, T, topk, H, I, capacity, workspaces, ranks, nranks,
+                        recv, out, flags, barriers, epoch, &a, &ctas))
+    return rc;
+  return tp_launch("moe_combine_allreduce_emulated", a, 0, ctas, nranks, stream);
 }
 
 }  // extern "C"

@@ -8,10 +8,16 @@ Operators", and gives asm_moe an expert_mask (section "Blockscale FP8 MoE
 Computation"), the hook of expert parallelism. Two forms are built here:
 
 Tensor parallelism over I (TensorParallelMoE). Every rank routes every token and
-runs its shard of each expert's intermediate columns (MoELayer.tp_shard); the
-ranks' bf16 partial outputs are summed by tp_reduce: an fp32 reduce-scatter (each
-rank sums one slice of the tokens over all ranks) and a bf16 all-gather of the
-rounded slices.
+runs its shard of each expert's intermediate columns (MoELayer.tp_shard). The
+ranks' partial outputs are summed either by the library's combine fused with the
+all-reduce over peer memory (reduce="peer": each rank combines its pair rows per
+token and stores the bf16 partial straight into the receive buffer of the rank that
+owns the token's slice, over NVLink; the owners sum in rank order and store the
+result into every rank's output; TpPeerAllReduce holds the buffers, in torch's
+symmetric memory), or by tp_reduce (reduce="nccl": an fp32 reduce-scatter over
+NCCL, each rank summing one slice of the tokens, and a bf16 all-gather). Both sum
+the same bf16 partials in fp32 and round once; the peer form fixes the order (rank
+order) and saves the combine's separate pass over the partial output.
 
 Expert parallelism over E (ExpertParallelMoE). Rank r holds experts
 [r*E/n, (r+1)*E/n) and its own batch of tokens. It routes and quantises its
@@ -70,23 +76,116 @@ def tp_reduce(partial: torch.Tensor, group=None) -> torch.Tensor:
     return out[:T]
 
 
+@dataclasses.dataclass(frozen=True)
+class TpBufferLayout:
+    """Byte offsets of one rank's buffers for moe_combine_allreduce inside one allocation:
+    the receive buffer bf16 [n][ceil(T/n)][H], the output bf16 [T][H] and the flag words
+    (each part starting at a multiple of 256 bytes)."""
+    recv: int
+    out: int
+    flags: int
+    total: int
+
+
+def tp_buffer_layout(T: int, H: int, n: int) -> TpBufferLayout:
+    if not 1 <= n <= B.TP_MAX_RANKS or T < 1 or H < 1:
+        raise ValueError(f"bad tensor-parallel buffer shape T={T}, H={H}, n={n}")
+    up = lambda v: -(-v // 256) * 256   # noqa: E731
+    Ts = -(-T // n)
+    recv = 0
+    out = up(n * Ts * H * 2)
+    flags = out + up(T * H * 2)
+    return TpBufferLayout(recv, out, flags, flags + up(B.TP_FLAG_WORDS * 8))
+
+
+class TpPeerAllReduce:
+    """One rank's buffers for the combine fused with the all-reduce (moe_combine_allreduce):
+    the receive buffer, the output and the flag words in one allocation of torch's symmetric
+    memory, exchanged over the group so that every rank's buffers are addressable from every
+    GPU (over NVLink); the CTA barrier words in this GPU's memory; the call counter (epoch).
+    Every rank of the group must construct it and then make the same calls."""
+
+    def __init__(self, T: int, H: int, group=None, device=None):
+        import torch.distributed._symmetric_memory as symm
+        n, r = _world(group), _rank(group)
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.T, self.H, self.n, self.rank = T, H, n, r
+        self.layout = L = tp_buffer_layout(T, H, n)
+        self.buf = symm.empty(L.total, dtype=torch.uint8, device=dev)
+        self.buf.zero_()
+        handle = symm.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
+        bases = [int(b) for b in handle.buffer_ptrs]
+        self._handle = handle
+        self.recv = [b + L.recv for b in bases]
+        self.outs = [b + L.out for b in bases]
+        self.flags = [b + L.flags for b in bases]
+        self.out = self.buf[L.out:L.out + T * H * 2].view(torch.bfloat16).view(T, H)
+        self.barrier = torch.zeros(B.TP_BARRIER_WORDS, dtype=torch.int64, device=dev)
+        self.epoch = 0
+        torch.cuda.synchronize(dev)
+        if dist.is_initialized() and n > 1:
+            dist.barrier(group)            # every rank's flags are zero before any rank's first call
+
+    def __call__(self, workspace, capacity: int, topk: int, I: int) -> torch.Tensor:
+        """Combine this rank's pair rows (left in `workspace` by the pairs call) and all-reduce
+        them; returns this rank's output buffer bf16 [T, H] (rewritten by the next call)."""
+        self.epoch += 1
+        B.moe_combine_allreduce(workspace, capacity, self.T, topk, self.H, I, self.rank, self.recv, self.outs,
+                                self.flags, self.barrier, self.epoch)
+        return self.out
+
+
+class EmulatedTpAllReduce:
+    """Every rank of the fused combine + all-reduce on one GPU: each rank's receive buffer,
+    output, flags and barrier words in this GPU's memory, all ranks run by one cooperative
+    launch (moe_combine_allreduce_emulated) through the same per-rank code and flags as the
+    multi-GPU form."""
+
+    def __init__(self, T: int, H: int, n: int, device="cuda"):
+        tp_buffer_layout(T, H, n)
+        Ts = -(-T // n)
+        self.T, self.H, self.n = T, H, n
+        self.recv = [torch.empty(n, Ts, H, dtype=torch.bfloat16, device=device) for _ in range(n)]
+        self.out = [torch.empty(T, H, dtype=torch.bfloat16, device=device) for _ in range(n)]
+        self.flags = [torch.zeros(B.TP_FLAG_WORDS, dtype=torch.int64, device=device) for _ in range(n)]
+        self.barriers = [torch.zeros(B.TP_BARRIER_WORDS, dtype=torch.int64, device=device) for _ in range(n)]
+        self.epoch = 0
+
+    def __call__(self, workspaces, capacity: int, topk: int, I: int):
+        """workspaces[r]: rank r's pairs-call workspace. Returns the n ranks' outputs."""
+        self.epoch += 1
+        B.moe_combine_allreduce_emulated(workspaces, capacity, self.T, topk, self.H, I, self.recv, self.out,
+                                         self.flags, self.barriers, self.epoch)
+        return self.out
+
+
 class TensorParallelMoE:
     """One rank of the layer split over I: its shard (rank, n) of every expert, the whole
-    routing, and tp_reduce of the partial outputs."""
+    routing, and the sum of the ranks' partial outputs: reduce="peer" (the combine fused
+    with the all-reduce over peer memory, TpPeerAllReduce) or reduce="nccl" (tp_reduce)."""
 
-    def __init__(self, layer, group=None):
+    def __init__(self, layer, group=None, reduce: str = "nccl"):
         """layer: the whole MoELayer (its shard is copied out) or an already-sharded one
         whose cfg.tp_ranks / tp_rank match the group."""
-        self.group = group
+        if reduce not in ("peer", "nccl"):
+            raise ValueError("reduce must be 'peer' or 'nccl'")
+        self.group, self.reduce = group, reduce
         n, r = _world(group), _rank(group)
         if layer.cfg.tp_ranks == n and layer.cfg.tp_rank == r:
             self.shard = layer
         else:
             self.shard = layer.tp_shard(r, n) if n > 1 else layer
+        self.peer = None
 
     def forward(self, logits, bias, x):
-        partial = self.shard.forward(logits, bias, x)
-        return tp_reduce(partial, self.group)
+        if self.reduce == "nccl":
+            partial = self.shard.forward(logits, bias, x)
+            return tp_reduce(partial, self.group)
+        sh = self.shard
+        if self.peer is None:
+            self.peer = TpPeerAllReduce(x.shape[0], sh.cfg.H, self.group, x.device)
+        ws = sh.forward_pairs(logits, bias, x)
+        return self.peer(ws, sh.sorted.capacity, sh.cfg.K, sh.cfg.I)
 
 
 # ---------------------------------------------------------------------------------- expert parallel

@@ -121,6 +121,22 @@ class MoELayer:
         expert_mask: optional int32 [E] on the device (nonzero = an expert this GPU holds).
         The result is then the sum over the kept experts' pairs only, the partial output
         of one expert-parallel rank."""
+        self._route_sort_quant(logits, bias, x, expert_mask)
+        B.fused_moe_fp8_blockscale_g1u1(self.out, self.a8, self.w1, self.w2, self.sorted, self.cfg.K, self.a8_scale,
+                                        self.w1_scale, self.w2_scale, workspace=self.workspace)
+        return self.out
+
+    def forward_pairs(self, logits, bias, x):
+        """forward() without the combine: routing, sorting, quantisation and
+        fused_moe_fp8_blockscale_g1u1_pairs. The weighted pair rows and the pair flags are
+        left in self.workspace, where moe_combine_allreduce (a tensor-parallel rank's
+        combine fused with the all-reduce) reads them; returns that workspace."""
+        self._route_sort_quant(logits, bias, x, None)
+        return B.fused_moe_fp8_blockscale_g1u1_pairs(self.a8, self.w1, self.w2, self.sorted, self.cfg.K,
+                                                      self.a8_scale, self.w1_scale, self.w2_scale,
+                                                      workspace=self.workspace)
+
+    def _route_sort_quant(self, logits, bias, x, expert_mask):
         cfg = self.cfg
         T = x.shape[0]
         if T != self.max_tokens:
@@ -135,9 +151,6 @@ class MoELayer:
         B.moe_align_sort(self.topk_ids, self.topk_w, cfg.E, self.block_m, out=self.sorted,
                          workspace=self.sort_workspace, expert_mask=expert_mask)
         main.wait_event(self._join)
-        B.fused_moe_fp8_blockscale_g1u1(self.out, self.a8, self.w1, self.w2, self.sorted, cfg.K, self.a8_scale,
-                                        self.w1_scale, self.w2_scale, workspace=self.workspace)
-        return self.out
 
     @property
     def launches_per_forward(self):

@@ -366,6 +366,96 @@ int fused_moe_fp8_blockscale_g1u1_noalloc(uint16_t* out, const uint8_t* a8,
                                           const float* fc2_smooth_scale,
                                           void* stream);
 
+/*
+ * S4-S6 for tensor parallelism: the fused call without its combine.
+ * ("Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang", sections
+ * "Blockscale FP8 MoE Computation" and "Performance Reproduction for
+ * AITER-Optimized in SGLang": the layer at --tp 8, each rank holding a slice of
+ * every expert's intermediate columns.)
+ *
+ * Arguments, limits and workspace as fused_moe_fp8_blockscale_g1u1 (weights_tiled
+ * == 0) or fused_moe_fp8_blockscale_g1u1_tiled (weights_tiled != 0), minus out:
+ * the call stops after the down GEMM and leaves the weighted pair rows, the
+ * listed-pair count and the pair flags in the workspace (the layout given
+ * above), where moe_combine_allreduce reads them. I is the rank's share of the
+ * intermediate columns.
+ */
+int fused_moe_fp8_blockscale_g1u1_pairs(const uint8_t* a8, const uint8_t* w1,
+                                        const uint8_t* w2,
+                                        const int32_t* sorted_ids,
+                                        const float* sorted_weights,
+                                        const int32_t* sorted_expert_ids,
+                                        const int32_t* num_valid_ids,
+                                        int T, int H, int I, int E, int topk,
+                                        int block_m, size_t capacity,
+                                        const float* a1_scale, const float* fc1_scale,
+                                        const float* fc2_scale, int scale_blk_n,
+                                        int scale_blk_k, const float* fc2_smooth_scale,
+                                        int weights_tiled, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
+ * S7 fused with the tensor-parallel all-reduce, over peer (NVLink) memory.
+ * ("Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang", section
+ * "Other Operators": the custom all-reduce that sums the TP ranks' outputs.)
+ *
+ * Rank `rank` of `nranks` (<= FP8MOE_TP_MAX_RANKS), after its
+ * fused_moe_fp8_blockscale_g1u1_pairs call on `workspace` (same capacity, T,
+ * topk, H and I): with Ts = ceil(T / nranks), token t belongs to rank t / Ts.
+ *   1. For every token t, partial_r[t] = bf16(fp32 sum of the rank's listed pair
+ *      rows of t in k order) is stored into recv[p] at [r][t - p*Ts] of the
+ *      owning rank p.
+ *   2. For the tokens of its slice, every rank sums the nranks partials in rank
+ *      order in fp32, rounds to bf16 once and stores the row into out[p] of every
+ *      rank p. Every rank's out ends up bitwise identical:
+ *        out[t] = bf16( sum_{q=0..n-1} partial_q[t] ).
+ * One cooperative launch per rank; the call's kernel returns once every rank
+ * has written this rank's out.
+ *
+ * recv[p]   rank p's receive buffer, bf16 [nranks][Ts][H]
+ *           (moe_tp_recv_bytes bytes), 16-byte aligned
+ * out[p]    rank p's output, bf16 [T][H], 16-byte aligned
+ * flags[p]  rank p's FP8MOE_TP_FLAG_WORDS 64-bit words, zero before the first
+ *           call, 8-byte aligned
+ *           (recv, out and flags are host arrays of nranks device pointers, each
+ *           as this GPU addresses that rank's memory: peer memory mapped by
+ *           CUDA IPC or virtual memory management, or local memory for this rank)
+ * barrier   FP8MOE_TP_BARRIER_WORDS 64-bit words in this GPU's memory, zero
+ *           before the first call (the rank's CTAs meet there)
+ * epoch     larger than the epoch of every earlier call on these flags (for
+ *           example 1, 2, 3, ...); every rank of a call passes the same epoch
+ * Ownership: every buffer belongs to the caller; nothing is allocated. Every rank
+ * must make the same sequence of calls; a rank that does not arrive leaves the
+ * others waiting until the bounded wait (about 2 s) expires, which sets
+ * FP8MOE_DEVERR_TIMEOUT, after which the output is unspecified and flags and
+ * barrier must be zeroed again before the next call. out may be read by later
+ * work on the same stream; a second call overwrites it.
+ * Returns FP8MOE_EINVAL for a bad rank, size, alignment or null pointer and
+ * FP8MOE_ECUDA when the cooperative launch fails.
+ */
+#define FP8MOE_TP_MAX_RANKS 8
+#define FP8MOE_TP_FLAG_WORDS 16
+#define FP8MOE_TP_BARRIER_WORDS 2
+size_t moe_tp_recv_bytes(int T, int H, int nranks);
+int moe_combine_allreduce(const void* workspace, size_t capacity, int T, int topk,
+                          int H, int I, int nranks, int rank, void* const* recv,
+                          void* const* out, uint64_t* const* flags, uint64_t* barrier,
+                          uint64_t epoch, void* stream);
+
+/*
+ * All nranks ranks of moe_combine_allreduce on this one GPU, in one cooperative
+ * launch (each rank's share of the CTAs runs exactly the code of a one-rank
+ * launch; the ranks wait on one another through the same flags and barriers).
+ * workspaces[r] and barriers[r] are rank r's; every buffer is in this GPU's
+ * memory. For testing the multi-rank protocol on a single GPU; the ranks' CTAs
+ * must fit on the GPU at once (FP8MOE_EUNSUPPORTED otherwise).
+ */
+int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacity,
+                                   int T, int topk, int H, int I, int nranks,
+                                   void* const* recv, void* const* out,
+                                   uint64_t* const* flags, uint64_t* const* barriers,
+                                   uint64_t epoch, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -141,3 +141,27 @@ def test_single_rank_forms_need_no_process_group():
     assert torch.equal(D.ep_combine(rows, plan), rows)
     with pytest.raises(ValueError):
         D.ep_expert_range(10, 0, 4)
+
+
+def test_tensor_parallel_buffer_layout():
+    """One allocation per rank for the fused combine + all-reduce: the receive buffer bf16
+    [n][ceil(T/n)][H], the output bf16 [T][H] and the flag words, each 256-byte aligned and
+    not overlapping."""
+    for T, H, n in ((4096, 7168, 8), (300, 1024, 8), (1, 128, 1), (37, 640, 3)):
+        L = D.tp_buffer_layout(T, H, n)
+        Ts = -(-T // n)
+        assert L.recv == 0 and L.out >= n * Ts * H * 2 and L.flags >= L.out + T * H * 2
+        assert L.total >= L.flags + 16 * 8
+        assert L.out % 256 == 0 and L.flags % 256 == 0
+    assert D.tp_buffer_layout(4096, 7168, 8).total == 117440768
+    for bad in ((0, 128, 1), (16, 128, 0), (16, 128, 9)):
+        with pytest.raises(ValueError):
+            D.tp_buffer_layout(*bad)
+
+
+def test_tensor_parallel_reduce_choice_is_checked():
+    class _Layer:
+        cfg = I.MoEConfig("t", T=4, H=128, E=4, G=1, TG=1, K=2, I=128, tp_ranks=1, tp_rank=0)
+    assert D.TensorParallelMoE(_Layer(), reduce="peer").reduce == "peer"
+    with pytest.raises(ValueError):
+        D.TensorParallelMoE(_Layer(), reduce="ring")

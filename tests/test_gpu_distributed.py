@@ -3,6 +3,8 @@ runs (its experts' weights only, the received rows' local ids with other ranks' 
 sentinel that the masked sort drops) against the oracle's partial outputs, for every rank of
 a four-way split, and the one-rank expert- and tensor-parallel layers against the oracle. The
 collectives between ranks are tested with gloo ranks on the CPU."""
+import dataclasses
+
 import pytest
 import torch
 
@@ -58,3 +60,123 @@ def test_one_rank_expert_and_tensor_parallel_layers_match_the_oracle():
     tp = D.TensorParallelMoE(MoELayer(cfg, DEV).load_synthetic_weights())
     out = tp.forward(*args)
     assert_moe_close(out, ref)
+
+
+# ---------------------------------------------------------------- combine fused with the TP all-reduce
+TPCFG = I.MoEConfig("tp_t300_h1024_e16", T=300, H=1024, E=16, G=4, TG=2, K=4, I=1024, seed=7)
+
+
+def _rank_partials_and_workspaces(shards, args):
+    """Each shard's combined partial (the fused call's own combine) and then its pairs-call
+    workspace (the same pair rows, left uncombined)."""
+    partials = [sh.forward(*args).clone() for sh in shards]
+    workspaces = [sh.forward_pairs(*args) for sh in shards]
+    return partials, workspaces
+
+
+@pytest.mark.parametrize("n", [2, 4, 8])
+def test_emulated_tp_combine_allreduce_is_the_rank_order_sum_of_the_partials(n):
+    """Every rank of the fused combine + all-reduce on one GPU (one cooperative launch, each
+    rank's CTAs running the one-rank code through the shared flags): every rank's output must
+    equal, bit for bit, bf16 of the fp32 sum in rank order of the ranks' bf16 partials (each
+    the fused call's own combine of that rank's pair rows), over three calls (epochs) whose
+    inputs alternate; and the result must match the whole layer's oracle."""
+    cfg = TPCFG
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [layer.tp_shard(r, n) for r in range(n)]
+    emu = D.EmulatedTpAllReduce(cfg.T, cfg.H, n, DEV)
+    sets = []
+    for seed in (cfg.seed, cfg.seed + 50):
+        act = I.moe_activations(dataclasses.replace(cfg, seed=seed))
+        sets.append((act, (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))))
+    for call in range(3):
+        act, args = sets[call % 2]
+        partials, workspaces = _rank_partials_and_workspaces(shards, args)
+        outs = emu(workspaces, shards[0].sorted.capacity, cfg.K, cfg.I // n)
+        torch.cuda.synchronize()
+        want = partials[0].float()
+        for p in partials[1:]:
+            want = want + p.float()
+        want = want.to(torch.bfloat16)
+        for r in range(n):
+            assert torch.equal(outs[r], want), f"call {call}, rank {r}"
+        if call < 2:
+            ref, _, _ = oracle_moe_rows(cfg, act, None)
+            assert_moe_close(outs[0], ref)
+    assert emu.epoch == 3
+
+
+def test_tp_combine_allreduce_bounded_wait_runs_out_without_its_peer():
+    """Failure handling without a fault: rank 0 of 2 launched alone (rank 1's buffers are
+    local stand-ins that nothing else touches) waits for rank 1's flags, which nothing sets;
+    each bounded wait expires (about 2 s), FP8MOE_DEVERR_TIMEOUT is raised and the kernel
+    ends; the context stays usable."""
+    cfg = TPCFG
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shard = layer.tp_shard(0, 2)
+    act = I.moe_activations(cfg)
+    ws = shard.forward_pairs(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    Ts = -(-cfg.T // 2)
+    recv = [torch.empty(2, Ts, cfg.H, dtype=torch.bfloat16, device=DEV) for _ in range(2)]
+    out = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=DEV) for _ in range(2)]
+    flags = [torch.zeros(B.TP_FLAG_WORDS, dtype=torch.int64, device=DEV) for _ in range(2)]
+    barrier = torch.zeros(B.TP_BARRIER_WORDS, dtype=torch.int64, device=DEV)
+    B.moe_combine_allreduce(ws, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I // 2, 0, recv, out, flags,
+                            barrier, 1)
+    assert B.device_status() & 1                       # FP8MOE_DEVERR_TIMEOUT (read and cleared)
+    assert B.device_status() == 0
+    assert int(flags[1][0]) == 1 and int(flags[0][0]) == 1    # rank 0 published its partials to both
+    got = layer.forward(act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    ref, _, _ = oracle_moe_rows(cfg, act, None)
+    assert_moe_close(got, ref)                         # the context is intact
+
+
+def test_tp_combine_allreduce_rejects_bad_arguments():
+    cfg = TPCFG
+    shard = MoELayer(cfg, DEV).tp_shard(0, 1)
+    t = torch.zeros(16, dtype=torch.int64, device=DEV)
+    buf = torch.zeros(1 << 20, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(B.Fp8MoeError):                 # epoch 0
+        B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I, 0, [buf], [buf],
+                                [t], t, 0)
+    with pytest.raises(B.Fp8MoeError):                 # rank outside [0, nranks)
+        B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I, 1, [buf], [buf],
+                                [t], t, 1)
+    with pytest.raises(ValueError):                    # more ranks than the protocol takes
+        B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I, 0, [buf] * 9,
+                                [buf] * 9, [t] * 9, t, 1)
+    assert B.device_status() == 0
+
+
+def test_one_rank_peer_all_reduce_through_symmetric_memory():
+    """The multi-GPU form's host side on a one-rank NCCL group: the buffers come from torch's
+    symmetric memory and the pointers from its rendezvous; with one rank the fused combine +
+    all-reduce is the combine, so the output equals the layer's own bit for bit."""
+    import gc
+    import os
+    import socket
+
+    import torch.distributed as dist
+    cfg = TPCFG
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device(DEV, 0))
+    try:
+        layer = MoELayer(cfg, DEV).load_synthetic_weights()
+        act = I.moe_activations(cfg)
+        args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+        want = layer.forward(*args).clone()
+        tp = D.TensorParallelMoE(layer, reduce="peer")
+        for _ in range(2):
+            got = tp.forward(*args)
+            torch.cuda.synchronize()
+            assert torch.equal(got, want)
+        assert tp.peer.epoch == 2
+        del tp, got
+        gc.collect()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
