@@ -637,6 +637,85 @@ def run_distributed(args, world, rank, local):
     }
 
 
+def run_tp_emulated(args, local):
+    """prefill_tp with --tp-emulate N on one GPU: the N tensor-parallel ranks' forwards one
+    after another, each without its combine (fused_moe_fp8_blockscale_g1u1_pairs), then their
+    combine fused with the all-reduce as one cooperative launch (moe_combine_allreduce_emulated),
+    every rank's CTAs running the one-rank code. A step is all N ranks' work on one GPU, so the
+    line is no multi-GPU number; what it measures is the fused all-reduce kernel against the
+    HBM copy rate (its stores stay in this GPU's memory)."""
+    from fp8_block_scaled_biased_b200 import binding as B
+    from fp8_block_scaled_biased_b200 import distributed as D
+    from fp8_block_scaled_biased_b200.layer import MoELayer
+
+    n = args.tp_emulate
+    cfg = DIST_WORKLOADS["prefill_tp"]
+    dev = torch.device("cuda", local)
+    act = I.moe_activations(cfg)
+    logits, bias, x = act.logits.to(dev), act.bias.to(dev), act.x.to(dev)
+    full = MoELayer(cfg, dev).load_synthetic_weights()
+    shards = [full.tp_shard(r, n) for r in range(n)]
+    del full
+    torch.cuda.empty_cache()
+    emu = D.EmulatedTpAllReduce(cfg.T, cfg.H, n, dev)
+    cap, Is = shards[0].sorted.capacity, cfg.I // n
+    stream = torch.cuda.current_stream()
+
+    def step(mid=None):
+        ws = [sh.forward_pairs(logits, bias, x) for sh in shards]
+        if mid is not None:
+            mid.record(stream)
+        return emu(ws, cap, cfg.K, Is)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert B.device_status() == 0, "device error word set during warm-up"
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    for i in range(DIST_PREHEAT_STEPS // 10):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step(ev[i][1])
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if B.device_status():
+        raise RuntimeError("device error word set during the timed steps")
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    ar_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    ms_per_step = sum(step_ms) / args.steps
+    ar = sum(ar_ms) / args.steps
+    # per rank: its pair rows read (T*K*H bf16), its partial rows stored (T*H), its slice's n
+    # partials read (~T*H) and the reduced slice stored into n outputs (~T*H)
+    ar_bytes = n * cfg.T * cfg.H * 2 * (cfg.K + 3)
+    hbm = load_peaks()["hbm_gbs"]
+    return {
+        "metric": METRIC, "value": cfg.T / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "none (all ranks on one GPU)", "vs_baseline": None,
+        "dtype": "fp8_e4m3fn x fp8_e4m3fn -> fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded; random-init weights quantised to FP8 in 128x128 blocks)",
+        "config": {"workload": f"{cfg.name}_tp{n}_emulated_on_1_gpu", "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                   "topk": cfg.K, "I": cfg.I, "parallelism": f"tp{n} emulated: the {n} ranks' forwards in turn on "
+                   "one GPU, then their fused combine + all-reduce as one cooperative launch",
+                   "l2": "flushed between steps (256 MB write)", "cuda_graph": False},
+        "allreduce": {"kernel": "tp_combine_allreduce_kernel", "bound": "hbm", "ms": ar,
+                      "bytes": ar_bytes, "achieved": ar_bytes / (ar * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                      "frac": ar_bytes / (ar * 1e-3) / 1e9 / hbm, "peak_source": "measured",
+                      "note": "CUDA events around the emulated launch; the ranks' stores stay in this GPU's memory"},
+        "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
+        "gpu_launches": None, "clocks": clocks,
+    }
+
+
 def workload_config(args):
     """The MoE workload's configuration; with --tokens T, the same recipe (shapes, routing,
     value distributions, seed) at T tokens: one point of a batch-size sweep."""
@@ -650,6 +729,8 @@ def run_ours(args, world, rank, local):
     from fp8_block_scaled_biased_b200.layer import MoELayer
 
     if args.workload in DIST_WORKLOADS:
+        if args.tp_emulate:
+            return run_tp_emulated(args, local)
         return run_distributed(args, world, rank, local)
     cfg = workload_config(args)
     dev = torch.device("cuda", local)
@@ -898,6 +979,9 @@ def main():
     ap.add_argument("--tp-reduce", choices=["peer", "nccl"], default="peer",
                     help="prefill_tp: sum the ranks' partials with the combine fused with the all-reduce over "
                          "peer memory (peer) or with NCCL's reduce-scatter and all-gather (nccl)")
+    ap.add_argument("--tp-emulate", type=int, default=0,
+                    help="prefill_tp on one GPU: run all N ranks there, their fused combine + all-reduce as one "
+                         "launch (a kernel measurement, not a multi-GPU number)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -914,6 +998,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.tokens is not None and (args.tokens < 1 or args.workload not in WORKLOADS):
         ap.error("--tokens takes a positive count and a single-GPU MoE workload")
+    if args.tp_emulate and (args.workload != "prefill_tp" or args.gpus != 1 or not 2 <= args.tp_emulate <= 8
+                            or DIST_WORKLOADS["prefill_tp"].I % (128 * args.tp_emulate)):
+        ap.error("--tp-emulate takes 2..8 ranks that split I into 128-column blocks, with prefill_tp on one GPU")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

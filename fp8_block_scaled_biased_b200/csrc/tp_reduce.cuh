@@ -41,6 +41,7 @@ namespace fp8moe {
 constexpr int kTpMaxRanks = 8;
 constexpr int kTpThreads = 256;
 constexpr int kTpFlagWords = 2 * kTpMaxRanks;   // per rank: [phase][source rank]
+constexpr int kTpBatch = 4;                      // pair rows loaded before they are added
 
 struct TpArgs {
   // per rank, in that rank's GPU memory (only [rank] is read by a one-rank launch)
@@ -153,9 +154,22 @@ tp_combine_allreduce_kernel(const __grid_constant__ TpArgs a, int rank_first, in
 #pragma unroll
     for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
     const __nv_bfloat16* row = y + static_cast<size_t>(t) * K * H + c;
-    for (int k = 0; k < K; ++k)
-      if (all_present || flag[static_cast<size_t>(t) * K + k])
-        add_bf16x8(acc, __ldcs(reinterpret_cast<const uint4*>(row + static_cast<size_t>(k) * H)));
+    if (all_present) {
+      // up to kTpBatch rows in flight per thread, then added in k order
+      for (int k0 = 0; k0 < K; k0 += kTpBatch) {
+        uint4 v[kTpBatch];
+#pragma unroll
+        for (int j = 0; j < kTpBatch; ++j)
+          if (k0 + j < K) v[j] = __ldcs(reinterpret_cast<const uint4*>(row + static_cast<size_t>(k0 + j) * H));
+#pragma unroll
+        for (int j = 0; j < kTpBatch; ++j)
+          if (k0 + j < K) add_bf16x8(acc, v[j]);
+      }
+    } else {
+      for (int k = 0; k < K; ++k)
+        if (flag[static_cast<size_t>(t) * K + k])
+          add_bf16x8(acc, __ldcs(reinterpret_cast<const uint4*>(row + static_cast<size_t>(k) * H)));
+    }
     const int p = t / Ts;
     __nv_bfloat16* dst = a.recv[p] + (static_cast<size_t>(rank) * Ts + (t - p * Ts)) * H + c;
     *reinterpret_cast<uint4*>(dst) = pack_bf16x8(acc);
@@ -178,8 +192,15 @@ tp_combine_allreduce_kernel(const __grid_constant__ TpArgs a, int rank_first, in
     float acc[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
-    for (int q = 0; q < n; ++q)
-      add_bf16x8(acc, *reinterpret_cast<const uint4*>(mine + (static_cast<size_t>(q) * Ts + r) * H + c));
+    // the n partials in flight together, read at L2 (other ranks wrote them during this
+    // kernel), then added in rank order
+    uint4 part[kTpMaxRanks];
+#pragma unroll
+    for (int q = 0; q < kTpMaxRanks; ++q)
+      if (q < n) part[q] = __ldcg(reinterpret_cast<const uint4*>(mine + (static_cast<size_t>(q) * Ts + r) * H + c));
+#pragma unroll
+    for (int q = 0; q < kTpMaxRanks; ++q)
+      if (q < n) add_bf16x8(acc, part[q]);
     const uint4 v = pack_bf16x8(acc);
     for (int p = 0; p < n; ++p)
       *reinterpret_cast<uint4*>(a.out[p] + static_cast<size_t>(t0 + r) * H + c) = v;

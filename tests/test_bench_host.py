@@ -146,3 +146,12 @@ def test_tokens_option_keeps_the_recipe_at_another_batch_size():
     bad = subprocess.run([sys.executable, "bench.py", "--workload", "gemm", "--tokens", "3"], cwd=ROOT,
                          capture_output=True, text=True, timeout=600)
     assert bad.returncode != 0 and "--tokens" in bad.stderr
+
+
+def test_tp_emulate_option_is_checked():
+    """--tp-emulate runs the tensor-parallel workload's ranks on one GPU; it takes 2..8 ranks
+    that split I into whole 128-column blocks, and only the prefill_tp workload."""
+    for bad in (["--workload", "prefill", "--tp-emulate", "8"], ["--workload", "prefill_tp", "--tp-emulate", "9"],
+                ["--workload", "prefill_tp", "--tp-emulate", "1"], ["--workload", "prefill_tp", "--tp-emulate", "3"]):
+        r = subprocess.run([sys.executable, "bench.py", *bad], cwd=ROOT, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0 and "--tp-emulate" in r.stderr, bad
