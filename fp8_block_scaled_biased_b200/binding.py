@@ -60,6 +60,14 @@ _SIGNATURES = {
                                        ctypes.c_uint64, _p]),
     "moe_combine_allreduce_emulated": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p,
                                                 ctypes.c_uint64, _p]),
+    "moe_ep_routing": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p]),
+    "fused_moe_fp8_blockscale_g1u1_multi": (_c_int, [_p, _p, _c_int, _c_int, _p, _p, _p, _p, _p, _p, _c_int, _c_int,
+                                                     _c_int, _c_int, _c_int, _c_size, _p, _p, _c_int, _c_int, _p,
+                                                     _c_int, _p, _c_size, _p]),
+    "moe_ep_return": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p]),
+    "moe_ep_barrier": (_c_int, [_c_int, _c_int, _p, ctypes.c_uint64, _p]),
+    "moe_ep_barrier_emulated": (_c_int, [_c_int, _p, ctypes.c_uint64, _p]),
+    "moe_combine_pairs": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _p, _p]),
 }
 EXPORTED = tuple(_SIGNATURES)
 
@@ -67,6 +75,8 @@ NOALLOC_SCRATCH_BYTES = 64 << 20   # FP8MOE_NOALLOC_SCRATCH_BYTES in include/fp8
 TP_MAX_RANKS = 8                   # FP8MOE_TP_MAX_RANKS
 TP_FLAG_WORDS = 16                 # FP8MOE_TP_FLAG_WORDS (64-bit words per rank)
 TP_BARRIER_WORDS = 2               # FP8MOE_TP_BARRIER_WORDS
+EP_MAX_RANKS = 8                   # FP8MOE_EP_MAX_RANKS
+EP_BARRIER_WORDS = 8               # FP8MOE_EP_BARRIER_WORDS
 SCALE_ROW_MAJOR = 0
 SCALE_COL_MAJOR = 1
 FP8 = torch.float8_e4m3fn
@@ -502,3 +512,99 @@ def moe_combine_allreduce_emulated(workspaces, capacity, T, topk, H, I, recv, ou
         _addresses(workspaces, "workspaces"), capacity, T, topk, H, I, n, _addresses(recv, "recv"),
         _addresses(out, "out"), _addresses(flags, "flags"), _addresses(barriers, "barriers"), epoch, _stream())
     _check("moe_combine_allreduce_emulated", rc)
+
+
+# ---------------------------------------------------------------- expert parallelism over peer memory
+def moe_ep_routing(ids, w, Tq, topk, E, e0, ne, ids_out, w_out):
+    """Every rank's routing as this owner's local ids (include/fp8moe.h). ids, w: one device
+    address (or tensor) per rank; ids_out int32 / w_out fp32 [n*Tq, topk] on this GPU."""
+    n = len(ids)
+    if len(w) != n or not 1 <= n <= EP_MAX_RANKS:
+        raise ValueError("one ids and one weights buffer per rank (at most EP_MAX_RANKS)")
+    _cuda(ids_out, torch.int32, "ids_out")
+    _cuda(w_out, torch.float32, "w_out")
+    if ids_out.numel() < n * Tq * topk or w_out.numel() < n * Tq * topk:
+        raise ValueError("ids_out / w_out smaller than n*Tq*topk")
+    rc = load_library().moe_ep_routing(_addresses(ids, "ids"), _addresses(w, "w"), n, Tq, topk, E, e0, ne,
+                                       _ptr(ids_out), _ptr(w_out), _stream())
+    _check("moe_ep_routing", rc)
+
+
+def fused_moe_fp8_blockscale_g1u1_multi(a8, a1_scale, Tq, H, w1, w2, sorted_pairs: SortedPairs, topk, fc1_scale,
+                                        fc2_scale, workspace=None):
+    """The owner's fused MoE over every rank's tokens (without the combine): a8[q] fp8 [Tq, H]
+    and a1_scale[q] fp32 [H/128, Tq] of rank q, as addresses or tensors; the owner's weights;
+    the sort over n*Tq tokens. Returns the workspace holding the weighted pair rows."""
+    n = len(a8)
+    if len(a1_scale) != n or not 1 <= n <= EP_MAX_RANKS:
+        raise ValueError("one activation and one scale buffer per rank (at most EP_MAX_RANKS)")
+    for name, t in (("w1", w1), ("w2", w2)):
+        _cuda(t, FP8, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    E, twoI, H1 = _expert_matrix_shape(w1)
+    E2, H2, I = _expert_matrix_shape(w2)
+    if is_tiled(w1) != is_tiled(w2) or twoI != 2 * I or H1 != H or (E2, H2) != (E, H) or H % 128 or I % 128:
+        raise ValueError(f"w1 {tuple(w1.shape)} and w2 {tuple(w2.shape)} do not form a g1u1 pair for H={H}")
+    for name, t, shape in (("fc1_scale", fc1_scale, (E, 2 * I // 128, H // 128)),
+                           ("fc2_scale", fc2_scale, (E, H // 128, I // 128))):
+        _cuda(t, torch.float32, name)
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {shape}")
+    sp = sorted_pairs
+    for name, t, dt in (("sorted_ids", sp.sorted_ids, torch.int32), ("sorted_weights", sp.sorted_weights, torch.float32),
+                        ("sorted_expert_ids", sp.sorted_expert_ids, torch.int32),
+                        ("num_valid_ids", sp.num_valid_ids, torch.int32)):
+        _cuda(t, dt, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if workspace is None:
+        need = fused_moe_workspace_bytes(n * Tq, topk, E, H, I, sp.block_m, capacity=sp.capacity)
+        workspace = torch.empty(need, dtype=torch.uint8, device=w1.device)
+    rc = load_library().fused_moe_fp8_blockscale_g1u1_multi(
+        _addresses(a8, "a8"), _addresses(a1_scale, "a1_scale"), n, Tq, _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids),
+        _ptr(sp.sorted_weights), _ptr(sp.sorted_expert_ids), _ptr(sp.num_valid_ids), H, I, E, topk, sp.block_m,
+        sp.capacity, _ptr(fc1_scale), _ptr(fc2_scale), 128, 128, None, 1 if is_tiled(w1) else 0, _ptr(workspace),
+        workspace.numel(), _stream())
+    _check("fused_moe_fp8_blockscale_g1u1_multi", rc)
+    return workspace
+
+
+def moe_ep_return(workspace, capacity, Tq, topk, H, I, sorted_pairs: SortedPairs, rows, pair_flags):
+    """Each listed pair's weighted row into its origin's return rows, its flag set. rows,
+    pair_flags: one address (or tensor) per rank."""
+    n = len(rows)
+    if len(pair_flags) != n or not 1 <= n <= EP_MAX_RANKS:
+        raise ValueError("one rows and one flags buffer per rank (at most EP_MAX_RANKS)")
+    _cuda(workspace, torch.uint8, "workspace")
+    sp = sorted_pairs
+    rc = load_library().moe_ep_return(_ptr(workspace), capacity, n, Tq, topk, H, I, _ptr(sp.sorted_ids),
+                                      _ptr(sp.num_valid_ids), _addresses(rows, "rows"),
+                                      _addresses(pair_flags, "pair_flags"), _stream())
+    _check("moe_ep_return", rc)
+
+
+def moe_ep_barrier(rank, words, epoch):
+    """Flag barrier of len(words) ranks (include/fp8moe.h); words: one address (or int64
+    tensor of EP_BARRIER_WORDS) per rank."""
+    rc = load_library().moe_ep_barrier(len(words), rank, _addresses(words, "words"), epoch, _stream())
+    _check("moe_ep_barrier", rc)
+
+
+def moe_ep_barrier_emulated(words, epoch):
+    rc = load_library().moe_ep_barrier_emulated(len(words), _addresses(words, "words"), epoch, _stream())
+    _check("moe_ep_barrier_emulated", rc)
+
+
+def moe_combine_pairs(rows, flag_region, T, topk, out):
+    """out bf16 [T, H] = the combine over pair rows bf16 [T*topk, H] and their flag region
+    (16-byte count, then one flag byte per pair)."""
+    _cuda(rows, torch.bfloat16, "rows")
+    _cuda(flag_region, torch.uint8, "flag_region")
+    _cuda(out, torch.bfloat16, "out")
+    H = out.shape[-1]
+    if rows.numel() < T * topk * H or flag_region.numel() < 16 + T * topk or out.numel() < T * H:
+        raise ValueError("rows, flag_region or out smaller than the call needs")
+    rc = load_library().moe_combine_pairs(_ptr(rows), _ptr(flag_region), T, topk, H, _ptr(out), _stream())
+    _check("moe_combine_pairs", rc)
+    return out

@@ -18,6 +18,7 @@
 #include "route.cuh"
 #include "sort.cuh"
 #include "tp_reduce.cuh"
+#include "ep_peer.cuh"
 
 static_assert(fp8moe::kMoeBlockRows == fp8moe::kBM, "sorted blocks are GEMM tiles");
 
@@ -510,21 +511,24 @@ size_t fused_moe_fp8_blockscale_g1u1_workspace(int T, int topk, int E, int H, in
 
 // The fused MoE call on row-major (tiled == false) or tiled (fp8_tile_weights) weights;
 // with combine == false it stops after the down GEMM (the weighted pair rows and the
-// pair flags stay in the workspace) and out is not used.
+// pair flags stay in the workspace) and out is not used. With srcs, the activation
+// rows and scales are gathered from several sources (a8 and a1_scale unused; T is the
+// sources' tokens together).
 static int fused_moe_impl(const char* name, bool tiled, bool combine, uint16_t* out, const uint8_t* a8,
                           const uint8_t* w1,
                           const uint8_t* w2, const int32_t* sorted_ids, const float* sorted_weights,
                           const int32_t* sorted_expert_ids, const int32_t* num_valid_ids, int T, int H, int I, int E,
                           int topk, int block_m, size_t capacity, const float* a1_scale, const float* fc1_scale,
                           const float* fc2_scale, int scale_blk_n, int scale_blk_k, const float* fc2_smooth_scale,
-                          void* workspace, size_t workspace_bytes, void* stream) {
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          const GatherSources* srcs = nullptr) {
   (void)name;
   if (scale_blk_n != 128 || scale_blk_k != 128)
     return fail(FP8MOE_EUNSUPPORTED, "only (128, 128) scale blocks are supported (got %d, %d)", scale_blk_n,
                 scale_blk_k);
   if (fc2_smooth_scale) return fail(FP8MOE_EUNSUPPORTED, "fc2_smooth_scale must be NULL");
   if (block_m != kBM) return fail(FP8MOE_EUNSUPPORTED, "block_m must be %d (got %d)", kBM, block_m);
-  if (T < 0 || E < 1 || topk < 1 || topk > E) return fail(FP8MOE_EINVAL, "bad T, E or topk");
+  if (T < 0 || E < 1 || topk < 1) return fail(FP8MOE_EINVAL, "bad T, E or topk");
   if (topk > 32) return fail(FP8MOE_EUNSUPPORTED, "topk must be <= 32 (got %d)", topk);
   if (H < 128 || I < 128 || H % 128 || I % 128)
     return fail(FP8MOE_EUNSUPPORTED, "H and I must be positive multiples of 128 (H=%d, I=%d)", H, I);
@@ -533,8 +537,8 @@ static int fused_moe_impl(const char* name, bool tiled, bool combine, uint16_t* 
     return fail(FP8MOE_EINVAL, "capacity %zu below the sort's bound %zu", capacity,
                 moe_align_sort_capacity(T, topk, E, block_m));
   if (T == 0) return FP8MOE_OK;
-  if ((combine && !out) || !a8 || !w1 || !w2 || !sorted_ids || !sorted_weights || !sorted_expert_ids || !num_valid_ids ||
-      !a1_scale || !fc1_scale || !fc2_scale)
+  if ((combine && !out) || (!srcs && (!a8 || !a1_scale)) || !w1 || !w2 || !sorted_ids || !sorted_weights ||
+      !sorted_expert_ids || !num_valid_ids || !fc1_scale || !fc2_scale)
     return fail(FP8MOE_EINVAL, "null pointer argument");
   if (!aligned16(a8) || !aligned16(w1) || !aligned16(w2) || !aligned16(sorted_ids) || !aligned16(out))
     return fail(FP8MOE_EINVAL, "a8, w1, w2, sorted_ids and out must be 16-byte aligned");
@@ -576,11 +580,20 @@ static int fused_moe_impl(const char* name, bool tiled, bool combine, uint16_t* 
   // pair -> slot map of the gather, kept in the pair-row region (P * 4 <= P * H * 2
   // bytes) that the down GEMM writes only later
   int* inv = reinterpret_cast<int*>(ystage);
-  moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a1_scale, sorted_ids, sorted_expert_ids, num_valid_ids,
-                                                            T, topk, H, static_cast<int>(capacity), s1s, pair_flag,
-                                                            n_present, inv);
-  if (int rc = check_launch("fused_moe (gather)")) return rc;
-  moe_gather_rows_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, T, topk, H, pair_flag, inv, a8s);
+  if (srcs) {
+    moe_gather_kernel<true><<<sms * 4, 32 * kGatherWarps, 0, st>>>(
+        nullptr, sorted_ids, sorted_expert_ids, num_valid_ids, T, topk, H, static_cast<int>(capacity), s1s,
+        pair_flag, n_present, inv, *srcs);
+    if (int rc = check_launch("fused_moe (gather)")) return rc;
+    moe_gather_rows_kernel<true><<<sms * 4, 32 * kGatherWarps, 0, st>>>(nullptr, T, topk, H, pair_flag, inv, a8s,
+                                                                       *srcs);
+  } else {
+    moe_gather_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a1_scale, sorted_ids, sorted_expert_ids, num_valid_ids,
+                                                              T, topk, H, static_cast<int>(capacity), s1s, pair_flag,
+                                                              n_present, inv);
+    if (int rc = check_launch("fused_moe (gather)")) return rc;
+    moe_gather_rows_kernel<<<sms * 4, 32 * kGatherWarps, 0, st>>>(a8, T, topk, H, pair_flag, inv, a8s);
+  }
   if (int rc = check_launch("fused_moe (gather rows)")) return rc;
   timing_record(1, st);
 
@@ -869,6 +882,138 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
                         recv, out, flags, barriers, epoch, &a, &ctas))
     return rc;
   return tp_launch("moe_combine_allreduce_emulated", a, 0, ctas, nranks, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ expert-parallel dispatch and return
+static_assert(FP8MOE_EP_MAX_RANKS == kMaxSources && FP8MOE_EP_BARRIER_WORDS == kMaxSources, "header and kernels agree");
+
+extern "C" {
+
+int moe_ep_routing(const int32_t* const* ids, const float* const* w, int n, int Tq, int topk, int E, int e0, int ne,
+                   int32_t* ids_out, float* w_out, void* stream) {
+  if (n < 1 || n > kMaxSources) return fail(FP8MOE_EINVAL, "moe_ep_routing: n must be in [1, %d]", kMaxSources);
+  if (Tq < 0 || topk < 1 || E < 1 || ne < 1 || e0 < 0 || e0 + ne > E)
+    return fail(FP8MOE_EINVAL, "moe_ep_routing: bad sizes (Tq=%d, topk=%d, E=%d, e0=%d, ne=%d)", Tq, topk, E, e0, ne);
+  if (static_cast<long long>(Tq) * topk * n >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "moe_ep_routing: too many pairs");
+  if (Tq == 0) return FP8MOE_OK;
+  if (!ids || !w || !ids_out || !w_out) return fail(FP8MOE_EINVAL, "moe_ep_routing: null pointer argument");
+  EpRouting src{};
+  for (int q = 0; q < n; ++q) {
+    if (!ids[q] || !w[q]) return fail(FP8MOE_EINVAL, "moe_ep_routing: null routing of rank %d", q);
+    src.ids[q] = ids[q];
+    src.w[q] = w[q];
+  }
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  const long long total = static_cast<long long>(Tq) * topk * n;
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4ll * sms));
+  ep_routing_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(src, n, Tq, topk, E, e0, ne, ids_out,
+                                                                           w_out);
+  return check_launch("moe_ep_routing");
+}
+
+int fused_moe_fp8_blockscale_g1u1_multi(const uint8_t* const* a8, const float* const* a1_scale, int n, int Tq,
+                                        const uint8_t* w1, const uint8_t* w2, const int32_t* sorted_ids,
+                                        const float* sorted_weights, const int32_t* sorted_expert_ids,
+                                        const int32_t* num_valid_ids, int H, int I, int E, int topk, int block_m,
+                                        size_t capacity, const float* fc1_scale, const float* fc2_scale,
+                                        int scale_blk_n, int scale_blk_k, const float* fc2_smooth_scale,
+                                        int weights_tiled, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n < 1 || n > kMaxSources) return fail(FP8MOE_EINVAL, "n must be in [1, %d]", kMaxSources);
+  if (Tq < 0 || static_cast<long long>(Tq) * n >= (1ll << 31)) return fail(FP8MOE_EINVAL, "bad Tq");
+  if (!a8 || !a1_scale) return fail(FP8MOE_EINVAL, "null pointer argument");
+  GatherSources srcs{};
+  for (int q = 0; q < n; ++q) {
+    if (!a8[q] || !a1_scale[q]) return fail(FP8MOE_EINVAL, "null activations of source %d", q);
+    if (!aligned16(a8[q])) return fail(FP8MOE_EINVAL, "activations of source %d must be 16-byte aligned", q);
+    srcs.a8[q] = a8[q];
+    srcs.a1_scale[q] = a1_scale[q];
+  }
+  srcs.n = n;
+  srcs.Tq = Tq;
+  return fused_moe_impl("fused_moe_fp8_blockscale_g1u1_multi", weights_tiled != 0, false, nullptr, nullptr, w1, w2,
+                        sorted_ids, sorted_weights, sorted_expert_ids, num_valid_ids, n * Tq, H, I, E, topk, block_m,
+                        capacity, nullptr, fc1_scale, fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, workspace,
+                        workspace_bytes, stream, &srcs);
+}
+
+int moe_ep_return(const void* workspace, size_t capacity, int n, int Tq, int topk, int H, int I,
+                  const int32_t* sorted_ids, const int32_t* num_valid_ids, void* const* rows, void* const* pair_flags,
+                  void* stream) {
+  if (n < 1 || n > kMaxSources) return fail(FP8MOE_EINVAL, "moe_ep_return: n must be in [1, %d]", kMaxSources);
+  if (Tq < 0 || topk < 1 || H < 128 || H % 128 || I < 128 || I % 128 || capacity >= (1ull << 31))
+    return fail(FP8MOE_EINVAL, "moe_ep_return: bad sizes");
+  if (static_cast<long long>(Tq) * topk * n >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "moe_ep_return: too many pairs");
+  if (Tq == 0) return FP8MOE_OK;
+  if (!workspace || !sorted_ids || !num_valid_ids || !rows || !pair_flags)
+    return fail(FP8MOE_EINVAL, "moe_ep_return: null pointer argument");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(FP8MOE_EINVAL, "moe_ep_return: workspace alignment");
+  EpReturn dst{};
+  for (int q = 0; q < n; ++q) {
+    if (!rows[q] || !pair_flags[q]) return fail(FP8MOE_EINVAL, "moe_ep_return: null buffer of rank %d", q);
+    if (!aligned16(rows[q])) return fail(FP8MOE_EINVAL, "moe_ep_return: rows of rank %d must be 16-byte aligned", q);
+    dst.rows[q] = static_cast<__nv_bfloat16*>(rows[q]);
+    dst.flags[q] = static_cast<uint8_t*>(pair_flags[q]);
+  }
+  const MoeWorkspace lay = moe_workspace_layout(capacity, n * Tq, topk, H, I);
+  const auto* ystage = reinterpret_cast<const __nv_bfloat16*>(static_cast<const uint8_t*>(workspace) + lay.y_off);
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  ep_return_kernel<<<sms * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      sorted_ids, num_valid_ids, static_cast<int>(capacity), ystage, n, Tq * topk, H, dst);
+  return check_launch("moe_ep_return");
+}
+
+static int ep_barrier_launch(const char* name, int n, int rank_first, int ctas, uint64_t* const* words, uint64_t epoch,
+                             void* stream) {
+  if (n < 1 || n > kMaxSources) return fail(FP8MOE_EINVAL, "%s: n must be in [1, %d]", name, kMaxSources);
+  if (epoch == 0) return fail(FP8MOE_EINVAL, "%s: epoch must be >= 1", name);
+  if (!words) return fail(FP8MOE_EINVAL, "%s: null pointer argument", name);
+  EpBarrierArgs a{};
+  for (int p = 0; p < n; ++p) {
+    if (!words[p] || (reinterpret_cast<uintptr_t>(words[p]) & 7u))
+      return fail(FP8MOE_EINVAL, "%s: barrier words of rank %d null or not 8-byte aligned", name, p);
+    a.flags[p] = reinterpret_cast<unsigned long long*>(words[p]);
+  }
+  a.n = n;
+  a.epoch = epoch;
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  void* args[] = {&a, &rank_first};
+  const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(ep_barrier_kernel), dim3(ctas),
+                                                    dim3(32), args, 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FP8MOE_ECUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+  }
+  return check_launch(name);
+}
+
+int moe_ep_barrier(int n, int rank, uint64_t* const* words, uint64_t epoch, void* stream) {
+  if (rank < 0 || rank >= n) return fail(FP8MOE_EINVAL, "moe_ep_barrier: bad rank");
+  return ep_barrier_launch("moe_ep_barrier", n, rank, 1, words, epoch, stream);
+}
+
+int moe_ep_barrier_emulated(int n, uint64_t* const* words, uint64_t epoch, void* stream) {
+  return ep_barrier_launch("moe_ep_barrier_emulated", n, 0, n, words, epoch, stream);
+}
+
+int moe_combine_pairs(const uint16_t* rows, const void* flag_region, int T, int topk, int H, uint16_t* out,
+                      void* stream) {
+  if (T < 0 || topk < 1 || topk > 32 || H < 8 || H % 8) return fail(FP8MOE_EINVAL, "moe_combine_pairs: bad sizes");
+  if (static_cast<long long>(T) * topk >= (1ll << 31)) return fail(FP8MOE_EUNSUPPORTED, "moe_combine_pairs: T too large");
+  if (T == 0) return FP8MOE_OK;
+  if (!rows || !flag_region || !out) return fail(FP8MOE_EINVAL, "moe_combine_pairs: null pointer argument");
+  if (!aligned16(rows) || !aligned16(out) || (reinterpret_cast<uintptr_t>(flag_region) & 15u))
+    return fail(FP8MOE_EINVAL, "moe_combine_pairs: rows, out and the flag region must be 16-byte aligned");
+  const int* count = static_cast<const int*>(flag_region);
+  const uint8_t* flags = static_cast<const uint8_t*>(flag_region) + 16;
+  const size_t threads = static_cast<size_t>(T) * (H / 8);
+  moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(rows), flags, count, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
+  return check_launch("moe_combine_pairs");
 }
 
 }  // extern "C"

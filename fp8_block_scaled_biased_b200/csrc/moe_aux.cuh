@@ -18,6 +18,17 @@ namespace fp8moe {
 constexpr int kMoeBlockRows = 128;            // rows per sorted block (the GEMM tile's M)
 
 constexpr int kGatherWarps = 8;
+
+// The activations of several GPUs' tokens, read where they lie (expert parallelism:
+// the GPU that owns an expert gathers the rows of every GPU's tokens routed to it).
+// Global token g is token g % Tq of source g / Tq; the pointers are as this GPU
+// addresses each source's memory (peer memory over NVLink, or local).
+constexpr int kMaxSources = 8;
+struct GatherSources {
+  const uint8_t* a8[kMaxSources];        // fp8 [Tq, H]
+  const float* a1_scale[kMaxSources];    // fp32 [H/128, Tq]
+  int n, Tq;
+};
 // Slot-ordered pass over the sorted list: sets pair_flag[p] = 1 for every listed
 // pair p and adds the number of distinct listed pairs to *n_present (the caller
 // zeroes both first; pair_flag is 4-byte aligned; a pair id listed twice, which
@@ -26,11 +37,14 @@ constexpr int kGatherWarps = 8;
 // flag is set) and copies each slot's H/128 scales from a1_scale [H/128, T] into
 // slot order. Padding slots are skipped: the GEMMs treat rows independently and
 // never store padding rows.
+// MULTI: the scales of token t come from its source (src), not from a1_scale.
+template <bool MULTI = false>
 __global__ void __launch_bounds__(32 * kGatherWarps)
 moe_gather_kernel(const float* __restrict__ a1_scale, const int32_t* __restrict__ sorted_ids,
                   const int32_t* __restrict__ sorted_expert_ids, const int32_t* __restrict__ num_valid_ids, int T,
                   int topk, int H, int cap, float* __restrict__ s1s, uint8_t* __restrict__ pair_flag,
-                  int* __restrict__ n_present, int* __restrict__ inv) {
+                  int* __restrict__ n_present, int* __restrict__ inv,
+                  const __grid_constant__ GatherSources src = {}) {
   __shared__ int cta_present;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) cta_present = 0;
@@ -58,8 +72,15 @@ moe_gather_kernel(const float* __restrict__ a1_scale, const int32_t* __restrict_
     const int sid = slot < nv ? sorted_ids[slot] : -1;
     if (sid < 0 || sid >= P) continue;
     const int t = sid / topk;
-    for (int kb = 0; kb < KB; ++kb)
-      __stcs(&s1s[static_cast<size_t>(kb) * cap + slot], __ldg(a1_scale + static_cast<size_t>(kb) * T + t));
+    if constexpr (MULTI) {
+      const int q = t / src.Tq, lt = t - q * src.Tq;
+      const float* sc = src.a1_scale[q];
+      for (int kb = 0; kb < KB; ++kb)
+        __stcs(&s1s[static_cast<size_t>(kb) * cap + slot], __ldcg(sc + static_cast<size_t>(kb) * src.Tq + lt));
+    } else {
+      for (int kb = 0; kb < KB; ++kb)
+        __stcs(&s1s[static_cast<size_t>(kb) * cap + slot], __ldg(a1_scale + static_cast<size_t>(kb) * T + t));
+    }
   }
 }
 
@@ -70,10 +91,13 @@ moe_gather_kernel(const float* __restrict__ a1_scale, const int32_t* __restrict_
 // (so that a small batch still spreads over the GPU); stores are marked
 // evict-first.
 constexpr int kRowChunkVec = 4;               // 16-byte vectors per lane per chunk
+// MULTI: token t's row comes from its source (src), not from a8.
+template <bool MULTI = false>
 __global__ void __launch_bounds__(32 * kGatherWarps)
 moe_gather_rows_kernel(const uint8_t* __restrict__ a8, int T, int topk, int H,
                        const uint8_t* __restrict__ pair_flag, const int* __restrict__ inv,
-                       uint8_t* __restrict__ a8s) {
+                       uint8_t* __restrict__ a8s,
+                       const __grid_constant__ GatherSources src = {}) {
   const int lane = threadIdx.x & 31;
   const int vec_per_row = H / 16;
   const int chunks = (vec_per_row + 32 * kRowChunkVec - 1) / (32 * kRowChunkVec);
@@ -87,12 +111,23 @@ moe_gather_rows_kernel(const uint8_t* __restrict__ a8, int T, int topk, int H,
       const int p = t * topk + lane;
       if (pair_flag[p]) slot_k = inv[p];
     }
-    const uint4* src = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
+    if (__ballot_sync(0xffffffffu, slot_k >= 0) == 0) continue;   // no listed pair: the row is not read
     uint4 buf[kRowChunkVec];
+    if constexpr (MULTI) {
+      const int q = t / src.Tq;
+      const uint4* row = reinterpret_cast<const uint4*>(src.a8[q] + static_cast<size_t>(t - q * src.Tq) * H);
 #pragma unroll
-    for (int i = 0; i < kRowChunkVec; ++i) {
-      const int v = v0 + i * 32 + lane;
-      if (v < vec_per_row) buf[i] = __ldg(src + v);
+      for (int i = 0; i < kRowChunkVec; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < vec_per_row) buf[i] = __ldcg(row + v);
+      }
+    } else {
+      const uint4* row = reinterpret_cast<const uint4*>(a8 + static_cast<size_t>(t) * H);
+#pragma unroll
+      for (int i = 0; i < kRowChunkVec; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < vec_per_row) buf[i] = __ldg(row + v);
+      }
     }
     for (int k = 0; k < topk; ++k) {
       const int slot = __shfl_sync(0xffffffffu, slot_k, k);

@@ -353,3 +353,161 @@ class ExpertParallelMoE:
         received, plan = ep_dispatch(a8, a8_scale, ids, w, cfg.E, self.group)
         partial = self.local(*received)
         return ep_combine(partial, plan, self.group)
+
+
+# ------------------------------------------------------------------ expert parallel over peer memory
+
+@dataclasses.dataclass(frozen=True)
+class EpBufferLayout:
+    """Byte offsets of what one expert-parallel rank publishes to the others, in one
+    allocation (each part at a multiple of 256 bytes): its routing (ids int32 [T, K],
+    weights fp32 [T, K]), its activations (fp8 [T, H]) and their scales (fp32 [H/128, T]),
+    its return buffer (bf16 rows [T*K, H], then a 16-byte count and one flag byte per pair)
+    and its barrier words (int64 [EP_BARRIER_WORDS])."""
+    ids: int
+    w: int
+    a8: int
+    scale: int
+    rows: int
+    flags: int
+    barrier: int
+    total: int
+
+
+def ep_buffer_layout(T: int, K: int, H: int) -> EpBufferLayout:
+    if T < 1 or K < 1 or H < 128 or H % 128:
+        raise ValueError(f"bad expert-parallel buffer shape T={T}, K={K}, H={H}")
+    up = lambda v: -(-v // 256) * 256   # noqa: E731
+    off, parts = 0, []
+    for size in (T * K * 4, T * K * 4, T * H, (H // 128) * T * 4, T * K * H * 2, 16 + T * K, B.EP_BARRIER_WORDS * 8):
+        parts.append(off)
+        off = up(off + size)
+    return EpBufferLayout(*parts, total=off)
+
+
+class EpRankBuffers:
+    """Typed views of one rank's published buffers (a uint8 tensor laid out by
+    ep_buffer_layout) and their addresses."""
+
+    def __init__(self, buf: torch.Tensor, T: int, K: int, H: int):
+        L = ep_buffer_layout(T, K, H)
+        self.layout, self.buf = L, buf
+        self.ids = buf[L.ids:L.ids + T * K * 4].view(torch.int32).view(T, K)
+        self.w = buf[L.w:L.w + T * K * 4].view(torch.float32).view(T, K)
+        self.a8 = buf[L.a8:L.a8 + T * H].view(B.FP8).view(T, H)
+        self.scale = buf[L.scale:L.scale + (H // 128) * T * 4].view(torch.float32).view(H // 128, T)
+        self.rows = buf[L.rows:L.rows + T * K * H * 2].view(torch.bfloat16).view(T * K, H)
+        self.flags = buf[L.flags:L.flags + 16 + T * K]
+        self.barrier = buf[L.barrier:L.barrier + B.EP_BARRIER_WORDS * 8].view(torch.int64)
+
+    @staticmethod
+    def addresses(base: int, T: int, K: int, H: int) -> dict:
+        L = ep_buffer_layout(T, K, H)
+        return {name: base + getattr(L, name) for name in ("ids", "w", "a8", "scale", "rows", "flags", "barrier")}
+
+
+class EpPeerRank:
+    """One expert-parallel rank's steps over peer memory (include/fp8moe.h): publish its
+    routing and activations, gather every rank's pairs of its own experts (routing read
+    from the other ranks, activation rows pulled by the fused call's gather), return each
+    pair's weighted row to its origin, and combine its own tokens' rows. `peers` maps each
+    buffer name to the n ranks' addresses, as this GPU sees them."""
+
+    def __init__(self, cfg: I.MoEConfig, shard: "ExpertShard", n: int, rank: int, T: int, mine: EpRankBuffers,
+                 peers: dict):
+        self.cfg, self.shard, self.n, self.rank, self.T, self.mine, self.peers = cfg, shard, n, rank, T, mine, peers
+        dev = mine.buf.device
+        K, ne = cfg.K, shard.e1 - shard.e0
+        self.ids_g = torch.empty(n * T, K, dtype=torch.int32, device=dev)
+        self.w_g = torch.empty(n * T, K, dtype=torch.float32, device=dev)
+        self.sorted = B.alloc_sorted(n * T, K, ne + 1, shard.block_m, dev)
+        self.sort_ws = torch.empty(B.moe_align_sort_workspace_bytes(n * T, K, ne + 1, shard.block_m),
+                                   dtype=torch.uint8, device=dev)
+        self.workspace = torch.empty(B.fused_moe_workspace_bytes(n * T, K, ne, cfg.H, cfg.I, shard.block_m,
+                                                                 capacity=self.sorted.capacity),
+                                     dtype=torch.uint8, device=dev)
+        self.out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
+
+    def publish(self, logits, bias, x):
+        cfg, m = self.cfg, self.mine
+        B.moe_biased_grouped_topk(logits, bias, m.w, m.ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
+        B.fp8_per_token_group_quant(x, 128, column_major_scales=True, q=m.a8, scales=m.scale)
+        m.flags.zero_()
+
+    def compute(self):
+        cfg, sh, p = self.cfg, self.shard, self.peers
+        ne = sh.e1 - sh.e0
+        B.moe_ep_routing(p["ids"], p["w"], self.T, cfg.K, cfg.E, sh.e0, ne, self.ids_g, self.w_g)
+        B.moe_align_sort(self.ids_g, self.w_g, ne + 1, sh.block_m, out=self.sorted, workspace=self.sort_ws,
+                         expert_mask=sh.sort_mask)
+        B.fused_moe_fp8_blockscale_g1u1_multi(p["a8"], p["scale"], self.T, cfg.H, sh.w1, sh.w2, self.sorted, cfg.K,
+                                              sh.w1_scale, sh.w2_scale, workspace=self.workspace)
+        B.moe_ep_return(self.workspace, self.sorted.capacity, self.T, cfg.K, cfg.H, cfg.I, self.sorted, p["rows"],
+                        [f + 16 for f in p["flags"]])
+
+    def combine(self):
+        return B.moe_combine_pairs(self.mine.rows, self.mine.flags, self.T, self.cfg.K, self.out)
+
+
+class ExpertParallelPeerMoE:
+    """One expert-parallel rank over peer memory: its experts, its own batch of T tokens, the
+    published buffers in torch's symmetric memory (rendezvoused over the group), and the
+    forward publish -> barrier -> gather/compute/return -> barrier -> combine. The output is
+    the one-GPU layer's for this rank's tokens, bit for bit."""
+
+    def __init__(self, cfg: I.MoEConfig, shard: "ExpertShard", T: int, group=None):
+        import torch.distributed._symmetric_memory as symm
+        n, r = _world(group), _rank(group)
+        ep_expert_range(cfg.E, r, n)
+        dev = shard.w1.device
+        L = ep_buffer_layout(T, cfg.K, cfg.H)
+        self.buf = symm.empty(L.total, dtype=torch.uint8, device=dev)
+        self.buf.zero_()
+        handle = symm.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
+        self._handle = handle
+        bases = [int(b) for b in handle.buffer_ptrs]
+        addrs = [EpRankBuffers.addresses(b, T, cfg.K, cfg.H) for b in bases]
+        peers = {k: [a[k] for a in addrs] for k in addrs[0]}
+        self.rank = EpPeerRank(cfg, shard, n, r, T, EpRankBuffers(self.buf, T, cfg.K, cfg.H), peers)
+        self.r, self.epoch = r, 0
+        torch.cuda.synchronize(dev)
+        if dist.is_initialized() and n > 1:
+            dist.barrier(group)            # every rank's barrier words are zero before the first forward
+
+    def forward(self, logits, bias, x):
+        rk = self.rank
+        rk.publish(logits, bias, x)
+        self.epoch += 1
+        B.moe_ep_barrier(self.r, rk.peers["barrier"], self.epoch)
+        rk.compute()
+        self.epoch += 1
+        B.moe_ep_barrier(self.r, rk.peers["barrier"], self.epoch)
+        return rk.combine()
+
+
+class EmulatedExpertParallel:
+    """All n expert-parallel ranks on one GPU, each with its own published buffers in this
+    GPU's memory and its own experts; the steps run rank after rank on one stream and the
+    two barriers as one launch over all ranks (moe_ep_barrier_emulated)."""
+
+    def __init__(self, cfg: I.MoEConfig, shards, T: int, device="cuda"):
+        n = len(shards)
+        L = ep_buffer_layout(T, cfg.K, cfg.H)
+        self.bufs = [torch.zeros(L.total, dtype=torch.uint8, device=device) for _ in range(n)]
+        addrs = [EpRankBuffers.addresses(b.data_ptr(), T, cfg.K, cfg.H) for b in self.bufs]
+        peers = {k: [a[k] for a in addrs] for k in addrs[0]}
+        self.ranks = [EpPeerRank(cfg, sh, n, r, T, EpRankBuffers(self.bufs[r], T, cfg.K, cfg.H), peers)
+                      for r, sh in enumerate(shards)]
+        self.peers, self.epoch = peers, 0
+
+    def forward(self, inputs):
+        """inputs[r] = (logits, bias, x) of rank r; returns the n ranks' outputs."""
+        for rk, args in zip(self.ranks, inputs):
+            rk.publish(*args)
+        self.epoch += 1
+        B.moe_ep_barrier_emulated(self.peers["barrier"], self.epoch)
+        for rk in self.ranks:
+            rk.compute()
+        self.epoch += 1
+        B.moe_ep_barrier_emulated(self.peers["barrier"], self.epoch)
+        return [rk.combine() for rk in self.ranks]

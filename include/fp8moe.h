@@ -271,7 +271,8 @@ int fp8_blockscale_gemm(const uint8_t* A, const uint8_t* B,
  * id dropped as out of range) adds nothing; a token with no pair present gets
  * a zero row.
  * Limits: scale_blk_n == scale_blk_k == 128; H % 128 == 0; I % 128 == 0;
- * topk <= 32;
+ * topk <= 32 (it may exceed E: an expert-parallel rank holds fewer experts than a
+ * token picks);
  * fc2_smooth_scale must be NULL (the pages do not define it); workspace >=
  * fused_moe_fp8_blockscale_g1u1_workspace(); capacity >= the sort's padded
  * length; workspace 256-byte aligned.
@@ -455,6 +456,95 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
                                    void* const* recv, void* const* out,
                                    uint64_t* const* flags, uint64_t* const* barriers,
                                    uint64_t epoch, void* stream);
+
+/*
+ * Expert parallelism over peer (NVLink) memory: the dispatch and the return as
+ * stores and loads across GPUs instead of all-to-alls.
+ * ("Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang", section
+ * "Blockscale FP8 MoE Computation": asm_moe's expert_mask, the hook of expert
+ * parallelism.)
+ *
+ * n ranks (<= FP8MOE_EP_MAX_RANKS), rank r holding experts [e0, e0 + ne) of E and
+ * its own Tq tokens; global token g = q*Tq + t is token t of rank q and global
+ * pair p = g*topk + k. Every rank publishes, in memory all ranks can address, its
+ * routing (topk_ids int32 [Tq, topk], topk_weights fp32 [Tq, topk]), its
+ * activations (a8 fp8 [Tq, H], scales fp32 [H/128, Tq]) and a return buffer (bf16
+ * rows [Tq*topk, H], then a 16-byte count that must be 0 and one flag byte per
+ * pair, zeroed before each forward). One forward on rank r:
+ *   moe_ep_barrier                     (every rank's inputs published)
+ *   moe_ep_routing                     every rank's pairs as r's local ids
+ *   moe_align_sort_masked              over n*Tq tokens and ne + 1 experts, the
+ *                                      last (the sentinel) masked out
+ *   fused_moe_fp8_blockscale_g1u1_multi  the owner's fused MoE on its experts; the
+ *                                      gather reads each pair's row where it lies
+ *   moe_ep_return                      each pair's weighted row into its origin's
+ *                                      return buffer, flag set
+ *   moe_ep_barrier                     (every rank's rows returned)
+ *   moe_combine_pairs                  r's output from its return buffer
+ * The result on every rank is that of fused_moe_fp8_blockscale_g1u1 on its own
+ * tokens with all E experts, bit for bit (the same rows, combined in k order).
+ * Host arrays `ids`, `w`, `a8`, `a1_scale`, `rows`, `pair_flags` and `words` hold
+ * one device pointer per rank, as this GPU addresses that rank's memory.
+ * Ownership: every buffer belongs to the caller; nothing is allocated.
+ */
+#define FP8MOE_EP_MAX_RANKS 8
+#define FP8MOE_EP_BARRIER_WORDS 8
+
+/* ids_out int32 [n*Tq, topk]: id - e0 for the owner's experts, ne for another
+ * rank's, -1 for an id outside [0, E) (which the sort drops and flags);
+ * w_out fp32 [n*Tq, topk]: the weights as they are. */
+int moe_ep_routing(const int32_t* const* ids, const float* const* w, int n, int Tq,
+                   int topk, int E, int e0, int ne, int32_t* ids_out, float* w_out,
+                   void* stream);
+
+/* fused_moe_fp8_blockscale_g1u1_pairs over the n*Tq global tokens, with the
+ * activations a8[q] (fp8 [Tq, H], 16-byte aligned) and scales a1_scale[q] (fp32
+ * [H/128, Tq]) read from rank q's memory; w1, w2 and their scales are the
+ * owner's ne experts; sorted_* come from moe_align_sort_masked over the routing
+ * of moe_ep_routing (T = n*Tq, ne + 1 experts); workspace as for
+ * fused_moe_fp8_blockscale_g1u1 with T = n*Tq and that capacity. */
+int fused_moe_fp8_blockscale_g1u1_multi(const uint8_t* const* a8,
+                                        const float* const* a1_scale, int n, int Tq,
+                                        const uint8_t* w1, const uint8_t* w2,
+                                        const int32_t* sorted_ids,
+                                        const float* sorted_weights,
+                                        const int32_t* sorted_expert_ids,
+                                        const int32_t* num_valid_ids, int H, int I,
+                                        int E, int topk, int block_m, size_t capacity,
+                                        const float* fc1_scale, const float* fc2_scale,
+                                        int scale_blk_n, int scale_blk_k,
+                                        const float* fc2_smooth_scale, int weights_tiled,
+                                        void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/* Every listed pair of the owner's sorted list: its weighted row (in `workspace`
+ * after fused_moe_fp8_blockscale_g1u1_multi with the same capacity, n, Tq, topk, H
+ * and I) is stored into rows[q] at the origin's pair id (rows[q] bf16
+ * [Tq*topk, H], 16-byte aligned) and pair_flags[q] at that id set to 1. */
+int moe_ep_return(const void* workspace, size_t capacity, int n, int Tq, int topk,
+                  int H, int I, const int32_t* sorted_ids,
+                  const int32_t* num_valid_ids, void* const* rows,
+                  void* const* pair_flags, void* stream);
+
+/* Flag barrier: rank `rank` stores epoch into word `rank` of every rank's
+ * FP8MOE_EP_BARRIER_WORDS 64-bit words (zero before the first call; 8-byte
+ * aligned) and waits until its own words 0..n-1 hold >= epoch. epoch grows by at
+ * least one per barrier; every rank passes the same sequence. The stream's earlier
+ * work (peer stores included) is visible to every rank past the barrier. A rank
+ * that never arrives leaves the others waiting until the bounded wait (about 2 s)
+ * expires: FP8MOE_DEVERR_TIMEOUT, after which the words must be zeroed again. The
+ * _emulated form runs all n ranks' barriers on this GPU in one launch. */
+int moe_ep_barrier(int n, int rank, uint64_t* const* words, uint64_t epoch,
+                   void* stream);
+int moe_ep_barrier_emulated(int n, uint64_t* const* words, uint64_t epoch,
+                            void* stream);
+
+/* out bf16 [T, H] = the combine of fused_moe_fp8_blockscale_g1u1 over pair rows
+ * (bf16 [T*topk, H]) and a flag region laid out as the workspace's: a 16-byte
+ * count of listed pairs (T*topk: no flag is read), then one flag byte per pair
+ * (a pair whose flag is 0 adds nothing). rows, out, flag_region 16-byte aligned. */
+int moe_combine_pairs(const uint16_t* rows, const void* flag_region, int T, int topk,
+                      int H, uint16_t* out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -165,3 +165,18 @@ def test_tensor_parallel_reduce_choice_is_checked():
     assert D.TensorParallelMoE(_Layer(), reduce="peer").reduce == "peer"
     with pytest.raises(ValueError):
         D.TensorParallelMoE(_Layer(), reduce="ring")
+
+
+def test_expert_parallel_buffer_layout():
+    """What an expert-parallel rank publishes, in one allocation: routing ids and weights
+    [T, K], activations [T, H] and scales [H/128, T], return rows [T*K, H] with a 16-byte
+    count and T*K flag bytes, and the barrier words; 256-byte aligned, in that order."""
+    for T, K, H in ((4096, 8, 7168), (100, 4, 1024), (1, 1, 128)):
+        L = D.ep_buffer_layout(T, K, H)
+        ends = [(L.ids, T * K * 4), (L.w, T * K * 4), (L.a8, T * H), (L.scale, H // 128 * T * 4),
+                (L.rows, T * K * H * 2), (L.flags, 16 + T * K), (L.barrier, 8 * 8)]
+        for (a, size), (b, _) in zip(ends, ends[1:] + [(L.total, 0)]):
+            assert a % 256 == 0 and a + size <= b
+    for bad in ((0, 8, 7168), (16, 0, 128), (16, 8, 100)):
+        with pytest.raises(ValueError):
+            D.ep_buffer_layout(*bad)

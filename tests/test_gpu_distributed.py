@@ -3,6 +3,7 @@ runs (its experts' weights only, the received rows' local ids with other ranks' 
 sentinel that the masked sort drops) against the oracle's partial outputs, for every rank of
 a four-way split, and the one-rank expert- and tensor-parallel layers against the oracle. The
 collectives between ranks are tested with gloo ranks on the CPU."""
+import contextlib
 import dataclasses
 
 import pytest
@@ -148,23 +149,25 @@ def test_tp_combine_allreduce_rejects_bad_arguments():
     assert B.device_status() == 0
 
 
-def test_one_rank_peer_all_reduce_through_symmetric_memory():
+@contextlib.contextmanager
+def _one_rank_nccl_group(tmp_path):
+    """A one-rank NCCL process group on this GPU over a file store (no TCP port to race for)."""
+    import torch.distributed as dist
+    store = dist.FileStore(str(tmp_path / "store"), 1)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, device_id=torch.device(DEV, 0))
+    try:
+        yield
+    finally:
+        dist.destroy_process_group()
+
+
+def test_one_rank_peer_all_reduce_through_symmetric_memory(tmp_path):
     """The multi-GPU form's host side on a one-rank NCCL group: the buffers come from torch's
     symmetric memory and the pointers from its rendezvous; with one rank the fused combine +
     all-reduce is the combine, so the output equals the layer's own bit for bit."""
     import gc
-    import os
-    import socket
-
-    import torch.distributed as dist
     cfg = TPCFG
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        port = s.getsockname()[1]
-    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device(DEV, 0))
-    try:
+    with _one_rank_nccl_group(tmp_path):
         layer = MoELayer(cfg, DEV).load_synthetic_weights()
         act = I.moe_activations(cfg)
         args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
@@ -178,5 +181,68 @@ def test_one_rank_peer_all_reduce_through_symmetric_memory():
         del tp, got
         gc.collect()
         torch.cuda.synchronize()
-    finally:
-        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- expert parallelism over peer memory
+EPCFG = I.MoEConfig("ep_t100_h1024_e16", T=100, H=1024, E=16, G=4, TG=2, K=4, I=512, seed=9)
+EP_HOT = I.MoEConfig("ep_hot_t96_h512_e32", T=96, H=512, E=32, G=4, TG=2, K=6, I=256, hot_experts=3, seed=11)
+
+
+@pytest.mark.parametrize("cfg,n", [(EPCFG, 2), (EPCFG, 4), (EP_HOT, 4), (EP_HOT, 8)], ids=lambda v: str(getattr(v, "name", v)))
+def test_emulated_peer_expert_parallel_equals_the_one_gpu_layer(cfg, n):
+    """Every rank of the peer-memory expert-parallel form on one GPU (each with its own tokens
+    and only its experts' weights; routing read across ranks, activation rows pulled by the
+    owner's gather, pair rows returned to their origin, the two flag barriers as one launch
+    over the ranks): each rank's output must equal the one-GPU layer's output for its tokens
+    bit for bit, over two forwards. EP_HOT's boosted experts load the ranks unevenly."""
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [D.ExpertShard(cfg, *D.ep_expert_range(cfg.E, r, n), DEV).load_synthetic_weights() for r in range(n)]
+    emu = D.EmulatedExpertParallel(cfg, shards, cfg.T, DEV)
+    for call in range(2):
+        inputs, wants = [], []
+        for r in range(n):
+            act = I.moe_activations(dataclasses.replace(cfg, seed=cfg.seed + 10 * r + 100 * call))
+            args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+            inputs.append(args)
+            wants.append(layer.forward(*args).clone())
+        outs = emu.forward(inputs)
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert torch.equal(outs[r], wants[r]), f"forward {call}, rank {r}"
+    assert emu.epoch == 4
+
+
+def test_ep_barrier_bounded_wait_runs_out_without_its_peer():
+    """Rank 0 of 2 at the flag barrier alone: rank 1's word is never set, the bounded wait
+    expires (about 2 s), FP8MOE_DEVERR_TIMEOUT is raised and the context stays usable."""
+    words = [torch.zeros(B.EP_BARRIER_WORDS, dtype=torch.int64, device=DEV) for _ in range(2)]
+    B.moe_ep_barrier(0, words, 1)
+    assert B.device_status() & 1
+    assert B.device_status() == 0
+    assert int(words[0][0]) == 1 and int(words[1][0]) == 1     # rank 0 published to both
+    with pytest.raises(B.Fp8MoeError):
+        B.moe_ep_barrier(2, words, 2)                           # rank outside [0, n)
+    with pytest.raises(B.Fp8MoeError):
+        B.moe_ep_barrier(0, words, 0)                           # epoch 0
+
+
+def test_one_rank_peer_expert_parallel_through_symmetric_memory(tmp_path):
+    """The multi-GPU expert-parallel form's host side on a one-rank NCCL group (buffers from
+    torch's symmetric memory, addresses from its rendezvous): with one rank it is the whole
+    layer, so the output equals the layer's bit for bit."""
+    import gc
+    cfg = EPCFG
+    with _one_rank_nccl_group(tmp_path):
+        layer = MoELayer(cfg, DEV).load_synthetic_weights()
+        act = I.moe_activations(cfg)
+        args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+        want = layer.forward(*args).clone()
+        ep = D.ExpertParallelPeerMoE(cfg, D.ExpertShard(cfg, 0, cfg.E, DEV).load_synthetic_weights(), cfg.T)
+        for _ in range(2):
+            got = ep.forward(*args)
+            torch.cuda.synchronize()
+            assert torch.equal(got, want)
+        assert ep.epoch == 4
+        del ep, got
+        gc.collect()
+        torch.cuda.synchronize()
