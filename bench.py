@@ -567,7 +567,11 @@ def run_distributed(args, world, rank, local):
         torch.cuda.empty_cache()
     else:
         e0, e1 = D.ep_expert_range(cfg.E, rank, world)
-        model = D.ExpertParallelMoE(cfg, D.ExpertShard(cfg, e0, e1, dev).load_synthetic_weights())
+        shard = D.ExpertShard(cfg, e0, e1, dev).load_synthetic_weights()
+        if args.ep_exchange == "peer":
+            model = D.ExpertParallelPeerMoE(cfg, shard, cfg.T)
+        else:
+            model = D.ExpertParallelMoE(cfg, shard)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -626,7 +630,8 @@ def run_distributed(args, world, rank, local):
                                    ("by the combine fused with the all-reduce over peer memory" if args.tp_reduce ==
                                     "peer" else "by an fp32 NCCL reduce-scatter and a bf16 all-gather")) if tp else
                                   (f"ep{world}: experts split over the ranks, each rank its own batch of {cfg.T} "
-                                   "tokens, dispatch and return all-to-alls over NCCL"),
+                                   "tokens, " + ("dispatch and return over peer memory" if args.ep_exchange == "peer"
+                                                 else "dispatch and return all-to-alls over NCCL")),
                    "l2": "flushed between steps (256 MB write)", "cuda_graph": False},
         "tflops": flops / (ms_per_step * 1e-3) / 1e12,
         "layer_roofline": {"ms": t_roof, "frac": t_roof / ms_per_step, "flops": flops,
@@ -716,6 +721,73 @@ def run_tp_emulated(args, local):
     }
 
 
+def run_ep_emulated(args, local):
+    """prefill_ep with --ep-emulate N on one GPU: N expert-parallel ranks over peer memory
+    (EmulatedExpertParallel), each with its own batch of T tokens and E/N experts, their steps
+    in turn on one stream and their barriers as one launch; timed beside the one-GPU layer
+    run on the same N batches. The difference is what the exchange adds (routing read across
+    ranks, the owners' sorts over N*T tokens, the rows pulled in the gather and returned);
+    no multi-GPU number."""
+    from fp8_block_scaled_biased_b200 import binding as B
+    from fp8_block_scaled_biased_b200 import distributed as D
+    from fp8_block_scaled_biased_b200.layer import MoELayer
+
+    n = args.ep_emulate
+    cfg = DIST_WORKLOADS["prefill_ep"]
+    dev = torch.device("cuda", local)
+    layer = MoELayer(cfg, dev).load_synthetic_weights()
+    shards = [D.ExpertShard(cfg, *D.ep_expert_range(cfg.E, r, n), dev).load_synthetic_weights() for r in range(n)]
+    emu = D.EmulatedExpertParallel(cfg, shards, cfg.T, dev)
+    inputs = []
+    for r in range(n):
+        act = I.moe_activations(dataclasses.replace(cfg, seed=cfg.seed + r))
+        inputs.append((act.logits.to(dev), act.bias.to(dev), act.x.to(dev)))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i, (a, b) in enumerate(ev):
+            flush.fill_(i & 0xFF)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    for _ in range(3):
+        emu.forward(inputs)
+    ep_ms = timed(lambda: emu.forward(inputs))
+    one_ms = timed(lambda: [layer.forward(*inp) for inp in inputs])
+    clocks = sampler.stop()
+    if B.device_status():
+        raise RuntimeError("device error word set during the timed steps")
+    outs = emu.forward(inputs)
+    same = all(torch.equal(outs[r], layer.forward(*inputs[r])) for r in range(n))
+    ms = sum(ep_ms) / len(ep_ms)
+    base = sum(one_ms) / len(one_ms)
+    return {
+        "metric": METRIC, "value": n * cfg.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "none (all ranks on one GPU)", "vs_baseline": None,
+        "dtype": "fp8_e4m3fn x fp8_e4m3fn -> fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded; random-init weights quantised to FP8 in 128x128 blocks)",
+        "config": {"workload": f"{cfg.name}_ep{n}_emulated_on_1_gpu", "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                   "topk": cfg.K, "I": cfg.I, "parallelism": f"ep{n} over peer memory emulated: {n} ranks' batches "
+                   "and experts on one GPU, steps in turn, barriers as one launch",
+                   "l2": "flushed between steps (256 MB write)", "cuda_graph": False},
+        "one_gpu_layer_ms": base, "exchange_overhead": ms / base - 1.0, "outputs_equal_one_gpu_layer": same,
+        "step_ms": {"median": statistics.median(ep_ms), "min": min(ep_ms), "max": max(ep_ms)},
+        "gpu_launches": None, "clocks": clocks,
+    }
+
+
 def workload_config(args):
     """The MoE workload's configuration; with --tokens T, the same recipe (shapes, routing,
     value distributions, seed) at T tokens: one point of a batch-size sweep."""
@@ -731,6 +803,8 @@ def run_ours(args, world, rank, local):
     if args.workload in DIST_WORKLOADS:
         if args.tp_emulate:
             return run_tp_emulated(args, local)
+        if args.ep_emulate:
+            return run_ep_emulated(args, local)
         return run_distributed(args, world, rank, local)
     cfg = workload_config(args)
     dev = torch.device("cuda", local)
@@ -979,6 +1053,11 @@ def main():
     ap.add_argument("--tp-reduce", choices=["peer", "nccl"], default="peer",
                     help="prefill_tp: sum the ranks' partials with the combine fused with the all-reduce over "
                          "peer memory (peer) or with NCCL's reduce-scatter and all-gather (nccl)")
+    ap.add_argument("--ep-exchange", choices=["peer", "nccl"], default="peer",
+                    help="prefill_ep: dispatch and return over peer memory (peer) or NCCL all-to-alls (nccl)")
+    ap.add_argument("--ep-emulate", type=int, default=0,
+                    help="prefill_ep on one GPU: N expert-parallel ranks over peer memory there, timed beside the "
+                         "one-GPU layer on the same batches (a measurement of the exchange, not a multi-GPU number)")
     ap.add_argument("--tp-emulate", type=int, default=0,
                     help="prefill_tp on one GPU: run all N ranks there, their fused combine + all-reduce as one "
                          "launch (a kernel measurement, not a multi-GPU number)")
@@ -1001,6 +1080,9 @@ def main():
     if args.tp_emulate and (args.workload != "prefill_tp" or args.gpus != 1 or not 2 <= args.tp_emulate <= 8
                             or DIST_WORKLOADS["prefill_tp"].I % (128 * args.tp_emulate)):
         ap.error("--tp-emulate takes 2..8 ranks that split I into 128-column blocks, with prefill_tp on one GPU")
+    if args.ep_emulate and (args.workload != "prefill_ep" or args.gpus != 1 or not 2 <= args.ep_emulate <= 8
+                            or DIST_WORKLOADS["prefill_ep"].E % args.ep_emulate):
+        ap.error("--ep-emulate takes 2..8 ranks that split E evenly, with prefill_ep on one GPU")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -155,3 +155,10 @@ def test_tp_emulate_option_is_checked():
                 ["--workload", "prefill_tp", "--tp-emulate", "1"], ["--workload", "prefill_tp", "--tp-emulate", "3"]):
         r = subprocess.run([sys.executable, "bench.py", *bad], cwd=ROOT, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0 and "--tp-emulate" in r.stderr, bad
+
+
+def test_ep_emulate_option_is_checked():
+    for bad in (["--workload", "prefill", "--ep-emulate", "8"], ["--workload", "prefill_ep", "--ep-emulate", "9"],
+                ["--workload", "prefill_ep", "--ep-emulate", "3"]):
+        r = subprocess.run([sys.executable, "bench.py", *bad], cwd=ROOT, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0 and "--ep-emulate" in r.stderr, bad
