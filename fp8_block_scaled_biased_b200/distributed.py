@@ -1,11 +1,12 @@
 """Multi-GPU forms of the FP8 block-scaled MoE layer, one process per GPU over
-torch.distributed (NCCL between GPUs; gloo for the rank logic on the CPU).
+torch.distributed (between GPUs NCCL, or the library's kernels on peer memory from
+torch's symmetric memory; gloo for the rank logic on the CPU).
 
 "Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang" runs the layer at
 TP8 (section "Performance Reproduction for AITER-Optimized in SGLang", --tp 8),
 summing the ranks' outputs with the custom all-reduce of section "Other
 Operators", and gives asm_moe an expert_mask (section "Blockscale FP8 MoE
-Computation"), the hook of expert parallelism. Two forms are built here:
+Computation"), the hook of expert parallelism. Both are built here:
 
 Tensor parallelism over I (TensorParallelMoE). Every rank routes every token and
 runs its shard of each expert's intermediate columns (MoELayer.tp_shard). The
@@ -30,11 +31,21 @@ each received row's partial output (the bf16 sum over that rank's pairs), and th
 origin adds, per token, the partial rows in ascending rank order in fp32 and
 rounds to bf16 once. The result is deterministic for a given rank count.
 
-The compute is the library's kernels (routing, quantisation, sort, fused MoE);
-the collectives are NCCL's; what lies between them here is index bookkeeping and
-byte packing on the device (torch indexing), with the local compute passed in as
-a callable so that the rank logic runs unchanged on the CPU with the oracle in
-its place.
+Expert parallelism over peer memory (ExpertParallelPeerMoE). The same split with
+no all-to-all: every rank publishes its routing, activations and a return buffer
+in symmetric memory; each owner reads every rank's routing (moe_ep_routing),
+sorts the pairs of its experts over all ranks' tokens, gathers their activation
+rows where they lie inside its fused call (fused_moe_fp8_blockscale_g1u1_multi)
+and stores each pair's weighted row into its origin's return buffer
+(moe_ep_return); two flag barriers (moe_ep_barrier) order the steps. Each rank
+then combines its own tokens' rows exactly as one GPU does, so the output is the
+one-GPU layer's bit for bit. EmulatedExpertParallel runs all ranks on one GPU.
+
+The compute is the library's kernels (routing, quantisation, sort, fused MoE,
+and for the peer forms the exchange itself); the NCCL forms' collectives are
+NCCL's, with index bookkeeping and byte packing on the device (torch indexing)
+between them and the local compute passed in as a callable, so that their rank
+logic runs unchanged on the CPU with the oracle in its place.
 """
 from __future__ import annotations
 
@@ -475,6 +486,7 @@ class ExpertParallelPeerMoE:
             dist.barrier(group)            # every rank's barrier words are zero before the first forward
 
     def forward(self, logits, bias, x):
+        """This rank's tokens -> its output bf16 [T, H] (a buffer the next forward rewrites)."""
         rk = self.rank
         rk.publish(logits, bias, x)
         self.epoch += 1
