@@ -440,6 +440,8 @@ class EpPeerRank:
         self.out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
 
     def publish(self, logits, bias, x):
+        if x.shape[0] != self.T or logits.shape[0] != self.T:
+            raise ValueError(f"this rank's buffers are sized for {self.T} tokens, got {x.shape[0]}")
         cfg, m = self.cfg, self.mine
         B.moe_biased_grouped_topk(logits, bias, m.w, m.ids, cfg.G, cfg.TG, cfg.renorm, cfg.scale)
         B.fp8_per_token_group_quant(x, 128, column_major_scales=True, q=m.a8, scales=m.scale)
@@ -514,6 +516,8 @@ class EmulatedExpertParallel:
 
     def forward(self, inputs):
         """inputs[r] = (logits, bias, x) of rank r; returns the n ranks' outputs."""
+        if len(inputs) != len(self.ranks):
+            raise ValueError(f"one input set per rank ({len(self.ranks)}), got {len(inputs)}")
         for rk, args in zip(self.ranks, inputs):
             rk.publish(*args)
         self.epoch += 1
