@@ -694,6 +694,13 @@ def run_tp_emulated(args, local):
     clocks = sampler.stop()
     if B.device_status():
         raise RuntimeError("device error word set during the timed steps")
+    # every rank's output against bf16 of the rank-order fp32 sum of the ranks' own combines
+    partials = [sh.forward(logits, bias, x).float() for sh in shards]
+    want = partials[0]
+    for p in partials[1:]:
+        want = want + p
+    outs = step()
+    same = all(torch.equal(o, want.to(torch.bfloat16)) for o in outs)
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     ar_ms = [e[1].elapsed_time(e[2]) for e in ev]
     ms_per_step = sum(step_ms) / args.steps
@@ -716,6 +723,7 @@ def run_tp_emulated(args, local):
                       "bytes": ar_bytes, "achieved": ar_bytes / (ar * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                       "frac": ar_bytes / (ar * 1e-3) / 1e9 / hbm, "peak_source": "measured",
                       "note": "CUDA events around the emulated launch; the ranks' stores stay in this GPU's memory"},
+        "outputs_equal_rank_order_sum": same,
         "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
         "gpu_launches": None, "clocks": clocks,
     }
