@@ -222,8 +222,8 @@ def layer_work(cfg, ids, mask=None):
 # figure whose sources have changed since is not reported.
 GATE_UP_TRAFFIC = {
     "prefill_t4096_h7168_e256": {
-        "bytes": 6.810e9,
-        "sha256": "1b410dc9b6f77136e0368a93c182c91921b7c5aa3243d082a167790710085253",
+        "bytes": 6.752e9,
+        "sha256": "730be5c99bff17e3b4cfc065e91115dd7e912e0198471e5d7299704ee96b3daa",
         "capture": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum of "
                    "`python bench.py --steps 2 --warmup 3 --no-cpu-baseline --no-graph --no-workloads` "
                    "(2 launches, mean; tiled weights)",
@@ -772,6 +772,11 @@ def run_ep_emulated(args, local):
     for _ in range(3):
         emu.forward(inputs)
     ep_ms = timed(lambda: emu.forward(inputs))
+    for rk in emu.ranks:                  # the same with the rows returned by a separate kernel
+        rk.return_in_gemm = False
+    ep_kernel_ms = timed(lambda: emu.forward(inputs))
+    for rk in emu.ranks:
+        rk.return_in_gemm = True
     one_ms = timed(lambda: [layer.forward(*inp) for inp in inputs])
     clocks = sampler.stop()
     if B.device_status():
@@ -791,6 +796,7 @@ def run_ep_emulated(args, local):
                    "and experts on one GPU, steps in turn, barriers as one launch",
                    "l2": "flushed between steps (256 MB write)", "cuda_graph": False},
         "one_gpu_layer_ms": base, "exchange_overhead": ms / base - 1.0, "outputs_equal_one_gpu_layer": same,
+        "return_by_kernel_ms": sum(ep_kernel_ms) / len(ep_kernel_ms),
         "step_ms": {"median": statistics.median(ep_ms), "min": min(ep_ms), "max": max(ep_ms)},
         "gpu_launches": None, "clocks": clocks,
     }

@@ -63,7 +63,7 @@ _SIGNATURES = {
     "moe_ep_routing": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p]),
     "fused_moe_fp8_blockscale_g1u1_multi": (_c_int, [_p, _p, _c_int, _c_int, _p, _p, _p, _p, _p, _p, _c_int, _c_int,
                                                      _c_int, _c_int, _c_int, _c_size, _p, _p, _c_int, _c_int, _p,
-                                                     _c_int, _p, _c_size, _p]),
+                                                     _c_int, _p, _p, _p, _c_size, _p]),
     "moe_ep_return": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p]),
     "moe_ep_barrier": (_c_int, [_c_int, _c_int, _p, ctypes.c_uint64, _p]),
     "moe_ep_barrier_emulated": (_c_int, [_c_int, _p, ctypes.c_uint64, _p]),
@@ -531,11 +531,20 @@ def moe_ep_routing(ids, w, Tq, topk, E, e0, ne, ids_out, w_out):
 
 
 def fused_moe_fp8_blockscale_g1u1_multi(a8, a1_scale, Tq, H, w1, w2, sorted_pairs: SortedPairs, topk, fc1_scale,
-                                        fc2_scale, workspace=None):
+                                        fc2_scale, workspace=None, return_rows=None, return_flags=None):
     """The owner's fused MoE over every rank's tokens (without the combine): a8[q] fp8 [Tq, H]
     and a1_scale[q] fp32 [H/128, Tq] of rank q, as addresses or tensors; the owner's weights;
-    the sort over n*Tq tokens. Returns the workspace holding the weighted pair rows."""
+    the sort over n*Tq tokens. return_rows / return_flags: int64 [n] device tensors holding
+    every rank's return rows and pair-flag addresses, for the down GEMM to store each pair's
+    row into its origin's buffer; without them the rows stay in the returned workspace."""
     n = len(a8)
+    if (return_rows is None) != (return_flags is None):
+        raise ValueError("return_rows and return_flags go together")
+    if return_rows is not None:
+        for name, t in (("return_rows", return_rows), ("return_flags", return_flags)):
+            _cuda(t, torch.int64, name)
+            if t.numel() != n or not t.is_contiguous():
+                raise ValueError(f"{name} must hold one address per rank")
     if len(a1_scale) != n or not 1 <= n <= EP_MAX_RANKS:
         raise ValueError("one activation and one scale buffer per rank (at most EP_MAX_RANKS)")
     for name, t in (("w1", w1), ("w2", w2)):
@@ -564,8 +573,8 @@ def fused_moe_fp8_blockscale_g1u1_multi(a8, a1_scale, Tq, H, w1, w2, sorted_pair
     rc = load_library().fused_moe_fp8_blockscale_g1u1_multi(
         _addresses(a8, "a8"), _addresses(a1_scale, "a1_scale"), n, Tq, _ptr(w1), _ptr(w2), _ptr(sp.sorted_ids),
         _ptr(sp.sorted_weights), _ptr(sp.sorted_expert_ids), _ptr(sp.num_valid_ids), H, I, E, topk, sp.block_m,
-        sp.capacity, _ptr(fc1_scale), _ptr(fc2_scale), 128, 128, None, 1 if is_tiled(w1) else 0, _ptr(workspace),
-        workspace.numel(), _stream())
+        sp.capacity, _ptr(fc1_scale), _ptr(fc2_scale), 128, 128, None, 1 if is_tiled(w1) else 0, _ptr(return_rows),
+        _ptr(return_flags), _ptr(workspace), workspace.numel(), _stream())
     _check("fused_moe_fp8_blockscale_g1u1_multi", rc)
     return workspace
 

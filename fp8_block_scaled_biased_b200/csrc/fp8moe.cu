@@ -75,9 +75,9 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[kMaxDevices];
 
-template <int MODE, bool TILED_B = false>
+template <int MODE, bool TILED_B = false, bool ROUTED = false>
 cudaError_t enable_gemm_smem() {
-  return cudaFuncSetAttribute(blockscale_gemm_kernel<MODE, TILED_B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(blockscale_gemm_kernel<MODE, TILED_B, ROUTED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(kGemmSmemBytes));
 }
 
@@ -103,6 +103,8 @@ int device_setup(int* sm_count) {
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeUp, true>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, true>();
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, false, true>();
+    if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, true, true>();
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sort_scatter_smem(kSortMaxExperts)));
@@ -521,7 +523,8 @@ static int fused_moe_impl(const char* name, bool tiled, bool combine, uint16_t* 
                           int topk, int block_m, size_t capacity, const float* a1_scale, const float* fc1_scale,
                           const float* fc2_scale, int scale_blk_n, int scale_blk_k, const float* fc2_smooth_scale,
                           void* workspace, size_t workspace_bytes, void* stream,
-                          const GatherSources* srcs = nullptr) {
+                          const GatherSources* srcs = nullptr, __nv_bfloat16* const* y_src_rows = nullptr,
+                          uint8_t* const* y_src_flags = nullptr, int y_src_pairs = 0) {
   (void)name;
   if (scale_blk_n != 128 || scale_blk_k != 128)
     return fail(FP8MOE_EUNSUPPORTED, "only (128, 128) scale blocks are supported (got %d, %d)", scale_blk_n,
@@ -638,7 +641,14 @@ static int fused_moe_impl(const char* name, bool tiled, bool combine, uint16_t* 
   dn.nb_valid = H / 128;
   dn.b_rows_per_expert = H;
   dn.s2 = nullptr;
-  if (tiled)
+  dn.y_src_rows = y_src_rows;
+  dn.y_src_flags = y_src_flags;
+  dn.y_src_pairs = y_src_pairs;
+  if (dn.y_src_rows && tiled)
+    blockscale_gemm_kernel<kModeMoeDown, true, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, m_a264, dn);
+  else if (dn.y_src_rows)
+    blockscale_gemm_kernel<kModeMoeDown, false, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, m_a264, dn);
+  else if (tiled)
     blockscale_gemm_kernel<kModeMoeDown, true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, m_a264, dn);
   else
     blockscale_gemm_kernel<kModeMoeDown><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(m_a2, m_w2, m_a264, dn);
@@ -920,8 +930,11 @@ int fused_moe_fp8_blockscale_g1u1_multi(const uint8_t* const* a8, const float* c
                                         const int32_t* num_valid_ids, int H, int I, int E, int topk, int block_m,
                                         size_t capacity, const float* fc1_scale, const float* fc2_scale,
                                         int scale_blk_n, int scale_blk_k, const float* fc2_smooth_scale,
-                                        int weights_tiled, void* workspace, size_t workspace_bytes, void* stream) {
+                                        int weights_tiled, void* const* return_rows, void* const* return_flags,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
   if (n < 1 || n > kMaxSources) return fail(FP8MOE_EINVAL, "n must be in [1, %d]", kMaxSources);
+  if ((return_rows == nullptr) != (return_flags == nullptr))
+    return fail(FP8MOE_EINVAL, "return_rows and return_flags are given together or not at all");
   if (Tq < 0 || static_cast<long long>(Tq) * n >= (1ll << 31)) return fail(FP8MOE_EINVAL, "bad Tq");
   if (!a8 || !a1_scale) return fail(FP8MOE_EINVAL, "null pointer argument");
   GatherSources srcs{};
@@ -936,7 +949,8 @@ int fused_moe_fp8_blockscale_g1u1_multi(const uint8_t* const* a8, const float* c
   return fused_moe_impl("fused_moe_fp8_blockscale_g1u1_multi", weights_tiled != 0, false, nullptr, nullptr, w1, w2,
                         sorted_ids, sorted_weights, sorted_expert_ids, num_valid_ids, n * Tq, H, I, E, topk, block_m,
                         capacity, nullptr, fc1_scale, fc2_scale, scale_blk_n, scale_blk_k, fc2_smooth_scale, workspace,
-                        workspace_bytes, stream, &srcs);
+                        workspace_bytes, stream, &srcs, reinterpret_cast<__nv_bfloat16* const*>(return_rows),
+                        reinterpret_cast<uint8_t* const*>(return_flags), Tq * topk);
 }
 
 int moe_ep_return(const void* workspace, size_t capacity, int n, int Tq, int topk, int H, int I,

@@ -89,6 +89,12 @@ struct GemmArgs {
   uint8_t* a2;            // up output [M, I] (slot-ordered FP8 intermediate)
   float* s2;              // up output [I/128, M]
   __nv_bfloat16* ystage;  // down output [T*topk, H] (weighted rows by pair id, bf16)
+  // down, expert parallelism: when set, pair p = q * y_src_pairs + lp is stored into
+  // y_src_rows[q] + lp * H (rank q's return rows, possibly another GPU's memory) and
+  // y_src_flags[q][lp] set to 1, instead of into ystage (device arrays of pointers)
+  __nv_bfloat16* const* y_src_rows;
+  uint8_t* const* y_src_flags;
+  int y_src_pairs;
   // Failure-handling test hook (0 = off): with k + 1, the scale loader withholds
   // K block k's scales, so the epilogue's bounded wait for them runs out and the
   // CTA takes its abort path (device error word, TMEM freed, clean exit).
@@ -219,7 +225,9 @@ __device__ __forceinline__ void store_rows_64B(uint8_t* staging, int lane, const
 
 // The epilogue warpgroups: promotion of each K block's partial sums into fp32
 // registers, then the mode's output through the per-warp staging buffer.
-template <int MODE>
+// ROUTED (down GEMM, expert parallelism): every pair row goes to its origin's return
+// rows (args.y_src_*) instead of ystage.
+template <int MODE, bool ROUTED = false>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s, uint8_t* staging,
                                               uint32_t tmem_base, int warp, int lane, int m_blocks,
                                               int total_tiles, int num_kb, int P) {
@@ -408,10 +416,23 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
         uint8_t* my_staging = staging + ew * kStagingBytes;
         // destinations of the four rows this lane stores (null for padding rows)
         uint8_t* dst[4];
+        int prs[4];
+        if constexpr (!ROUTED) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int pr = __shfl_sync(0xffffffffu, pair, store_rows_row(i, lane));
-          dst[i] = (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x0) : nullptr;
+          for (int i = 0; i < 4; ++i) {
+            const int pr = __shfl_sync(0xffffffffu, pair, store_rows_row(i, lane));
+            dst[i] = (pr >= 0 && pr < P) ? reinterpret_cast<uint8_t*>(y + static_cast<size_t>(pr) * H + x0) : nullptr;
+          }
+        } else {                              // each row into its origin's return rows
+          // (pair ids held, the address made per store: fewer live registers)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) prs[i] = __shfl_sync(0xffffffffu, pair, store_rows_row(i, lane));
+          if (valid && nt == 0 && half == 0) {   // one thread per row sets the pair's flag
+            const int q = pair / args.y_src_pairs;
+            uint8_t* flags = reinterpret_cast<uint8_t*>(
+                __ldg(reinterpret_cast<const unsigned long long*>(args.y_src_flags) + q));
+            flags[pair - q * args.y_src_pairs] = 1;
+          }
         }
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {      // 4 chunks of 32 bf16 columns
@@ -427,7 +448,19 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
             }
             d[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          store_rows_64B(my_staging, lane, d, [&](int i) -> uint8_t* { return dst[i] ? dst[i] + ch * 64 : nullptr; });
+          store_rows_64B(my_staging, lane, d, [&](int i) -> uint8_t* {
+            if constexpr (!ROUTED) {
+              return dst[i] ? dst[i] + ch * 64 : nullptr;
+            } else {
+              const int pr = prs[i];
+              if (pr < 0 || pr >= P) return nullptr;
+              const int q = pr / args.y_src_pairs;
+              __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(
+                  __ldg(reinterpret_cast<const unsigned long long*>(args.y_src_rows) + q));
+              return reinterpret_cast<uint8_t*>(base + static_cast<size_t>(pr - q * args.y_src_pairs) * H + x0) +
+                     ch * 64;
+            }
+          });
         }
       }
     }
@@ -438,7 +471,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& args, GemmSmem* s,
   if (!ok) abort_all(s);
 }
 
-template <int MODE, bool TILED_B = false>
+template <int MODE, bool TILED_B = false, bool ROUTED = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmA64, const GemmArgs args) {
@@ -491,7 +524,7 @@ blockscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
   if (warp >= 4) {
     warpgroup_reg_alloc<kRegsEpilogue>();
-    epilogue_role<MODE>(args, s, staging, tmem_base, warp, lane, m_blocks, total_tiles, num_kb, P);
+    epilogue_role<MODE, ROUTED>(args, s, staging, tmem_base, warp, lane, m_blocks, total_tiles, num_kb, P);
   } else {
     warpgroup_reg_dealloc<kRegsWg0>();     // one instruction for all four warps of warpgroup 0
     if (warp == 0) {

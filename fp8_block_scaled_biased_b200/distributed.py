@@ -425,9 +425,14 @@ class EpPeerRank:
     buffer name to the n ranks' addresses, as this GPU sees them."""
 
     def __init__(self, cfg: I.MoEConfig, shard: "ExpertShard", n: int, rank: int, T: int, mine: EpRankBuffers,
-                 peers: dict):
+                 peers: dict, return_in_gemm: bool = True):
+        """return_in_gemm: the down GEMM stores each pair's row into its origin's buffer (True),
+        or the rows stay in the workspace and moe_ep_return copies them there (False)."""
         self.cfg, self.shard, self.n, self.rank, self.T, self.mine, self.peers = cfg, shard, n, rank, T, mine, peers
         dev = mine.buf.device
+        self.return_in_gemm = return_in_gemm
+        self.ret_rows = torch.tensor(peers["rows"], dtype=torch.int64, device=dev)
+        self.ret_flags = torch.tensor([f + 16 for f in peers["flags"]], dtype=torch.int64, device=dev)
         K, ne = cfg.K, shard.e1 - shard.e0
         self.ids_g = torch.empty(n * T, K, dtype=torch.int32, device=dev)
         self.w_g = torch.empty(n * T, K, dtype=torch.float32, device=dev)
@@ -453,10 +458,15 @@ class EpPeerRank:
         B.moe_ep_routing(p["ids"], p["w"], self.T, cfg.K, cfg.E, sh.e0, ne, self.ids_g, self.w_g)
         B.moe_align_sort(self.ids_g, self.w_g, ne + 1, sh.block_m, out=self.sorted, workspace=self.sort_ws,
                          expert_mask=sh.sort_mask)
-        B.fused_moe_fp8_blockscale_g1u1_multi(p["a8"], p["scale"], self.T, cfg.H, sh.w1, sh.w2, self.sorted, cfg.K,
-                                              sh.w1_scale, sh.w2_scale, workspace=self.workspace)
-        B.moe_ep_return(self.workspace, self.sorted.capacity, self.T, cfg.K, cfg.H, cfg.I, self.sorted, p["rows"],
-                        [f + 16 for f in p["flags"]])
+        if self.return_in_gemm:
+            B.fused_moe_fp8_blockscale_g1u1_multi(p["a8"], p["scale"], self.T, cfg.H, sh.w1, sh.w2, self.sorted,
+                                                  cfg.K, sh.w1_scale, sh.w2_scale, workspace=self.workspace,
+                                                  return_rows=self.ret_rows, return_flags=self.ret_flags)
+        else:
+            B.fused_moe_fp8_blockscale_g1u1_multi(p["a8"], p["scale"], self.T, cfg.H, sh.w1, sh.w2, self.sorted,
+                                                  cfg.K, sh.w1_scale, sh.w2_scale, workspace=self.workspace)
+            B.moe_ep_return(self.workspace, self.sorted.capacity, self.T, cfg.K, cfg.H, cfg.I, self.sorted,
+                            p["rows"], [f + 16 for f in p["flags"]])
 
     def combine(self):
         return B.moe_combine_pairs(self.mine.rows, self.mine.flags, self.T, self.cfg.K, self.out)
@@ -504,14 +514,14 @@ class EmulatedExpertParallel:
     GPU's memory and its own experts; the steps run rank after rank on one stream and the
     two barriers as one launch over all ranks (moe_ep_barrier_emulated)."""
 
-    def __init__(self, cfg: I.MoEConfig, shards, T: int, device="cuda"):
+    def __init__(self, cfg: I.MoEConfig, shards, T: int, device="cuda", return_in_gemm: bool = True):
         n = len(shards)
         L = ep_buffer_layout(T, cfg.K, cfg.H)
         self.bufs = [torch.zeros(L.total, dtype=torch.uint8, device=device) for _ in range(n)]
         addrs = [EpRankBuffers.addresses(b.data_ptr(), T, cfg.K, cfg.H) for b in self.bufs]
         peers = {k: [a[k] for a in addrs] for k in addrs[0]}
-        self.ranks = [EpPeerRank(cfg, sh, n, r, T, EpRankBuffers(self.bufs[r], T, cfg.K, cfg.H), peers)
-                      for r, sh in enumerate(shards)]
+        self.ranks = [EpPeerRank(cfg, sh, n, r, T, EpRankBuffers(self.bufs[r], T, cfg.K, cfg.H), peers,
+                                 return_in_gemm) for r, sh in enumerate(shards)]
         self.peers, self.epoch = peers, 0
 
     def forward(self, inputs):

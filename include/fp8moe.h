@@ -476,9 +476,11 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
  *   moe_align_sort_masked              over n*Tq tokens and ne + 1 experts, the
  *                                      last (the sentinel) masked out
  *   fused_moe_fp8_blockscale_g1u1_multi  the owner's fused MoE on its experts; the
- *                                      gather reads each pair's row where it lies
- *   moe_ep_return                      each pair's weighted row into its origin's
- *                                      return buffer, flag set
+ *                                      gather reads each pair's row where it lies,
+ *                                      the down GEMM stores each pair's weighted
+ *                                      row into its origin's return buffer and
+ *                                      sets its flag (or moe_ep_return does it
+ *                                      after the call)
  *   moe_ep_barrier                     (every rank's rows returned)
  *   moe_combine_pairs                  r's output from its return buffer
  * The result on every rank is that of fused_moe_fp8_blockscale_g1u1 on its own
@@ -502,7 +504,12 @@ int moe_ep_routing(const int32_t* const* ids, const float* const* w, int n, int 
  * [H/128, Tq]) read from rank q's memory; w1, w2 and their scales are the
  * owner's ne experts; sorted_* come from moe_align_sort_masked over the routing
  * of moe_ep_routing (T = n*Tq, ne + 1 experts); workspace as for
- * fused_moe_fp8_blockscale_g1u1 with T = n*Tq and that capacity. */
+ * fused_moe_fp8_blockscale_g1u1 with T = n*Tq and that capacity.
+ * return_rows, return_flags: NULL (the weighted pair rows stay in the workspace,
+ * for moe_ep_return), or DEVICE arrays of n pointers to every rank's return rows
+ * (bf16 [Tq*topk, H], 16-byte aligned) and pair flags (bytes [Tq*topk]): the down
+ * GEMM's epilogue then stores each pair's row straight into its origin's return
+ * rows and sets its flag, which takes the place of moe_ep_return. */
 int fused_moe_fp8_blockscale_g1u1_multi(const uint8_t* const* a8,
                                         const float* const* a1_scale, int n, int Tq,
                                         const uint8_t* w1, const uint8_t* w2,
@@ -514,8 +521,9 @@ int fused_moe_fp8_blockscale_g1u1_multi(const uint8_t* const* a8,
                                         const float* fc1_scale, const float* fc2_scale,
                                         int scale_blk_n, int scale_blk_k,
                                         const float* fc2_smooth_scale, int weights_tiled,
-                                        void* workspace, size_t workspace_bytes,
-                                        void* stream);
+                                        void* const* return_rows,
+                                        void* const* return_flags, void* workspace,
+                                        size_t workspace_bytes, void* stream);
 
 /* Every listed pair of the owner's sorted list: its weighted row (in `workspace`
  * after fused_moe_fp8_blockscale_g1u1_multi with the same capacity, n, Tq, topk, H

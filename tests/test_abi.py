@@ -208,4 +208,6 @@ def test_multi_gpu_entry_points_reject_bad_arguments(lib):
     assert lib.moe_combine_pairs(p, p, 10, 0, 1024, p, None) == 1
     assert lib.moe_combine_pairs(p, p, 10, 4, 1004, p, None) == 1          # H % 8 != 0
     assert lib.fused_moe_fp8_blockscale_g1u1_multi(one, one, 9, 10, p, p, p, p, p, p, 1024, 512, 4, 4, 128, 1 << 20,
-                                                   p, p, 128, 128, None, 1, p, 1 << 30, None) == 1
+                                                   p, p, 128, 128, None, 1, None, None, p, 1 << 30, None) == 1
+    assert lib.fused_moe_fp8_blockscale_g1u1_multi(one, one, 1, 10, p, p, p, p, p, p, 1024, 512, 4, 4, 128, 1 << 20,
+                                                   p, p, 128, 128, None, 1, p, None, p, 1 << 30, None) == 1

@@ -246,3 +246,22 @@ def test_one_rank_peer_expert_parallel_through_symmetric_memory(tmp_path):
         del ep, got
         gc.collect()
         torch.cuda.synchronize()
+
+
+def test_emulated_peer_expert_parallel_with_the_return_kernel():
+    """The same exchange with the pair rows left in each owner's workspace and copied to their
+    origins by moe_ep_return instead of stored there by the down GEMM: the same outputs."""
+    cfg, n = EP_HOT, 4
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [D.ExpertShard(cfg, *D.ep_expert_range(cfg.E, r, n), DEV).load_synthetic_weights() for r in range(n)]
+    emu = D.EmulatedExpertParallel(cfg, shards, cfg.T, DEV, return_in_gemm=False)
+    inputs, wants = [], []
+    for r in range(n):
+        act = I.moe_activations(dataclasses.replace(cfg, seed=cfg.seed + 7 * r))
+        args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+        inputs.append(args)
+        wants.append(layer.forward(*args).clone())
+    outs = emu.forward(inputs)
+    torch.cuda.synchronize()
+    for r in range(n):
+        assert torch.equal(outs[r], wants[r]), f"rank {r}"
