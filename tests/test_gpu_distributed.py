@@ -265,3 +265,52 @@ def test_emulated_peer_expert_parallel_with_the_return_kernel():
     torch.cuda.synchronize()
     for r in range(n):
         assert torch.equal(outs[r], wants[r]), f"rank {r}"
+
+
+# ---------------------------------------------------------------- degenerate splits
+EP_EDGE = I.MoEConfig("ep_edge_t20_h256_e16", T=20, H=256, E=16, G=4, TG=1, K=4, I=256, seed=13)
+
+
+def test_emulated_peer_expert_parallel_with_idle_owners():
+    """Every pair on one rank's experts: the bias makes group 0 (experts 0-3, all of rank 0's
+    four) the only group chosen, so ranks 1-3 own no pair at all (empty sorted lists, GEMMs
+    with no tile) while still publishing, returning nothing and combining. Outputs must still
+    equal the one-GPU layer's."""
+    cfg, n = EP_EDGE, 4
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [D.ExpertShard(cfg, *D.ep_expert_range(cfg.E, r, n), DEV).load_synthetic_weights() for r in range(n)]
+    emu = D.EmulatedExpertParallel(cfg, shards, cfg.T, DEV)
+    inputs, wants = [], []
+    for r in range(n):
+        act = I.moe_activations(dataclasses.replace(cfg, seed=cfg.seed + r))
+        bias = act.bias.clone()
+        bias[:4] += 100.0
+        args = (act.logits.to(DEV), bias.to(DEV), act.x.to(DEV))
+        inputs.append(args)
+        wants.append(layer.forward(*args).clone())
+    assert int((layer.topk_ids >= 4).sum()) == 0                # the last input set: all on experts 0-3
+    outs = emu.forward(inputs)
+    torch.cuda.synchronize()
+    for r in range(n):
+        assert torch.equal(outs[r], wants[r]), f"rank {r}"
+    assert [int(rk.sorted.num_valid_ids.item()) for rk in emu.ranks[1:]] == [0, 0, 0]
+
+
+def test_emulated_tp_combine_allreduce_with_fewer_tokens_than_ranks():
+    """T = 5 tokens over 8 ranks: slices of one token, and ranks 5-7 own no token (they still
+    combine, publish and wait). Every rank's output must be the rank-order sum."""
+    cfg = dataclasses.replace(TPCFG, name="tp_t5_h1024_e16", T=5)
+    n = 8
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [layer.tp_shard(r, n) for r in range(n)]
+    emu = D.EmulatedTpAllReduce(cfg.T, cfg.H, n, DEV)
+    act = I.moe_activations(cfg)
+    args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+    partials, workspaces = _rank_partials_and_workspaces(shards, args)
+    outs = emu(workspaces, shards[0].sorted.capacity, cfg.K, cfg.I // n)
+    torch.cuda.synchronize()
+    want = partials[0].float()
+    for p in partials[1:]:
+        want = want + p.float()
+    for r in range(n):
+        assert torch.equal(outs[r], want.to(torch.bfloat16)), f"rank {r}"
