@@ -6,12 +6,17 @@
  * (rocm.blogs.amd.com), section "Complete MoE Implementation" (Top-K routing,
  * MoE Sorting, Blockscale FP8 MoE Computation) and section "General Linear
  * Layer" (FP8 blockscale GEMM). FP8 is OCP E4M3 "fn" (largest finite 448), not
- * the MI300X "fnuz" variant.
+ * the MI300X "fnuz" variant. The tensor- and expert-parallel entry points at the
+ * end follow the same page's TP8 run and custom all-reduce ("Performance
+ * Reproduction for AITER-Optimized in SGLang", "Other Operators") and asm_moe's
+ * expert_mask.
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller; the library never
  *     allocates, frees or keeps them. Scratch memory is passed in as
- *     `workspace`, sized by the matching *_workspace query.
+ *     `workspace`, sized by the matching *_workspace query. The multi-GPU entry
+ *     points take host arrays with one device pointer per rank, each as this GPU
+ *     addresses that rank's memory (peer memory over NVLink, or local).
  *   - Matrices are row-major; `ld*` arguments are row strides in elements.
  *   - FP8 tensors are bytes (uint8_t) holding E4M3fn codes; bf16 tensors are
  *     uint16_t holding bfloat16 bit patterns.
