@@ -16,7 +16,9 @@
  *     allocates, frees or keeps them. Scratch memory is passed in as
  *     `workspace`, sized by the matching *_workspace query. The multi-GPU entry
  *     points take host arrays with one device pointer per rank, each as this GPU
- *     addresses that rank's memory (peer memory over NVLink, or local).
+ *     addresses that rank's memory (peer memory over NVLink, or local); only the
+ *     return_rows / return_flags arrays of fused_moe_fp8_blockscale_g1u1_multi are
+ *     device arrays, because its down GEMM reads them.
  *   - Matrices are row-major; `ld*` arguments are row strides in elements.
  *   - FP8 tensors are bytes (uint8_t) holding E4M3fn codes; bf16 tensors are
  *     uint16_t holding bfloat16 bit patterns.
