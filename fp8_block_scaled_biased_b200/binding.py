@@ -57,16 +57,16 @@ _SIGNATURES = {
                                                      _c_int, _p, _c_size, _p]),
     "moe_tp_recv_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_combine_allreduce": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p,
-                                       ctypes.c_uint64, _p]),
+                                       _p]),
     "moe_combine_allreduce_emulated": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p,
-                                                ctypes.c_uint64, _p]),
+                                                _p]),
     "moe_ep_routing": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p]),
     "fused_moe_fp8_blockscale_g1u1_multi": (_c_int, [_p, _p, _c_int, _c_int, _p, _p, _p, _p, _p, _p, _c_int, _c_int,
                                                      _c_int, _c_int, _c_int, _c_size, _p, _p, _c_int, _c_int, _p,
                                                      _c_int, _p, _p, _p, _c_size, _p]),
     "moe_ep_return": (_c_int, [_p, _c_size, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p]),
-    "moe_ep_barrier": (_c_int, [_c_int, _c_int, _p, ctypes.c_uint64, _p]),
-    "moe_ep_barrier_emulated": (_c_int, [_c_int, _p, ctypes.c_uint64, _p]),
+    "moe_ep_barrier": (_c_int, [_c_int, _c_int, _p, _p]),
+    "moe_ep_barrier_emulated": (_c_int, [_c_int, _p, _p]),
     "moe_combine_pairs": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _p, _p]),
 }
 EXPORTED = tuple(_SIGNATURES)
@@ -74,9 +74,9 @@ EXPORTED = tuple(_SIGNATURES)
 NOALLOC_SCRATCH_BYTES = 64 << 20   # FP8MOE_NOALLOC_SCRATCH_BYTES in include/fp8moe.h
 TP_MAX_RANKS = 8                   # FP8MOE_TP_MAX_RANKS
 TP_FLAG_WORDS = 16                 # FP8MOE_TP_FLAG_WORDS (64-bit words per rank)
-TP_BARRIER_WORDS = 2               # FP8MOE_TP_BARRIER_WORDS
+TP_BARRIER_WORDS = 3               # FP8MOE_TP_BARRIER_WORDS (arrivals, generation, calls)
 EP_MAX_RANKS = 8                   # FP8MOE_EP_MAX_RANKS
-EP_BARRIER_WORDS = 8               # FP8MOE_EP_BARRIER_WORDS
+EP_BARRIER_WORDS = 9               # FP8MOE_EP_BARRIER_WORDS (one per rank, then the calls)
 SCALE_ROW_MAJOR = 0
 SCALE_COL_MAJOR = 1
 FP8 = torch.float8_e4m3fn
@@ -474,10 +474,10 @@ def _addresses(items, name):
     return (ctypes.c_void_p * len(addrs))(*addrs)
 
 
-def moe_combine_allreduce(workspace, capacity, T, topk, H, I, rank, recv, out, flags, barrier, epoch):
+def moe_combine_allreduce(workspace, capacity, T, topk, H, I, rank, recv, out, flags, barrier):
     """One tensor-parallel rank's fused combine + all-reduce (include/fp8moe.h). recv, out,
     flags: one device address (or tensor) per rank, as this GPU addresses that rank's buffer;
-    barrier: int64 [TP_BARRIER_WORDS] on this GPU; epoch: larger than every earlier call's."""
+    barrier: int64 [TP_BARRIER_WORDS] on this GPU (it also counts the rank's calls)."""
     _cuda(workspace, torch.uint8, "workspace")
     _cuda(barrier, torch.int64, "barrier")
     n = len(recv)
@@ -487,11 +487,11 @@ def moe_combine_allreduce(workspace, capacity, T, topk, H, I, rank, recv, out, f
         raise ValueError("barrier too small")
     rc = load_library().moe_combine_allreduce(
         _ptr(workspace), capacity, T, topk, H, I, n, rank, _addresses(recv, "recv"), _addresses(out, "out"),
-        _addresses(flags, "flags"), _ptr(barrier), epoch, _stream())
+        _addresses(flags, "flags"), _ptr(barrier), _stream())
     _check("moe_combine_allreduce", rc)
 
 
-def moe_combine_allreduce_emulated(workspaces, capacity, T, topk, H, I, recv, out, flags, barriers, epoch):
+def moe_combine_allreduce_emulated(workspaces, capacity, T, topk, H, I, recv, out, flags, barriers):
     """Every rank of moe_combine_allreduce on this GPU in one launch (the rank protocol on one
     device). Per rank r: workspaces[r] (its pairs call's workspace), recv[r] bf16 [n, Ts, H],
     out[r] bf16 [T, H], flags[r] int64 [TP_FLAG_WORDS], barriers[r] int64 [TP_BARRIER_WORDS]."""
@@ -510,7 +510,7 @@ def moe_combine_allreduce_emulated(workspaces, capacity, T, topk, H, I, recv, ou
             raise ValueError(f"rank {r}: a buffer is smaller than the call needs")
     rc = load_library().moe_combine_allreduce_emulated(
         _addresses(workspaces, "workspaces"), capacity, T, topk, H, I, n, _addresses(recv, "recv"),
-        _addresses(out, "out"), _addresses(flags, "flags"), _addresses(barriers, "barriers"), epoch, _stream())
+        _addresses(out, "out"), _addresses(flags, "flags"), _addresses(barriers, "barriers"), _stream())
     _check("moe_combine_allreduce_emulated", rc)
 
 
@@ -593,15 +593,15 @@ def moe_ep_return(workspace, capacity, Tq, topk, H, I, sorted_pairs: SortedPairs
     _check("moe_ep_return", rc)
 
 
-def moe_ep_barrier(rank, words, epoch):
+def moe_ep_barrier(rank, words):
     """Flag barrier of len(words) ranks (include/fp8moe.h); words: one address (or int64
     tensor of EP_BARRIER_WORDS) per rank."""
-    rc = load_library().moe_ep_barrier(len(words), rank, _addresses(words, "words"), epoch, _stream())
+    rc = load_library().moe_ep_barrier(len(words), rank, _addresses(words, "words"), _stream())
     _check("moe_ep_barrier", rc)
 
 
-def moe_ep_barrier_emulated(words, epoch):
-    rc = load_library().moe_ep_barrier_emulated(len(words), _addresses(words, "words"), epoch, _stream())
+def moe_ep_barrier_emulated(words):
+    rc = load_library().moe_ep_barrier_emulated(len(words), _addresses(words, "words"), _stream())
     _check("moe_ep_barrier_emulated", rc)
 
 

@@ -86,23 +86,29 @@ ep_return_kernel(const int32_t* __restrict__ sorted_ids, const int32_t* __restri
   }
 }
 
-// Flag barrier of n ranks: rank r publishes epoch in every rank's word r (release,
-// system scope), then waits until its own words q hold >= epoch for every q. The
-// stream order before it makes every earlier store of this rank (peer stores
-// included) visible to the ranks that pass it. Bounded: on expiry the device error
-// word is set. One CTA per rank: rank = rank_first + blockIdx.x.
+// Flag barrier of n ranks: rank r publishes epoch (its own count of barrier calls
+// plus one, kept in word kMaxSources of its words, so a CUDA graph replay advances
+// it like a launch) in every rank's word r (release, system scope), then waits
+// until its own words q hold >= epoch for every q. The stream order before it makes
+// every earlier store of this rank (peer stores included) visible to the ranks
+// that pass it. Bounded: on expiry the device error word is set. One CTA (one
+// warp) per rank: rank = rank_first + blockIdx.x.
+constexpr int kEpBarrierWords = kMaxSources + 1;
 struct EpBarrierArgs {
-  unsigned long long* flags[kMaxSources];   // rank p's barrier words [kMaxSources]
+  unsigned long long* flags[kMaxSources];   // rank p's barrier words [kEpBarrierWords]
   int n;
-  unsigned long long epoch;
 };
 
 __global__ void __launch_bounds__(32) ep_barrier_kernel(const __grid_constant__ EpBarrierArgs a, int rank_first) {
   const int rank = rank_first + static_cast<int>(blockIdx.x);
+  unsigned long long epoch = 0;
+  if (threadIdx.x == 0) epoch = ld_acquire_gpu_u64(a.flags[rank] + kMaxSources) + 1;
+  epoch = __shfl_sync(0xffffffffu, epoch, 0);
   __threadfence_system();
-  if (threadIdx.x < a.n) st_release_sys_u64(a.flags[threadIdx.x] + rank, a.epoch);
-  if (threadIdx.x < a.n) tp_wait_ge(a.flags[rank] + threadIdx.x, a.epoch);
+  if (threadIdx.x < a.n) st_release_sys_u64(a.flags[threadIdx.x] + rank, epoch);
+  if (threadIdx.x < a.n) tp_wait_ge(a.flags[rank] + threadIdx.x, epoch);
   __syncwarp();
+  if (threadIdx.x == 0) atomicExch(a.flags[rank] + kMaxSources, epoch);
   __threadfence_system();
 }
 

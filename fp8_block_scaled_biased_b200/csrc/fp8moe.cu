@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "common.cuh"
 #include "gemm_sm100.cuh"
@@ -793,22 +794,23 @@ size_t moe_tp_recv_bytes(int T, int H, int nranks) {
 
 }  // extern "C"
 
-static_assert(FP8MOE_TP_MAX_RANKS == kTpMaxRanks && FP8MOE_TP_FLAG_WORDS == kTpFlagWords, "header and kernel agree");
+static_assert(FP8MOE_TP_MAX_RANKS == kTpMaxRanks && FP8MOE_TP_FLAG_WORDS == kTpFlagWords &&
+                  FP8MOE_TP_BARRIER_WORDS == kTpBarrierWords,
+              "header and kernel agree");
 
 // Checks shared by the one-rank and the emulated launches: fills `a` (the peer
 // buffers, and the workspace buffers of the nlocal ranks launched here) and
 // *ctas (CTAs per rank: all of the launch must be resident at once).
 static int tp_setup(const char* name, int nranks, int T, int topk, int H, int I, size_t capacity,
                     const void* const* workspaces, const int* ranks, int nlocal, void* const* recv,
-                    void* const* out, uint64_t* const* flags, uint64_t* const* barriers, uint64_t epoch,
-                    TpArgs* a, int* ctas) {
+                    void* const* out, uint64_t* const* flags, uint64_t* const* barriers, TpArgs* a,
+                    int* ctas) {
   if (nranks < 1 || nranks > kTpMaxRanks) return fail(FP8MOE_EINVAL, "%s: nranks must be in [1, %d]", name, kTpMaxRanks);
   if (T < 1 || topk < 1 || topk > 32) return fail(FP8MOE_EINVAL, "%s: T >= 1 and topk in [1, 32] required", name);
   if (H < 128 || H % 128 || I < 128 || I % 128)
     return fail(FP8MOE_EUNSUPPORTED, "%s: H and I must be positive multiples of 128", name);
   if (static_cast<long long>(T) * topk >= (1ll << 31) || static_cast<long long>(T) * (H / 8) >= (1ll << 40))
     return fail(FP8MOE_EUNSUPPORTED, "%s: T too large", name);
-  if (epoch == 0) return fail(FP8MOE_EINVAL, "%s: epoch must be >= 1", name);
   if (!recv || !out || !flags) return fail(FP8MOE_EINVAL, "%s: null pointer argument", name);
   *a = TpArgs{};
   for (int p = 0; p < nranks; ++p) {
@@ -836,7 +838,6 @@ static int tp_setup(const char* name, int nranks, int T, int topk, int H, int I,
   a->T = T;
   a->K = topk;
   a->H = H;
-  a->epoch = epoch;
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
   int per_sm = 0;
@@ -850,11 +851,27 @@ static int tp_setup(const char* name, int nranks, int T, int topk, int H, int I,
   return FP8MOE_OK;
 }
 
+// A cooperative launch (every CTA resident at once) through cudaLaunchKernelEx, which
+// stream capture records as a cooperative kernel node of the graph.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_cooperative(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t st,
+                                      Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 static int tp_launch(const char* name, const TpArgs& a, int rank_first, int ctas, int nlocal, void* stream) {
-  void* args[] = {const_cast<TpArgs*>(&a), &rank_first, &ctas};
-  const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(tp_combine_allreduce_kernel),
-                                                    dim3(ctas * nlocal), dim3(kTpThreads), args, 0,
-                                                    static_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_cooperative(tp_combine_allreduce_kernel, dim3(ctas * nlocal), dim3(kTpThreads),
+                                           static_cast<cudaStream_t>(stream), a, rank_first, ctas);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(FP8MOE_ECUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
@@ -866,7 +883,7 @@ extern "C" {
 
 int moe_combine_allreduce(const void* workspace, size_t capacity, int T, int topk, int H, int I, int nranks,
                           int rank, void* const* recv, void* const* out, uint64_t* const* flags, uint64_t* barrier,
-                          uint64_t epoch, void* stream) {
+                          void* stream) {
   if (nranks < 1 || rank < 0 || rank >= nranks) return fail(FP8MOE_EINVAL, "moe_combine_allreduce: bad rank");
   TpArgs a;
   int ctas = 0;
@@ -874,14 +891,14 @@ int moe_combine_allreduce(const void* workspace, size_t capacity, int T, int top
   uint64_t* bars[1] = {barrier};
   const int ranks[1] = {rank};
   if (int rc = tp_setup("moe_combine_allreduce", nranks, T, topk, H, I, capacity, ws, ranks, 1, recv, out, flags,
-                        bars, epoch, &a, &ctas))
+                        bars, &a, &ctas))
     return rc;
   return tp_launch("moe_combine_allreduce", a, rank, ctas, 1, stream);
 }
 
 int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacity, int T, int topk, int H, int I,
                                    int nranks, void* const* recv, void* const* out, uint64_t* const* flags,
-                                   uint64_t* const* barriers, uint64_t epoch, void* stream) {
+                                   uint64_t* const* barriers, void* stream) {
   if (!workspaces || !barriers) return fail(FP8MOE_EINVAL, "moe_combine_allreduce_emulated: null pointer argument");
   if (nranks < 1 || nranks > kTpMaxRanks) return fail(FP8MOE_EINVAL, "moe_combine_allreduce_emulated: bad nranks");
   TpArgs a;
@@ -889,7 +906,7 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
   int ranks[kTpMaxRanks];
   for (int r = 0; r < nranks; ++r) ranks[r] = r;
   if (int rc = tp_setup("moe_combine_allreduce_emulated", nranks, T, topk, H, I, capacity, workspaces, ranks, nranks,
-                        recv, out, flags, barriers, epoch, &a, &ctas))
+                        recv, out, flags, barriers, &a, &ctas))
     return rc;
   return tp_launch("moe_combine_allreduce_emulated", a, 0, ctas, nranks, stream);
 }
@@ -897,7 +914,8 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
 }  // extern "C"
 
 // ------------------------------------------------------------------ expert-parallel dispatch and return
-static_assert(FP8MOE_EP_MAX_RANKS == kMaxSources && FP8MOE_EP_BARRIER_WORDS == kMaxSources, "header and kernels agree");
+static_assert(FP8MOE_EP_MAX_RANKS == kMaxSources && FP8MOE_EP_BARRIER_WORDS == kEpBarrierWords,
+              "header and kernels agree");
 
 extern "C" {
 
@@ -980,10 +998,9 @@ int moe_ep_return(const void* workspace, size_t capacity, int n, int Tq, int top
   return check_launch("moe_ep_return");
 }
 
-static int ep_barrier_launch(const char* name, int n, int rank_first, int ctas, uint64_t* const* words, uint64_t epoch,
+static int ep_barrier_launch(const char* name, int n, int rank_first, int ctas, uint64_t* const* words,
                              void* stream) {
   if (n < 1 || n > kMaxSources) return fail(FP8MOE_EINVAL, "%s: n must be in [1, %d]", name, kMaxSources);
-  if (epoch == 0) return fail(FP8MOE_EINVAL, "%s: epoch must be >= 1", name);
   if (!words) return fail(FP8MOE_EINVAL, "%s: null pointer argument", name);
   EpBarrierArgs a{};
   for (int p = 0; p < n; ++p) {
@@ -992,12 +1009,10 @@ static int ep_barrier_launch(const char* name, int n, int rank_first, int ctas, 
     a.flags[p] = reinterpret_cast<unsigned long long*>(words[p]);
   }
   a.n = n;
-  a.epoch = epoch;
   int sms = 0;
   if (int rc = device_setup(&sms)) return rc;
-  void* args[] = {&a, &rank_first};
-  const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(ep_barrier_kernel), dim3(ctas),
-                                                    dim3(32), args, 0, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_cooperative(ep_barrier_kernel, dim3(ctas), dim3(32), static_cast<cudaStream_t>(stream),
+                                           a, rank_first);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(FP8MOE_ECUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
@@ -1005,13 +1020,13 @@ static int ep_barrier_launch(const char* name, int n, int rank_first, int ctas, 
   return check_launch(name);
 }
 
-int moe_ep_barrier(int n, int rank, uint64_t* const* words, uint64_t epoch, void* stream) {
+int moe_ep_barrier(int n, int rank, uint64_t* const* words, void* stream) {
   if (rank < 0 || rank >= n) return fail(FP8MOE_EINVAL, "moe_ep_barrier: bad rank");
-  return ep_barrier_launch("moe_ep_barrier", n, rank, 1, words, epoch, stream);
+  return ep_barrier_launch("moe_ep_barrier", n, rank, 1, words, stream);
 }
 
-int moe_ep_barrier_emulated(int n, uint64_t* const* words, uint64_t epoch, void* stream) {
-  return ep_barrier_launch("moe_ep_barrier_emulated", n, 0, n, words, epoch, stream);
+int moe_ep_barrier_emulated(int n, uint64_t* const* words, void* stream) {
+  return ep_barrier_launch("moe_ep_barrier_emulated", n, 0, n, words, stream);
 }
 
 int moe_combine_pairs(const uint16_t* rows, const void* flag_region, int T, int topk, int H, uint16_t* out,

@@ -14,7 +14,10 @@
 //      rounded to bf16 once, is stored into the receive buffer of the rank p that
 //      owns t's slice (recv_p[r][t - p*Ts], a store over NVLink when p != r);
 //   2. the rank's CTAs meet at a barrier (in this GPU's memory), then one thread
-//      publishes flag_p[0][r] = epoch to every rank p (release, system scope);
+//      publishes flag_p[0][r] = epoch to every rank p (release, system scope),
+//      epoch being the rank's call count plus one (a counter kept in its barrier
+//      words, so that no value comes from the host and a CUDA graph replay of the
+//      call advances it like a launch does);
 //   3. each rank waits for flag_r[0][q] >= epoch from every q (acquire, system
 //      scope), then sums its slice's n partial rows in rank order q = 0..n-1 in
 //      fp32, rounds to bf16 once and stores the row into every rank's output
@@ -41,6 +44,7 @@ namespace fp8moe {
 constexpr int kTpMaxRanks = 8;
 constexpr int kTpThreads = 256;
 constexpr int kTpFlagWords = 2 * kTpMaxRanks;   // per rank: [phase][source rank]
+constexpr int kTpBarrierWords = 3;               // per rank: arrivals, generation, calls
 constexpr int kTpBatch = 4;                      // pair rows loaded before they are added
 
 struct TpArgs {
@@ -48,13 +52,12 @@ struct TpArgs {
   const __nv_bfloat16* ystage[kTpMaxRanks];   // weighted pair rows [T*K, H]
   const uint8_t* pair_flag[kTpMaxRanks];       // [T*K]: 1 where the pair is listed
   const int* n_present[kTpMaxRanks];           // distinct listed pairs
-  unsigned long long* barrier[kTpMaxRanks];    // {arrivals, generation}
+  unsigned long long* barrier[kTpMaxRanks];    // {arrivals, generation, calls}
   // per rank p, as this GPU addresses it (peer memory for p != own rank)
   __nv_bfloat16* recv[kTpMaxRanks];            // [n][Ts][H]
   __nv_bfloat16* out[kTpMaxRanks];             // [T][H]
   unsigned long long* flags[kTpMaxRanks];      // [kTpFlagWords]
   int nranks, T, K, H;
-  unsigned long long epoch;
 };
 
 __device__ __forceinline__ void st_release_sys_u64(unsigned long long* p, unsigned long long v) {
@@ -142,6 +145,12 @@ tp_combine_allreduce_kernel(const __grid_constant__ TpArgs a, int rank_first, in
   const int Ts = (T + n - 1) / n;
   const long long stride = static_cast<long long>(ctas_per_rank) * kTpThreads;
   const long long first = static_cast<long long>(cta) * kTpThreads + threadIdx.x;
+  // this call's epoch: read by every CTA before the first barrier, advanced by CTA 0
+  // after it (when no CTA of this launch reads the counter any more)
+  __shared__ unsigned long long s_epoch;
+  if (threadIdx.x == 0) s_epoch = ld_acquire_gpu_u64(a.barrier[rank] + 2) + 1;
+  __syncthreads();
+  const unsigned long long epoch = s_epoch;
 
   // 1. combine this rank's pair rows per token; the bf16 partial goes to the slice owner
   const __nv_bfloat16* y = a.ystage[rank];
@@ -177,10 +186,10 @@ tp_combine_allreduce_kernel(const __grid_constant__ TpArgs a, int rank_first, in
 
   // 2. publish: this rank's partials are in every owner's receive buffer
   tp_rank_barrier(a.barrier[rank], ctas_per_rank);
-  if (cta == 0 && threadIdx.x < n) st_release_sys_u64(a.flags[threadIdx.x] + rank, a.epoch);
+  if (cta == 0 && threadIdx.x < n) st_release_sys_u64(a.flags[threadIdx.x] + rank, epoch);
 
   // 3. reduce this rank's slice in rank order and write it into every rank's output
-  if (threadIdx.x < n) tp_wait_ge(a.flags[rank] + threadIdx.x, a.epoch);
+  if (threadIdx.x < n) tp_wait_ge(a.flags[rank] + threadIdx.x, epoch);
   __syncthreads();
   __threadfence_system();
   const int t0 = rank * Ts;
@@ -208,9 +217,10 @@ tp_combine_allreduce_kernel(const __grid_constant__ TpArgs a, int rank_first, in
 
   // 4. publish the slice; leave once every rank has written this rank's output
   tp_rank_barrier(a.barrier[rank], ctas_per_rank);
-  if (cta == 0 && threadIdx.x < n) st_release_sys_u64(a.flags[threadIdx.x] + kTpMaxRanks + rank, a.epoch);
+  if (cta == 0 && threadIdx.x < n) st_release_sys_u64(a.flags[threadIdx.x] + kTpMaxRanks + rank, epoch);
   if (cta == 0) {
-    if (threadIdx.x < n) tp_wait_ge(a.flags[rank] + kTpMaxRanks + threadIdx.x, a.epoch);
+    if (threadIdx.x < n) tp_wait_ge(a.flags[rank] + kTpMaxRanks + threadIdx.x, epoch);
+    if (threadIdx.x == 0) atomicExch(a.barrier[rank] + 2, epoch);   // the next call's base
     __syncthreads();
     __threadfence_system();
   }

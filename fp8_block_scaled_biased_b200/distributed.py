@@ -113,8 +113,10 @@ class TpPeerAllReduce:
     """One rank's buffers for the combine fused with the all-reduce (moe_combine_allreduce):
     the receive buffer, the output and the flag words in one allocation of torch's symmetric
     memory, exchanged over the group so that every rank's buffers are addressable from every
-    GPU (over NVLink); the CTA barrier words in this GPU's memory; the call counter (epoch).
-    Every rank of the group must construct it and then make the same calls."""
+    GPU (over NVLink); the CTA barrier words (which also count the calls) in this GPU's
+    memory. Every rank of the group must construct it and then make the same calls; nothing
+    is passed from the host per call, so a forward holding it can be captured in a CUDA
+    graph."""
 
     def __init__(self, T: int, H: int, group=None, device=None):
         import torch.distributed._symmetric_memory as symm
@@ -132,7 +134,6 @@ class TpPeerAllReduce:
         self.flags = [b + L.flags for b in bases]
         self.out = self.buf[L.out:L.out + T * H * 2].view(torch.bfloat16).view(T, H)
         self.barrier = torch.zeros(B.TP_BARRIER_WORDS, dtype=torch.int64, device=dev)
-        self.epoch = 0
         torch.cuda.synchronize(dev)
         if dist.is_initialized() and n > 1:
             dist.barrier(group)            # every rank's flags are zero before any rank's first call
@@ -140,10 +141,14 @@ class TpPeerAllReduce:
     def __call__(self, workspace, capacity: int, topk: int, I: int) -> torch.Tensor:
         """Combine this rank's pair rows (left in `workspace` by the pairs call) and all-reduce
         them; returns this rank's output buffer bf16 [T, H] (rewritten by the next call)."""
-        self.epoch += 1
         B.moe_combine_allreduce(workspace, capacity, self.T, topk, self.H, I, self.rank, self.recv, self.outs,
-                                self.flags, self.barrier, self.epoch)
+                                self.flags, self.barrier)
         return self.out
+
+    @property
+    def calls(self) -> int:
+        """Calls made so far (the device-side counter; reading it synchronises)."""
+        return int(self.barrier[2])
 
 
 class EmulatedTpAllReduce:
@@ -160,14 +165,20 @@ class EmulatedTpAllReduce:
         self.out = [torch.empty(T, H, dtype=torch.bfloat16, device=device) for _ in range(n)]
         self.flags = [torch.zeros(B.TP_FLAG_WORDS, dtype=torch.int64, device=device) for _ in range(n)]
         self.barriers = [torch.zeros(B.TP_BARRIER_WORDS, dtype=torch.int64, device=device) for _ in range(n)]
-        self.epoch = 0
 
     def __call__(self, workspaces, capacity: int, topk: int, I: int):
         """workspaces[r]: rank r's pairs-call workspace. Returns the n ranks' outputs."""
-        self.epoch += 1
         B.moe_combine_allreduce_emulated(workspaces, capacity, self.T, topk, self.H, I, self.recv, self.out,
-                                         self.flags, self.barriers, self.epoch)
+                                         self.flags, self.barriers)
         return self.out
+
+    @property
+    def calls(self) -> int:
+        """Calls made so far, by every rank's device-side counter (which must agree)."""
+        counts = {int(b[2]) for b in self.barriers}
+        if len(counts) != 1:
+            raise RuntimeError(f"the ranks' call counters disagree: {sorted(counts)}")
+        return counts.pop()
 
 
 class TensorParallelMoE:
@@ -492,7 +503,7 @@ class ExpertParallelPeerMoE:
         addrs = [EpRankBuffers.addresses(b, T, cfg.K, cfg.H) for b in bases]
         peers = {k: [a[k] for a in addrs] for k in addrs[0]}
         self.rank = EpPeerRank(cfg, shard, n, r, T, EpRankBuffers(self.buf, T, cfg.K, cfg.H), peers)
-        self.r, self.epoch = r, 0
+        self.r = r
         torch.cuda.synchronize(dev)
         if dist.is_initialized() and n > 1:
             dist.barrier(group)            # every rank's barrier words are zero before the first forward
@@ -501,12 +512,15 @@ class ExpertParallelPeerMoE:
         """This rank's tokens -> its output bf16 [T, H] (a buffer the next forward rewrites)."""
         rk = self.rank
         rk.publish(logits, bias, x)
-        self.epoch += 1
-        B.moe_ep_barrier(self.r, rk.peers["barrier"], self.epoch)
+        B.moe_ep_barrier(self.r, rk.peers["barrier"])
         rk.compute()
-        self.epoch += 1
-        B.moe_ep_barrier(self.r, rk.peers["barrier"], self.epoch)
+        B.moe_ep_barrier(self.r, rk.peers["barrier"])
         return rk.combine()
+
+    @property
+    def barriers_passed(self) -> int:
+        """Barrier calls made so far (this rank's device-side counter; reading synchronises)."""
+        return int(self.rank.mine.barrier[B.EP_BARRIER_WORDS - 1])
 
 
 class EmulatedExpertParallel:
@@ -522,7 +536,7 @@ class EmulatedExpertParallel:
         peers = {k: [a[k] for a in addrs] for k in addrs[0]}
         self.ranks = [EpPeerRank(cfg, sh, n, r, T, EpRankBuffers(self.bufs[r], T, cfg.K, cfg.H), peers,
                                  return_in_gemm) for r, sh in enumerate(shards)]
-        self.peers, self.epoch = peers, 0
+        self.peers = peers
 
     def forward(self, inputs):
         """inputs[r] = (logits, bias, x) of rank r; returns the n ranks' outputs."""
@@ -530,10 +544,16 @@ class EmulatedExpertParallel:
             raise ValueError(f"one input set per rank ({len(self.ranks)}), got {len(inputs)}")
         for rk, args in zip(self.ranks, inputs):
             rk.publish(*args)
-        self.epoch += 1
-        B.moe_ep_barrier_emulated(self.peers["barrier"], self.epoch)
+        B.moe_ep_barrier_emulated(self.peers["barrier"])
         for rk in self.ranks:
             rk.compute()
-        self.epoch += 1
-        B.moe_ep_barrier_emulated(self.peers["barrier"], self.epoch)
+        B.moe_ep_barrier_emulated(self.peers["barrier"])
         return [rk.combine() for rk in self.ranks]
+
+    @property
+    def barriers_passed(self) -> int:
+        """Barrier calls made so far, by every rank's device-side counter (which must agree)."""
+        counts = {int(rk.mine.barrier[B.EP_BARRIER_WORDS - 1]) for rk in self.ranks}
+        if len(counts) != 1:
+            raise RuntimeError(f"the ranks' barrier counters disagree: {sorted(counts)}")
+        return counts.pop()

@@ -429,26 +429,27 @@ int fused_moe_fp8_blockscale_g1u1_pairs(const uint8_t* a8, const uint8_t* w1,
  *           as this GPU addresses that rank's memory: peer memory mapped by
  *           CUDA IPC or virtual memory management, or local memory for this rank)
  * barrier   FP8MOE_TP_BARRIER_WORDS 64-bit words in this GPU's memory, zero
- *           before the first call (the rank's CTAs meet there)
- * epoch     larger than the epoch of every earlier call on these flags (for
- *           example 1, 2, 3, ...); every rank of a call passes the same epoch
+ *           before the first call: where the rank's CTAs meet, and the rank's
+ *           count of calls, which gives each call its flag value (epoch). No
+ *           value comes from the host, so the call can be captured in a CUDA
+ *           graph: every replay advances the count as a launch does.
  * Ownership: every buffer belongs to the caller; nothing is allocated. Every rank
  * must make the same sequence of calls; a rank that does not arrive leaves the
  * others waiting until the bounded wait (about 2 s) expires, which sets
  * FP8MOE_DEVERR_TIMEOUT, after which the output is unspecified and flags and
- * barrier must be zeroed again before the next call. out may be read by later
- * work on the same stream; a second call overwrites it.
+ * barrier words must be zeroed again on every rank before the next call. out may
+ * be read by later work on the same stream; a second call overwrites it.
  * Returns FP8MOE_EINVAL for a bad rank, size, alignment or null pointer and
  * FP8MOE_ECUDA when the cooperative launch fails.
  */
 #define FP8MOE_TP_MAX_RANKS 8
 #define FP8MOE_TP_FLAG_WORDS 16
-#define FP8MOE_TP_BARRIER_WORDS 2
+#define FP8MOE_TP_BARRIER_WORDS 3
 size_t moe_tp_recv_bytes(int T, int H, int nranks);
 int moe_combine_allreduce(const void* workspace, size_t capacity, int T, int topk,
                           int H, int I, int nranks, int rank, void* const* recv,
                           void* const* out, uint64_t* const* flags, uint64_t* barrier,
-                          uint64_t epoch, void* stream);
+                          void* stream);
 
 /*
  * All nranks ranks of moe_combine_allreduce on this one GPU, in one cooperative
@@ -462,7 +463,7 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
                                    int T, int topk, int H, int I, int nranks,
                                    void* const* recv, void* const* out,
                                    uint64_t* const* flags, uint64_t* const* barriers,
-                                   uint64_t epoch, void* stream);
+                                   void* stream);
 
 /*
  * Expert parallelism over peer (NVLink) memory: the dispatch and the return as
@@ -497,7 +498,7 @@ int moe_combine_allreduce_emulated(const void* const* workspaces, size_t capacit
  * Ownership: every buffer belongs to the caller; nothing is allocated.
  */
 #define FP8MOE_EP_MAX_RANKS 8
-#define FP8MOE_EP_BARRIER_WORDS 8
+#define FP8MOE_EP_BARRIER_WORDS 9
 
 /* ids_out int32 [n*Tq, topk]: id - e0 for the owner's experts, ne for another
  * rank's, -1 for an id outside [0, E) (which the sort drops and flags);
@@ -541,18 +542,19 @@ int moe_ep_return(const void* workspace, size_t capacity, int n, int Tq, int top
                   const int32_t* num_valid_ids, void* const* rows,
                   void* const* pair_flags, void* stream);
 
-/* Flag barrier: rank `rank` stores epoch into word `rank` of every rank's
- * FP8MOE_EP_BARRIER_WORDS 64-bit words (zero before the first call; 8-byte
- * aligned) and waits until its own words 0..n-1 hold >= epoch. epoch grows by at
- * least one per barrier; every rank passes the same sequence. The stream's earlier
- * work (peer stores included) is visible to every rank past the barrier. A rank
- * that never arrives leaves the others waiting until the bounded wait (about 2 s)
- * expires: FP8MOE_DEVERR_TIMEOUT, after which the words must be zeroed again. The
- * _emulated form runs all n ranks' barriers on this GPU in one launch. */
-int moe_ep_barrier(int n, int rank, uint64_t* const* words, uint64_t epoch,
-                   void* stream);
-int moe_ep_barrier_emulated(int n, uint64_t* const* words, uint64_t epoch,
-                            void* stream);
+/* Flag barrier. Every rank has FP8MOE_EP_BARRIER_WORDS 64-bit words (zero before
+ * the first call; 8-byte aligned): one per rank, then its own count of barrier
+ * calls. Rank `rank` takes epoch = its count + 1, stores it into word `rank` of
+ * every rank's words, waits until its own words 0..n-1 hold >= epoch and stores
+ * the new count. No value comes from the host, so the call can be captured in a
+ * CUDA graph. Every rank makes the same sequence of barrier calls. The stream's
+ * earlier work (peer stores included) is visible to every rank past the barrier.
+ * A rank that never arrives leaves the others waiting until the bounded wait
+ * (about 2 s) expires: FP8MOE_DEVERR_TIMEOUT, after which every rank's words must
+ * be zeroed again. The _emulated form runs all n ranks' barriers on this GPU in
+ * one launch. */
+int moe_ep_barrier(int n, int rank, uint64_t* const* words, void* stream);
+int moe_ep_barrier_emulated(int n, uint64_t* const* words, void* stream);
 
 /* out bf16 [T, H] = the combine of fused_moe_fp8_blockscale_g1u1 over pair rows
  * (bf16 [T*topk, H]) and a flag region laid out as the workspace's: a 16-byte

@@ -184,26 +184,28 @@ def test_tile_weights_and_tiled_fused_call_reject_bad_arguments(lib):
 
 
 def test_multi_gpu_entry_points_reject_bad_arguments(lib):
-    """The tensor- and expert-parallel entry points check ranks, sizes, epochs and pointers
-    on the host and return a status before touching a GPU."""
+    """The tensor- and expert-parallel entry points check ranks, sizes and pointers on the
+    host and return a status before touching a GPU."""
     p = ctypes.c_void_p(16)
     one = (ctypes.c_void_p * 1)(16)
     nine = (ctypes.c_void_p * 9)(*([16] * 9))
     Ts = -(-300 // 8)
     assert lib.moe_tp_recv_bytes(300, 1024, 8) == 8 * Ts * 1024 * 2
     assert lib.moe_tp_recv_bytes(300, 1024, 9) == 0 and lib.moe_tp_recv_bytes(300, 1024, 0) == 0
-    # combine + all-reduce: nranks, rank, epoch
-    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1024, 512, 0, 0, one, one, one, p, 1, None) == 1
-    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1024, 512, 1, 1, one, one, one, p, 1, None) == 1
-    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1024, 512, 1, 0, one, one, one, p, 0, None) == 1
-    assert lib.moe_combine_allreduce_emulated(None, 1 << 20, 300, 4, 1024, 512, 1, one, one, one, one, 1, None) == 1
-    assert lib.moe_combine_allreduce_emulated(nine, 1 << 20, 300, 4, 1024, 512, 9, nine, nine, nine, nine, 1,
+    # combine + all-reduce: nranks, rank, sizes, pointers
+    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1024, 512, 0, 0, one, one, one, p, None) == 1
+    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1024, 512, 1, 1, one, one, one, p, None) == 1
+    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1000, 512, 1, 0, one, one, one, p, None) == 2   # H % 128
+    assert lib.moe_combine_allreduce(p, 1 << 20, 300, 4, 1024, 512, 1, 0, None, one, one, p, None) == 1
+    assert lib.moe_combine_allreduce_emulated(None, 1 << 20, 300, 4, 1024, 512, 1, one, one, one, one, None) == 1
+    assert lib.moe_combine_allreduce_emulated(nine, 1 << 20, 300, 4, 1024, 512, 9, nine, nine, nine, nine,
                                               None) == 1
-    # expert parallelism: ranks, expert ranges, epochs, sizes
+    # expert parallelism: ranks, expert ranges, sizes
     assert lib.moe_ep_routing(one, one, 0, 10, 4, 16, 0, 4, p, p, None) == 1
     assert lib.moe_ep_routing(one, one, 1, 10, 4, 16, 14, 4, p, p, None) == 1     # e0 + ne > E
-    assert lib.moe_ep_barrier(2, 2, one, 1, None) == 1
-    assert lib.moe_ep_barrier(1, 0, one, 0, None) == 1
+    assert lib.moe_ep_barrier(2, 2, one, None) == 1
+    assert lib.moe_ep_barrier(9, 0, nine, None) == 1
+    assert lib.moe_ep_barrier(1, 0, None, None) == 1
     assert lib.moe_ep_return(p, 1 << 20, 9, 10, 4, 1024, 512, p, p, nine, nine, None) == 1
     assert lib.moe_combine_pairs(p, p, 10, 0, 1024, p, None) == 1
     assert lib.moe_combine_pairs(p, p, 10, 4, 1004, p, None) == 1          # H % 8 != 0

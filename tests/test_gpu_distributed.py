@@ -80,8 +80,9 @@ def test_emulated_tp_combine_allreduce_is_the_rank_order_sum_of_the_partials(n):
     """Every rank of the fused combine + all-reduce on one GPU (one cooperative launch, each
     rank's CTAs running the one-rank code through the shared flags): every rank's output must
     equal, bit for bit, bf16 of the fp32 sum in rank order of the ranks' bf16 partials (each
-    the fused call's own combine of that rank's pair rows), over three calls (epochs) whose
-    inputs alternate; and the result must match the whole layer's oracle."""
+    the fused call's own combine of that rank's pair rows), over three calls whose inputs
+    alternate (each call's flag value comes from the ranks' device-side call counters); and
+    the result must match the whole layer's oracle."""
     cfg = TPCFG
     layer = MoELayer(cfg, DEV).load_synthetic_weights()
     shards = [layer.tp_shard(r, n) for r in range(n)]
@@ -104,7 +105,7 @@ def test_emulated_tp_combine_allreduce_is_the_rank_order_sum_of_the_partials(n):
         if call < 2:
             ref, _, _ = oracle_moe_rows(cfg, act, None)
             assert_moe_close(outs[0], ref)
-    assert emu.epoch == 3
+    assert emu.calls == 3
 
 
 def test_tp_combine_allreduce_bounded_wait_runs_out_without_its_peer():
@@ -123,7 +124,7 @@ def test_tp_combine_allreduce_bounded_wait_runs_out_without_its_peer():
     flags = [torch.zeros(B.TP_FLAG_WORDS, dtype=torch.int64, device=DEV) for _ in range(2)]
     barrier = torch.zeros(B.TP_BARRIER_WORDS, dtype=torch.int64, device=DEV)
     B.moe_combine_allreduce(ws, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I // 2, 0, recv, out, flags,
-                            barrier, 1)
+                            barrier)
     assert B.device_status() & 1                       # FP8MOE_DEVERR_TIMEOUT (read and cleared)
     assert B.device_status() == 0
     assert int(flags[1][0]) == 1 and int(flags[0][0]) == 1    # rank 0 published its partials to both
@@ -137,15 +138,15 @@ def test_tp_combine_allreduce_rejects_bad_arguments():
     shard = MoELayer(cfg, DEV).tp_shard(0, 1)
     t = torch.zeros(16, dtype=torch.int64, device=DEV)
     buf = torch.zeros(1 << 20, dtype=torch.bfloat16, device=DEV)
-    with pytest.raises(B.Fp8MoeError):                 # epoch 0
-        B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I, 0, [buf], [buf],
-                                [t], t, 0)
+    with pytest.raises(B.Fp8MoeError):                 # H not a multiple of 128
+        B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H - 8, cfg.I, 0, [buf],
+                                [buf], [t], t)
     with pytest.raises(B.Fp8MoeError):                 # rank outside [0, nranks)
         B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I, 1, [buf], [buf],
-                                [t], t, 1)
+                                [t], t)
     with pytest.raises(ValueError):                    # more ranks than the protocol takes
         B.moe_combine_allreduce(shard.workspace, shard.sorted.capacity, cfg.T, cfg.K, cfg.H, cfg.I, 0, [buf] * 9,
-                                [buf] * 9, [t] * 9, t, 1)
+                                [buf] * 9, [t] * 9, t)
     assert B.device_status() == 0
 
 
@@ -177,7 +178,7 @@ def test_one_rank_peer_all_reduce_through_symmetric_memory(tmp_path):
             got = tp.forward(*args)
             torch.cuda.synchronize()
             assert torch.equal(got, want)
-        assert tp.peer.epoch == 2
+        assert tp.peer.calls == 2
         del tp, got
         gc.collect()
         torch.cuda.synchronize()
@@ -209,21 +210,20 @@ def test_emulated_peer_expert_parallel_equals_the_one_gpu_layer(cfg, n):
         torch.cuda.synchronize()
         for r in range(n):
             assert torch.equal(outs[r], wants[r]), f"forward {call}, rank {r}"
-    assert emu.epoch == 4
+    assert emu.barriers_passed == 4
 
 
 def test_ep_barrier_bounded_wait_runs_out_without_its_peer():
     """Rank 0 of 2 at the flag barrier alone: rank 1's word is never set, the bounded wait
     expires (about 2 s), FP8MOE_DEVERR_TIMEOUT is raised and the context stays usable."""
     words = [torch.zeros(B.EP_BARRIER_WORDS, dtype=torch.int64, device=DEV) for _ in range(2)]
-    B.moe_ep_barrier(0, words, 1)
+    B.moe_ep_barrier(0, words)
     assert B.device_status() & 1
     assert B.device_status() == 0
     assert int(words[0][0]) == 1 and int(words[1][0]) == 1     # rank 0 published to both
+    assert int(words[0][B.EP_BARRIER_WORDS - 1]) == 1          # and counted its call
     with pytest.raises(B.Fp8MoeError):
-        B.moe_ep_barrier(2, words, 2)                           # rank outside [0, n)
-    with pytest.raises(B.Fp8MoeError):
-        B.moe_ep_barrier(0, words, 0)                           # epoch 0
+        B.moe_ep_barrier(2, words)                              # rank outside [0, n)
 
 
 def test_one_rank_peer_expert_parallel_through_symmetric_memory(tmp_path):
@@ -242,7 +242,7 @@ def test_one_rank_peer_expert_parallel_through_symmetric_memory(tmp_path):
             got = ep.forward(*args)
             torch.cuda.synchronize()
             assert torch.equal(got, want)
-        assert ep.epoch == 4
+        assert ep.barriers_passed == 4
         del ep, got
         gc.collect()
         torch.cuda.synchronize()
@@ -314,3 +314,82 @@ def test_emulated_tp_combine_allreduce_with_fewer_tokens_than_ranks():
         want = want + p.float()
     for r in range(n):
         assert torch.equal(outs[r], want.to(torch.bfloat16)), f"rank {r}"
+
+
+# ---------------------------------------------------------------- the peer forms inside CUDA graphs
+def test_tp_combine_allreduce_replays_in_a_cuda_graph():
+    """The ranks' forwards and the fused combine + all-reduce captured in one CUDA graph: no
+    value comes from the host per call (each call's flag value is the ranks' device-side call
+    count plus one), so every replay runs the protocol afresh. Two input sets alternate between
+    replays; every rank's output must be that set's rank-order sum each time."""
+    cfg, n = TPCFG, 4
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [layer.tp_shard(r, n) for r in range(n)]
+    emu = D.EmulatedTpAllReduce(cfg.T, cfg.H, n, DEV)
+    cap, Is = shards[0].sorted.capacity, cfg.I // n
+    sets, wants = [], []
+    for seed in (cfg.seed, cfg.seed + 1):
+        act = I.moe_activations(dataclasses.replace(cfg, seed=seed))
+        args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+        want = None
+        for sh in shards:
+            p = sh.forward(*args).float()
+            want = p if want is None else want + p
+        sets.append(args)
+        wants.append(want.to(torch.bfloat16))
+    bufs = tuple(t.clone() for t in sets[0])
+
+    def step():
+        return emu([sh.forward_pairs(*bufs) for sh in shards], cap, cfg.K, Is)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        outs = step()
+    for i in range(4):
+        for b, a in zip(bufs, sets[i % 2]):
+            b.copy_(a)
+        graph.replay()
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert torch.equal(outs[r], wants[i % 2]), f"replay {i}, rank {r}"
+    assert emu.calls == 5                               # one eager call and four replays
+    del graph
+
+
+def test_peer_expert_parallel_replays_in_a_cuda_graph():
+    """The peer-memory expert-parallel forward of all ranks (routing read across ranks, the
+    pulled gather, the rows stored into their origins by the down GEMM, both barriers) captured
+    in one CUDA graph and replayed with alternating inputs: every rank's output equals the
+    one-GPU layer's for its tokens on every replay."""
+    cfg, n = EP_HOT, 4
+    layer = MoELayer(cfg, DEV).load_synthetic_weights()
+    shards = [D.ExpertShard(cfg, *D.ep_expert_range(cfg.E, r, n), DEV).load_synthetic_weights() for r in range(n)]
+    emu = D.EmulatedExpertParallel(cfg, shards, cfg.T, DEV)
+    sets, wants = [], []
+    for call in range(2):
+        inputs, want = [], []
+        for r in range(n):
+            act = I.moe_activations(dataclasses.replace(cfg, seed=cfg.seed + 10 * r + 100 * call))
+            args = (act.logits.to(DEV), act.bias.to(DEV), act.x.to(DEV))
+            inputs.append(args)
+            want.append(layer.forward(*args).clone())
+        sets.append(inputs)
+        wants.append(want)
+    bufs = [tuple(t.clone() for t in args) for args in sets[0]]
+    emu.forward(bufs)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        outs = emu.forward(bufs)
+    for i in range(4):
+        for rb, ra in zip(bufs, sets[i % 2]):
+            for b, a in zip(rb, ra):
+                b.copy_(a)
+        graph.replay()
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert torch.equal(outs[r], wants[i % 2][r]), f"replay {i}, rank {r}"
+    assert emu.barriers_passed == 10                    # two barriers per forward, five forwards
+    del graph
