@@ -100,6 +100,23 @@ def test_routing_ties_resolve_like_the_oracle(E, G, TG, K):
     assert torch.equal(w.cpu().view(torch.int32), w_ref.view(torch.int32))
 
 
+@pytest.mark.parametrize("E,G,TG,K", [(512, 16, 4, 32), (512, 1, 1, 32), (384, 32, 32, 32)],
+                         ids=["e512_g16_k32", "e512_g1_k32", "e384_g32_k32"])
+def test_routing_at_the_size_limits(E, G, TG, K):
+    """The routing kernel's limits: 512 experts (16 per lane), topk 32, 32 groups, and a group
+    size (12) that takes the kernel's generic experts-per-lane path."""
+    g = torch.Generator().manual_seed(E * K + G)
+    T = 300
+    logits = torch.randn(T, E, generator=g) * 2
+    bias = torch.randn(E, generator=g) * 0.1
+    w = torch.empty(T, K, device=DEV)
+    ids = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    B.moe_biased_grouped_topk(logits.to(DEV), bias.to(DEV), w, ids, G, TG, True, 2.5)
+    w_ref, ids_ref = O.biased_grouped_topk(logits, bias, K, G, TG, True, 2.5)
+    assert torch.equal(ids.cpu(), ids_ref)
+    assert torch.equal(w.cpu().view(torch.int32), w_ref.view(torch.int32))
+
+
 # ---------------------------------------------------------------- S2 align/sort
 @pytest.mark.parametrize("cfg,block_m", [(I.TINY, 4), (I.TINY, 128), (I.DECODE, 128), (I.DECODE, 16),
                                          (I.PREFILL, 128), (I.PREFILL, 64), (I.SKEWED, 128)],
@@ -118,6 +135,22 @@ def test_sort_bit_exact(cfg, block_m):
     assert torch.equal(sp.sorted_weights[:nv].cpu().view(torch.int32), sw.view(torch.int32))
     assert torch.equal(sp.sorted_expert_ids[: nv // block_m].cpu(), se)
     assert (sp.sorted_ids[nv:] == -5).all() and (sp.sorted_expert_ids[nv // block_m:] == -5).all()
+
+
+@pytest.mark.parametrize("T", [30, 100], ids=["one_chunk", "four_chunks"])
+def test_sort_at_the_size_limits(T):
+    """1024 experts (the sort's limit) and topk 32: 960 pairs take the one-CTA path, 3200 the
+    count + scatter path; both bit-exact against the oracle."""
+    E, K = 1024, 32
+    g = torch.Generator().manual_seed(T)
+    ids = torch.stack([torch.randperm(E, generator=g)[:K] for _ in range(T)]).to(torch.int32)
+    w = torch.rand(T, K, generator=g)
+    sp = B.moe_align_sort(ids.to(DEV), w.to(DEV), E, 128)
+    sid, sw, se, nv = O.align_sort(ids, w, E, 128)
+    assert sp.num_valid_ids.item() == nv
+    assert torch.equal(sp.sorted_ids[:nv].cpu(), sid)
+    assert torch.equal(sp.sorted_weights[:nv].cpu().view(torch.int32), sw.view(torch.int32))
+    assert torch.equal(sp.sorted_expert_ids[: nv // 128].cpu(), se)
 
 
 def test_sort_empty_and_single_token():
@@ -258,9 +291,12 @@ SKEW_SMALL = I.MoEConfig("skew_t512_h512_e64", T=512, H=512, E=64, G=8, TG=4, K=
 ODD_ONE = I.MoEConfig("odd_t1_h384_e8_k1", T=1, H=384, E=8, G=1, TG=1, K=1, I=128, renorm=False, scale=1.0, seed=3)
 ODD_E24 = I.MoEConfig("odd_t37_h640_e24_k5", T=37, H=640, E=24, G=4, TG=3, K=5, I=384, seed=4)
 FEW_EXPERTS = I.MoEConfig("few_t300_h256_e6_k2", T=300, H=256, E=6, G=2, TG=1, K=2, I=256, seed=5)
+# topk at its limit (32): every token picks half the experts
+TOPK32 = I.MoEConfig("topk32_t40_h256_e64", T=40, H=256, E=64, G=1, TG=1, K=32, I=256, seed=8)
 
 
-@pytest.mark.parametrize("cfg", [I.TINY, MID, SKEW_SMALL, ODD_ONE, ODD_E24, FEW_EXPERTS], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [I.TINY, MID, SKEW_SMALL, ODD_ONE, ODD_E24, FEW_EXPERTS, TOPK32],
+                         ids=lambda c: c.name)
 def test_fused_moe_full_small_layers(cfg):
     layer = MoELayer(cfg, DEV).load_synthetic_weights()
     act = I.moe_activations(cfg)
