@@ -143,3 +143,71 @@ def gemm_inputs(cfg: GemmConfig, device="cpu"):
     a = (torch.randn(cfg.M, cfg.K, generator=g, device=device) * cfg.a_std).to(torch.bfloat16)
     b = torch.randn(cfg.N, cfg.K, generator=g, device=device) * cfg.b_std
     return a, b
+
+
+# ---------------------------------------------------------------------------
+# MLA decode (section "Attention Mechanisms", "MLA For Decode")
+# ---------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class MlaConfig:
+    """A decode batch of multi-head latent attention over a paged KV buffer.
+
+    L is the number of cached tokens of every sequence (an int) or of each one (a
+    tuple of B ints, 0 allowed)."""
+    name: str
+    B: int
+    Hq: int
+    L: int | tuple
+    page_size: int = 1
+    Dk: int = 576
+    Dv: int = 512
+    q_std: float = 1.0
+    kv_std: float = 1.0
+    seed: int = 0
+
+    def lengths(self) -> list[int]:
+        return [self.L] * self.B if isinstance(self.L, int) else list(self.L)
+
+
+# The pages' decode benchmark (bench_one_batch: batch 64, 512 input tokens, 32 output
+# tokens, --tp 8): DeepSeek-R1's 128 query heads split over 8 GPUs, SGLang's page
+# size of 1, and the KV length of the last decode step.
+MLA_DECODE = MlaConfig("mla_decode_b64_h16_l544", B=64, Hq=16, L=544)
+# The same batch with an 8K context: 604 MB of KV, more than L2.
+MLA_LONG = MlaConfig("mla_decode_b64_h16_l8192", B=64, Hq=16, L=8192)
+MLA_CONFIGS = {c.name: c for c in (MLA_DECODE, MLA_LONG)}
+
+
+@dataclass
+class MlaInputs:
+    q: torch.Tensor                  # bf16 [B, Hq, Dk]
+    kv_buffer: torch.Tensor          # bf16 [pages, page_size, 1, Dk]
+    kv_indptr: torch.Tensor          # int32 [B + 1]
+    kv_indices: torch.Tensor         # int32 [kv_indptr[B]]
+    kv_last_page_lens: torch.Tensor  # int32 [B]
+
+
+def mla_inputs(cfg: MlaConfig, device="cpu", spare_pages: int = 0) -> MlaInputs:
+    """Seeded inputs on `device`: q ~N(0, q_std) and every KV entry ~N(0, kv_std), rounded to
+    bf16, drawn in that order from one generator; then the page table, which hands the
+    sequences' pages out in a random order (a permutation drawn from a CPU generator with
+    the same seed), as a paged allocator would after some churn. `spare_pages` pages that
+    no sequence lists are added to the buffer. A sequence of L tokens holds ceil(L /
+    page_size) pages, its last one holding the rest (a full page when L is a multiple)."""
+    lens = cfg.lengths()
+    assert len(lens) == cfg.B
+    pages_of = [(n + cfg.page_size - 1) // cfg.page_size for n in lens]
+    n_pages = sum(pages_of) + spare_pages
+    g = torch.Generator(device=device).manual_seed(cfg.seed)
+    q = (torch.randn(cfg.B, cfg.Hq, cfg.Dk, generator=g, device=device) * cfg.q_std).to(torch.bfloat16)
+    kv = (torch.randn(max(n_pages, 1), cfg.page_size, 1, cfg.Dk, generator=g, device=device)
+          * cfg.kv_std).to(torch.bfloat16)
+    gc = torch.Generator(device="cpu").manual_seed(cfg.seed + 1)
+    perm = torch.randperm(max(n_pages, 1), generator=gc)[: sum(pages_of)].to(torch.int32)
+    indptr = torch.zeros(cfg.B + 1, dtype=torch.int32)
+    indptr[1:] = torch.cumsum(torch.tensor(pages_of, dtype=torch.int64), 0).to(torch.int32)
+    last = torch.tensor([(n - (p - 1) * cfg.page_size) if p else 0 for n, p in zip(lens, pages_of)],
+                        dtype=torch.int32)
+    return MlaInputs(q=q.contiguous(), kv_buffer=kv.contiguous(), kv_indptr=indptr.to(device),
+                     kv_indices=perm.to(device), kv_last_page_lens=last.to(device))
