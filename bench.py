@@ -1,6 +1,7 @@
 """Benchmark of the fused FP8 block-scaled MoE layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed|tiny|profile]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload prefill|decode|skewed|tiny|profile|gemm|mla_decode|mla_long|prefill_tp|prefill_ep]
                     [--tokens T] [--impl ours|reference]
 
 One step = one forward of the whole layer on the device: biased grouped top-k
@@ -16,6 +17,10 @@ events on the launching stream with a 256 MB L2 flush between steps (outside
 the events); barrier + synchronize around the whole timed loop; max over
 ranks. Under torchrun every rank runs its own batch of T tokens on its own
 full copy of the layer (weak scaling, no collective on the data path).
+
+--workload mla_decode / mla_long time the section's other decode kernel, MLA
+decode over a paged latent KV cache (64 sequences, 16 heads, 544 or 8192 cached
+tokens); the default run reports both under "workloads".
 
 --impl reference times the CPU oracle (the plain reference of the same
 computation) on the host cores on a bounded token sample of the same workload.
@@ -544,7 +549,7 @@ def measure_layer(args, world, local, cfg, layer, flush, headline=True):
 
 # The other workloads of the same layer timed by the default run, next to the prefill
 # headline: the decode and skewed batches (same expert weights) and the standalone GEMM.
-EXTRA_WORKLOADS = ("decode", "skewed", "gemm")
+EXTRA_WORKLOADS = ("decode", "skewed", "gemm", "mla_decode", "mla_long")
 EXTRA_KEYS = ("value", "unit", "ms_per_step", "steps", "warmup", "tflops", "step_ms", "layer_roofline", "roofline",
               "kernels_ms", "kernels_mcycles", "clocks", "config", "gpu_launches", "l2_warm")
 
@@ -833,6 +838,8 @@ def run_ours(args, world, rank, local):
         for name in EXTRA_WORKLOADS:
             if name == "gemm":
                 r = run_gemm(args, world, rank, local, cpu=False)
+            elif name in MLA_WORKLOADS:
+                r = run_mla(args, world, rank, local, MLA_WORKLOADS[name], cpu=False)
             else:
                 other = MoELayer(WORKLOADS[name], dev, weights_from=layer)
                 r = measure_layer(args, world, local, WORKLOADS[name], other, flush, headline=False)
@@ -997,6 +1004,163 @@ def run_gemm(args, world, rank, local, cpu=True):
     return result
 
 
+MLA_WORKLOADS = {"mla_decode": I.MLA_DECODE, "mla_long": I.MLA_LONG}
+MLA_METRIC = "MLA decode (paged latent KV, 576/512 head dims) sequences decoded/s at 1 B200; % of HBM roofline"
+
+
+def mla_work(cfg):
+    """Algorithmic bytes of one decode step: every cached KV row once, q, o, lse and the
+    page table (the split partials are the kernel's own traffic, not counted), and FLOPs:
+    QK^T over 576 entries and PV over 512 per head and token."""
+    rows = sum(cfg.lengths())
+    pages = sum((n + cfg.page_size - 1) // cfg.page_size for n in cfg.lengths())
+    nbytes = (rows * cfg.Dk * 2 + cfg.B * cfg.Hq * (cfg.Dk * 2 + cfg.Dv * 2 + 4)
+              + pages * 4 + (2 * cfg.B + 1) * 4)
+    flops = 2 * rows * cfg.Hq * (cfg.Dk + cfg.Dv)
+    return nbytes, flops
+
+
+class MlaOracleSample:
+    """The MLA oracle, as it stands, over the first n sequences of a workload (inputs drawn
+    once, untimed); step() times one decode of the sample."""
+
+    def __init__(self, cfg, n_seqs):
+        from oracle import mla_oracle as M
+        self.M = M
+        sub = I.MlaConfig(cfg.name + "_sample", B=n_seqs, Hq=cfg.Hq, L=tuple(cfg.lengths()[:n_seqs]),
+                          page_size=cfg.page_size, seed=cfg.seed)
+        self.x = I.mla_inputs(sub)
+        self.n = n_seqs
+
+    def step(self):
+        x = self.x
+        t0 = time.perf_counter()
+        self.M.mla_decode(x.q, x.kv_buffer, x.kv_indptr, x.kv_indices, x.kv_last_page_lens)
+        return time.perf_counter() - t0
+
+
+def run_mla(args, world, rank, local, cfg, cpu=True):
+    """MLA decode (mla_decode_fwd) on a seeded paged batch: device-timed steps with L2
+    flushed between them, the roofline of the call, end to end with q and the page
+    table copied in and o copied out, and the oracle's CPU baseline."""
+    from fp8_block_scaled_biased_b200 import binding as B
+
+    dev = torch.device("cuda", local)
+    x = I.mla_inputs(cfg, device=dev)
+    o = torch.empty(cfg.B, cfg.Hq, cfg.Dv, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(cfg.B, cfg.Hq, dtype=torch.float32, device=dev)
+    splits = B.mla_decode_num_splits(cfg.B, cfg.Hq)
+    need = B.mla_decode_workspace_bytes(cfg.B, cfg.Hq, splits)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        B.mla_decode_fwd(x.q, x.kv_buffer, o, x.kv_indptr, x.kv_indices, x.kv_last_page_lens, lse=lse,
+                         num_kv_splits=splits, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def timed(flush_l2):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        preheat(step, flush)
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            if flush_l2:
+                flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = [a.elapsed_time(b) for a, b in ev]
+        return max_over_ranks(sum(ms), world) / args.steps, ms
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    ms_flushed, per_step = timed(True)
+    clocks = sampler.stop()
+    ms_warm, _ = timed(False)
+    if B.device_status():
+        raise RuntimeError("device error word set by MLA decode")
+
+    # end to end: q and the page table from pinned host memory, o back to it (the KV cache stays resident)
+    h_in = [t.cpu().pin_memory() for t in (x.q, x.kv_indptr, x.kv_indices, x.kv_last_page_lens)]
+    h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0[i].record(stream)
+        for d, h in zip((x.q, x.kv_indptr, x.kv_indices, x.kv_last_page_lens), h_in):
+            d.copy_(h, non_blocking=True)
+        step()
+        h_o.copy_(o, non_blocking=True)
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), world) / args.steps
+
+    nbytes, flops = mla_work(cfg)
+    peaks = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    gbs = nbytes / (ms_flushed * 1e-3) / 1e9
+    result = {
+        "metric": MLA_METRIC,
+        "value": cfg.B * world / (ms_flushed * 1e-3), "unit": "sequences/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_flushed, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 x bf16 -> fp32 (softmax weights rounded to bf16), bf16 out",
+        "data": "synthetic (seeded)",
+        "config": {"workload": cfg.name, "B": cfg.B, "heads": cfg.Hq, "kv_len": cfg.L, "page_size": cfg.page_size,
+                   "qk_head_dim": cfg.Dk, "v_head_dim": cfg.Dv, "num_kv_splits": splits,
+                   "l2": "flushed between steps (256 MB write)", "parallelism": f"dp{world} (independent batches)"},
+        "tflops": flops / (ms_flushed * 1e-3) / 1e12,
+        "l2_warm": {"ms_per_step": ms_warm, "gbs": nbytes / (ms_warm * 1e-3) / 1e9},
+        "step_ms": {"median": statistics.median(per_step), "min": min(per_step), "max": max(per_step)},
+        "roofline": {"kernel": "mla_decode_fwd (decode kernel + split combine, timed together)", "bound": "hbm",
+                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "traffic": None,
+                     "algorithmic_bytes": nbytes, "peak_source": peaks["source"]},
+        "e2e": {"value": cfg.B * world / (e2e_ms * 1e-3), "unit": "sequences/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
+                "d2h_bytes_per_step": o.numel() * 2},
+        "gpu_launches": args.steps * (2 if splits > 1 else 1),
+        "clocks": clocks,
+    }
+    if cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        runner = MlaOracleSample(cfg, min(cfg.B, 8))
+        times = []
+        while sum(times) < 5.0:
+            times.append(runner.step())
+        sec = sum(times) / len(times)
+        result["cpu_baseline"] = {"value": runner.n / sec, "unit": "sequences/s", "cores": torch.get_num_threads(),
+                                  "kind": "oracle",
+                                  "sample": f"first {runner.n} sequences of {cfg.name}, {len(times)} passes in "
+                                            f"{sum(times):.1f} s"}
+    return result
+
+
+def run_reference_mla(args, world, cfg):
+    runner = MlaOracleSample(cfg, min(cfg.B, 4))
+    for _ in range(args.warmup):
+        runner.step()
+    times = [runner.step() for _ in range(args.steps)]
+    sec = statistics.mean(times)
+    value = runner.n / sec
+    return {
+        "impl": "reference", "metric": MLA_METRIC, "value": value, "unit": "sequences/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": cfg.name, "B": cfg.B, "heads": cfg.Hq, "kv_len": cfg.L, "page_size": cfg.page_size},
+        "cpu_baseline": {"value": value, "unit": "sequences/s", "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": f"first {runner.n} sequences of {cfg.name} per step"},
+        "e2e": {"value": value, "unit": "sequences/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference_gemm(args, world):
     """The oracle's block-scale GEMM on a fixed sample of 8 rows of A per step (operands quantised before timing)."""
     from oracle import fp8moe_oracle as O
@@ -1029,6 +1193,8 @@ def run_reference_gemm(args, world):
 def run_reference(args, world, rank):
     if args.workload == "gemm":
         return run_reference_gemm(args, world)
+    if args.workload in MLA_WORKLOADS:
+        return run_reference_mla(args, world, MLA_WORKLOADS[args.workload])
     cfg = workload_config(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     runner = OracleSample(cfg, args.ref_sample_tokens, device=dev)
@@ -1059,8 +1225,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DIST_WORKLOADS) + ["gemm"], default="prefill",
-                    help="MoE layer workload, or gemm: the standalone block-scale GEMM (M=2048, N=4096, K=7168)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DIST_WORKLOADS) + ["gemm"] + sorted(MLA_WORKLOADS),
+                    default="prefill",
+                    help="MoE layer workload; gemm: the standalone block-scale GEMM (M=2048, N=4096, K=7168); "
+                         "mla_decode / mla_long: MLA decode of 64 sequences of 544 / 8192 cached tokens, 16 heads")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the MoE workload's recipe at this many tokens (a batch-size sweep point; the "
                          "workloads timed beside the prefill headline are then left out)")
@@ -1079,7 +1247,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
-                    help="prefill only: leave out the decode, skewed and GEMM workloads timed beside the headline")
+                    help="prefill only: leave out the decode, skewed, GEMM and MLA decode workloads timed beside the "
+                         "headline")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8,
                     help="tokens of the workload the oracle runs for cpu_baseline")
     ap.add_argument("--ref-sample-tokens", type=int, default=1,
@@ -1103,7 +1272,12 @@ def main():
             if rank == 0:
                 print(json.dumps(run_reference(args, world, rank)), flush=True)
         else:
-            res = run_gemm(args, world, rank, local) if args.workload == "gemm" else run_ours(args, world, rank, local)
+            if args.workload == "gemm":
+                res = run_gemm(args, world, rank, local)
+            elif args.workload in MLA_WORKLOADS:
+                res = run_mla(args, world, rank, local, MLA_WORKLOADS[args.workload])
+            else:
+                res = run_ours(args, world, rank, local)
             if rank == 0:
                 print(json.dumps(res), flush=True)
     finally:

@@ -11,6 +11,7 @@ current torch CUDA stream.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from dataclasses import dataclass
 
@@ -68,6 +69,10 @@ _SIGNATURES = {
     "moe_ep_barrier": (_c_int, [_c_int, _c_int, _p, _p]),
     "moe_ep_barrier_emulated": (_c_int, [_c_int, _p, _p]),
     "moe_combine_pairs": (_c_int, [_p, _p, _c_int, _c_int, _c_int, _p, _p]),
+    "mla_decode_num_splits": (_c_int, [_c_int, _c_int]),
+    "mla_decode_workspace": (_c_size, [_c_int, _c_int, _c_int]),
+    "mla_decode_fwd": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                _c_float, _c_int, _p, _c_size, _p]),
 }
 EXPORTED = tuple(_SIGNATURES)
 
@@ -77,6 +82,8 @@ TP_FLAG_WORDS = 16                 # FP8MOE_TP_FLAG_WORDS (64-bit words per rank
 TP_BARRIER_WORDS = 3               # FP8MOE_TP_BARRIER_WORDS (arrivals, generation, calls)
 EP_MAX_RANKS = 8                   # FP8MOE_EP_MAX_RANKS
 EP_BARRIER_WORDS = 9               # FP8MOE_EP_BARRIER_WORDS (one per rank, then the calls)
+MLA_QK_HEAD_DIM = 576              # query/key width of the MLA decode call (512 latent + 64 rotary)
+MLA_V_HEAD_DIM = 512               # its value width
 SCALE_ROW_MAJOR = 0
 SCALE_COL_MAJOR = 1
 FP8 = torch.float8_e4m3fn
@@ -617,3 +624,54 @@ def moe_combine_pairs(rows, flag_region, T, topk, out):
     rc = load_library().moe_combine_pairs(_ptr(rows), _ptr(flag_region), T, topk, H, _ptr(out), _stream())
     _check("moe_combine_pairs", rc)
     return out
+
+
+def mla_decode_num_splits(batch, num_heads):
+    """The split count mla_decode_fwd uses when num_kv_splits is not given."""
+    return load_library().mla_decode_num_splits(batch, num_heads)
+
+
+def mla_decode_workspace_bytes(batch, num_heads, num_kv_splits=0):
+    return load_library().mla_decode_workspace(batch, num_heads, num_kv_splits)
+
+
+def mla_decode_fwd(q, kv_buffer, o, kv_indptr, kv_indices, kv_last_page_lens, sm_scale=None, logit_cap=0.0,
+                   num_kv_splits=0, lse=None, workspace=None):
+    """MLA decode: o bf16 [B, Hq, 512] from q bf16 [B, Hq, 576] and the paged latent KV
+    buffer bf16 [pages, page_size, 1, 576] (kv_indptr int32 [B+1], kv_indices int32,
+    kv_last_page_lens int32 [B]). sm_scale defaults to 1/sqrt(576); lse (fp32 [B, Hq],
+    optional) receives the log-sum-exp of the scores. Returns o."""
+    _cuda(q, torch.bfloat16, "q")
+    _cuda(kv_buffer, torch.bfloat16, "kv_buffer")
+    _cuda(o, torch.bfloat16, "o")
+    for t, name in ((kv_indptr, "kv_indptr"), (kv_indices, "kv_indices"), (kv_last_page_lens, "kv_last_page_lens")):
+        _cuda(t, torch.int32, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dim() != 3 or q.shape[2] != MLA_QK_HEAD_DIM or not q.is_contiguous():
+        raise ValueError(f"q must be a contiguous [B, Hq, {MLA_QK_HEAD_DIM}] tensor")
+    B, Hq = q.shape[0], q.shape[1]
+    if kv_buffer.dim() != 4 or kv_buffer.shape[2] != 1 or kv_buffer.shape[3] != MLA_QK_HEAD_DIM \
+            or not kv_buffer.is_contiguous():
+        raise ValueError(f"kv_buffer must be a contiguous [pages, page_size, 1, {MLA_QK_HEAD_DIM}] tensor")
+    if o.shape != (B, Hq, MLA_V_HEAD_DIM) or not o.is_contiguous():
+        raise ValueError(f"o must be a contiguous [{B}, {Hq}, {MLA_V_HEAD_DIM}] tensor")
+    if kv_indptr.numel() != B + 1 or kv_last_page_lens.numel() != B:
+        raise ValueError("kv_indptr must hold B+1 entries and kv_last_page_lens B")
+    if lse is not None:
+        _cuda(lse, torch.float32, "lse")
+        if lse.shape != (B, Hq) or not lse.is_contiguous():
+            raise ValueError(f"lse must be a contiguous [{B}, {Hq}] tensor")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(MLA_QK_HEAD_DIM)
+    need = mla_decode_workspace_bytes(B, Hq, num_kv_splits)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _cuda(workspace, torch.uint8, "workspace")
+    rc = load_library().mla_decode_fwd(
+        _ptr(q), _ptr(kv_buffer), _ptr(o), _ptr(kv_indptr), _ptr(kv_indices), _ptr(kv_last_page_lens), _ptr(lse),
+        B, Hq, kv_buffer.shape[0], kv_buffer.shape[1], kv_indices.numel(), float(sm_scale), float(logit_cap),
+        int(num_kv_splits), _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream())
+    _check("mla_decode_fwd", rc)
+    return o

@@ -4,7 +4,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -20,6 +22,7 @@
 #include "sort.cuh"
 #include "tp_reduce.cuh"
 #include "ep_peer.cuh"
+#include "mla_decode.cuh"
 
 static_assert(fp8moe::kMoeBlockRows == fp8moe::kBM, "sorted blocks are GEMM tiles");
 
@@ -106,6 +109,8 @@ int device_setup(int* sm_count) {
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, true>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, false, true>();
     if (r == cudaSuccess) r = enable_gemm_smem<kModeMoeDown, true, true>();
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmemBytes);
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sort_scatter_smem(kSortMaxExperts)));
@@ -1043,6 +1048,79 @@ int moe_combine_pairs(const uint16_t* rows, const void* flag_region, int T, int 
   moe_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const __nv_bfloat16*>(rows), flags, count, T, topk, H, reinterpret_cast<__nv_bfloat16*>(out));
   return check_launch("moe_combine_pairs");
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ MLA decode
+extern "C" {
+
+int mla_decode_num_splits(int batch, int num_heads) {
+  if (batch < 1 || num_heads < kMlaHeads) return 1;
+  const long long ctas = static_cast<long long>(batch) * (num_heads / kMlaHeads);
+  return static_cast<int>(std::max(1ll, std::min<long long>(kMlaMaxSplits, FP8MOE_MLA_TARGET_CTAS / ctas)));
+}
+
+size_t mla_decode_workspace(int batch, int num_heads, int num_kv_splits) {
+  const int splits = num_kv_splits > 0 ? num_kv_splits : mla_decode_num_splits(batch, num_heads);
+  if (batch < 1 || num_heads < 1 || splits <= 1) return 0;
+  return static_cast<size_t>(batch) * num_heads * splits * (kMlaDv + 1) * sizeof(float);
+}
+
+int mla_decode_fwd(const uint16_t* q, const uint16_t* kv_buffer, uint16_t* o, const int32_t* kv_indptr,
+                   const int32_t* kv_indices, const int32_t* kv_last_page_lens, float* lse, int batch, int num_heads,
+                   int num_pages, int page_size, int num_indices, float sm_scale, float logit_cap, int num_kv_splits,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch < 0 || num_pages < 0 || num_indices < 0) return fail(FP8MOE_EINVAL, "mla_decode_fwd: negative size");
+  if (num_heads < kMlaHeads || num_heads > 128 || num_heads % kMlaHeads)
+    return fail(FP8MOE_EUNSUPPORTED, "mla_decode_fwd: num_heads must be 16, 32, ..., 128 (got %d)", num_heads);
+  if (page_size < 1) return fail(FP8MOE_EINVAL, "mla_decode_fwd: page_size must be >= 1");
+  if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return fail(FP8MOE_EINVAL, "mla_decode_fwd: sm_scale must be finite and > 0");
+  if (!(logit_cap >= 0.0f) || !std::isfinite(logit_cap)) return fail(FP8MOE_EINVAL, "mla_decode_fwd: logit_cap must be finite and >= 0");
+  if (num_kv_splits > kMlaMaxSplits) return fail(FP8MOE_EUNSUPPORTED, "mla_decode_fwd: at most %d splits", kMlaMaxSplits);
+  if (batch == 0) return FP8MOE_OK;
+  if (batch > 65535) return fail(FP8MOE_EUNSUPPORTED, "mla_decode_fwd: batch above 65535");
+  if (!q || !o || !kv_indptr || !kv_last_page_lens) return fail(FP8MOE_EINVAL, "mla_decode_fwd: null pointer argument");
+  if ((num_indices > 0 && (!kv_indices || !kv_buffer || num_pages < 1)))
+    return fail(FP8MOE_EINVAL, "mla_decode_fwd: page indices given without a KV buffer");
+  if (!aligned16(q) || !aligned16(o) || (kv_buffer && !aligned16(kv_buffer)))
+    return fail(FP8MOE_EINVAL, "mla_decode_fwd: q, o and kv_buffer must be 16-byte aligned");
+  if (static_cast<long long>(num_pages) * page_size * kMlaDk >= (1ll << 40))
+    return fail(FP8MOE_EUNSUPPORTED, "mla_decode_fwd: KV buffer too large");
+  const int splits = num_kv_splits > 0 ? num_kv_splits : mla_decode_num_splits(batch, num_heads);
+  const size_t need = mla_decode_workspace(batch, num_heads, splits);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(FP8MOE_EWORKSPACE, "mla_decode_fwd: workspace of %zu bytes (16-byte aligned) needed", need);
+  int sms = 0;
+  if (int rc = device_setup(&sms)) return rc;
+  MlaArgs a{};
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.kv = reinterpret_cast<const __nv_bfloat16*>(kv_buffer);
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.indptr = kv_indptr;
+  a.indices = kv_indices;
+  a.last_lens = kv_last_page_lens;
+  a.part_o = need ? static_cast<float*>(workspace) : nullptr;
+  a.part_lse = need ? a.part_o + static_cast<size_t>(batch) * num_heads * splits * kMlaDv : nullptr;
+  a.B = batch;
+  a.Hq = num_heads;
+  a.num_pages = num_pages;
+  a.page_size = page_size;
+  a.num_indices = num_indices;
+  a.splits = splits;
+  a.sm_scale = sm_scale;
+  a.logit_cap = logit_cap;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(num_heads / kMlaHeads, splits, batch);
+  mla_decode_kernel<<<grid, kMlaThreads, kMlaSmemBytes, st>>>(a);
+  if (int rc = check_launch("mla_decode_fwd")) return rc;
+  if (splits > 1) {
+    const int bh = batch * num_heads;
+    mla_combine_kernel<<<(bh + 7) / 8, 256, 0, st>>>(a.part_o, a.part_lse, bh, splits, a.o, lse);
+    return check_launch("mla_decode_fwd (combine)");
+  }
+  return FP8MOE_OK;
 }
 
 }  // extern "C"

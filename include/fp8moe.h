@@ -58,7 +58,8 @@ enum fp8moe_device_error {
   FP8MOE_DEVERR_EXPERT_ID = 2u,   /* an expert id outside [0, E) was met          */
   FP8MOE_DEVERR_PAIR_ID = 4u,     /* a sorted pair id outside [0, T*topk] was met */
   FP8MOE_DEVERR_NUM_VALID = 8u,   /* num_valid_ids above capacity or not a multiple of block_m */
-  FP8MOE_DEVERR_BLOCK_ORDER = 16u /* sorted_expert_ids decreases somewhere: not a moe_align_sort result */
+  FP8MOE_DEVERR_BLOCK_ORDER = 16u, /* sorted_expert_ids decreases somewhere: not a moe_align_sort result */
+  FP8MOE_DEVERR_PAGE = 32u         /* MLA decode: a page-table entry outside its range (see mla_decode_fwd) */
 };
 
 /* Message describing the calling thread's most recent failure ("" if none). */
@@ -562,6 +563,53 @@ int moe_ep_barrier_emulated(int n, uint64_t* const* words, void* stream);
  * (a pair whose flag is 0 adds nothing). rows, out, flag_region 16-byte aligned. */
 int moe_combine_pairs(const uint16_t* rows, const void* flag_region, int T, int topk,
                       int H, uint16_t* out, void* stream);
+
+/* ---------------------------------------------------------------- MLA decode
+ * "Accelerate DeepSeek-R1 Inference: Integrate AITER into SGLang", section
+ * "Attention Mechanisms", subsection "MLA For Decode" (mla_decode_fwd(q,
+ * kv_buffer, o, kv_indptr, kv_indices, kv_last_page_lens, sm_scale, logit_cap,
+ * num_kv_splits)): multi-head latent attention for one decode step, the latent KV
+ * shared by every query head.
+ *
+ *   q            bf16 [batch, num_heads, 576], contiguous (512 latent + 64 rotary
+ *                entries per head, weights absorbed), 16-byte aligned
+ *   kv_buffer    bf16 [num_pages, page_size, 1, 576], contiguous, 16-byte aligned:
+ *                each row is a token's key; its first 512 entries are its value
+ *   o            bf16 [batch, num_heads, 512], contiguous, 16-byte aligned (output)
+ *   kv_indptr    int32 [batch + 1]: sequence b's pages are
+ *                kv_indices[kv_indptr[b] .. kv_indptr[b + 1]), in token order
+ *   kv_indices   int32 [num_indices], each in [0, num_pages)
+ *   kv_last_page_lens  int32 [batch]: tokens in each sequence's last page, in
+ *                [1, page_size] (ones for page_size 1, as in the section)
+ *   lse          fp32 [batch, num_heads] or NULL: ln(sum_j exp(s_j)) (output)
+ *   sm_scale     > 0 (the section's default is 1/sqrt(576))
+ *   logit_cap    0: scores unchanged; > 0: s -> logit_cap * tanh(s / logit_cap)
+ *   num_kv_splits  <= 0: mla_decode_num_splits(batch, num_heads); otherwise the
+ *                number of parts (<= 64) each sequence's tokens are split into,
+ *                merged by a second kernel (log-sum-exp weights, split order)
+ *   workspace    mla_decode_workspace(batch, num_heads, num_kv_splits) bytes
+ *                (0 when there is one split), 16-byte aligned
+ * The score of token j is s_j = sm_scale * <q, key_j> over the 576 entries, and
+ * o = sum_j softmax(s)_j value_j. A sequence with no page gets o = 0 and lse =
+ * -inf. num_heads must be a multiple of 16 up to 128 (FP8MOE_EUNSUPPORTED
+ * otherwise). Scores and sums are fp32; the softmax weights are rounded to bf16
+ * before they multiply the values (their running sum adds the rounded weights).
+ * A page-table entry out of range (an index outside [0, num_pages), kv_indptr not
+ * non-decreasing within [0, num_indices], a last-page length outside [1,
+ * page_size]) is not read: the device error word gets FP8MOE_DEVERR_PAGE and that
+ * sequence's output is unspecified. Deterministic: the same inputs give the same
+ * bits.
+ */
+#define FP8MOE_MLA_TARGET_CTAS 296   /* two resident CTAs on each of the B200's 148 SMs */
+int mla_decode_num_splits(int batch, int num_heads);
+size_t mla_decode_workspace(int batch, int num_heads, int num_kv_splits);
+int mla_decode_fwd(const uint16_t* q, const uint16_t* kv_buffer, uint16_t* o,
+                   const int32_t* kv_indptr, const int32_t* kv_indices,
+                   const int32_t* kv_last_page_lens, float* lse,
+                   int batch, int num_heads, int num_pages, int page_size,
+                   int num_indices, float sm_scale, float logit_cap,
+                   int num_kv_splits, void* workspace, size_t workspace_bytes,
+                   void* stream);
 
 #ifdef __cplusplus
 }

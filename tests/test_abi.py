@@ -213,3 +213,28 @@ def test_multi_gpu_entry_points_reject_bad_arguments(lib):
                                                    p, p, 128, 128, None, 1, None, None, p, 1 << 30, None) == 1
     assert lib.fused_moe_fp8_blockscale_g1u1_multi(one, one, 1, 10, p, p, p, p, p, p, 1024, 512, 4, 4, 128, 1 << 20,
                                                    p, p, 128, 128, None, 1, p, None, p, 1 << 30, None) == 1
+
+
+def test_mla_decode_rejects_bad_arguments_and_sizes_its_workspace(lib):
+    """The MLA decode entry point checks heads, sizes, scales, pointers, alignment and the
+    workspace on the host, and sizes the split partials by the stated formula."""
+    p = ctypes.c_void_p(16)
+    odd = ctypes.c_void_p(18)
+    assert lib.mla_decode_num_splits(64, 16) == 296 // 64
+    assert lib.mla_decode_num_splits(64, 128) == 1 and lib.mla_decode_num_splits(1, 16) == 64
+    assert lib.mla_decode_workspace(64, 16, 4) == 64 * 16 * 4 * 513 * 4
+    assert lib.mla_decode_workspace(64, 16, 1) == 0 and lib.mla_decode_workspace(64, 128, 0) == 0
+
+    def call(q=p, kv=p, o=p, ip=p, ix=p, ll=p, B=2, H=16, pages=4, ps=1, ni=4, scale=0.04, cap=0.0, splits=1,
+             ws=None, wsb=0):
+        return lib.mla_decode_fwd(q, kv, o, ip, ix, ll, None, B, H, pages, ps, ni, scale, cap, splits, ws, wsb, None)
+
+    assert call(H=8) == 2 and call(H=24) == 2 and call(H=144) == 2        # heads: 16, 32, ..., 128
+    assert call(ps=0) == 1 and call(B=-1) == 1 and call(ni=-1) == 1
+    assert call(scale=0.0) == 1 and call(scale=float("nan")) == 1 and call(cap=-1.0) == 1
+    assert call(splits=65) == 2
+    assert call(q=None) == 1 and call(ip=None) == 1 and call(kv=None) == 1
+    assert call(q=odd) == 1 and call(kv=odd) == 1
+    assert call(splits=2) == 3                                             # partials need a workspace
+    assert call(splits=2, ws=p, wsb=lib.mla_decode_workspace(2, 16, 2) - 1) == 3
+    assert call(B=0) == 0                                                  # nothing to do
