@@ -15,8 +15,9 @@
 //   - warp 0 issues one bulk asynchronous copy (cp.async.bulk, 1152 bytes) per
 //     row from wherever its page lies into a shared-memory stage, completing on
 //     the stage's mbarrier; two stages, so the next chunk's rows stream in while
-//     this one is computed. Rows past the split's end copy the chunk's first row
-//     instead (a finite value that gets weight 0);
+//     this one is computed, and a stage is refilled (chunk c + 2) as soon as every
+//     warp is past chunk c's P V. Rows past the split's end copy the chunk's first
+//     row instead (a finite value that gets weight 0);
 //   - S = Q K^T: warp w scores rows 8w..8w+7 for all 16 heads (36 MMAs over the
 //     576 entries, Q and K read from shared memory with ldmatrix);
 //   - online softmax in base 2: per-head maxima and sums meet across the warps in
@@ -244,11 +245,6 @@ __global__ void __launch_bounds__(kMlaThreads, 2) mla_decode_kernel(const __grid
       failed = true;
       break;
     }
-    // the previous chunk's stage is free: stream in the chunk after this one
-    if (c >= 1 && c + 1 < nchunks) {
-      if (warp == 0) mla_issue_chunk(a, smem, c + 1, row0, row1, page0);
-      issued = c + 2;
-    }
 
     float mnew[2], alpha[2];
 #pragma unroll
@@ -305,6 +301,12 @@ __global__ void __launch_bounds__(kMlaThreads, 2) mla_decode_kernel(const __grid
         mma_bf16_16816(o[n], pa, vb[0], vb[1]);
         mma_bf16_16816(o[n + 1], pa, vb[2], vb[3]);
       }
+    }
+    // this chunk's stage is free once every warp is past P V: stream in chunk c + 2
+    if (c + kMlaStages < nchunks) {
+      __syncthreads();
+      if (warp == 0) mla_issue_chunk(a, smem, c + kMlaStages, row0, row1, page0);
+      issued = c + kMlaStages + 1;
     }
   }
 
