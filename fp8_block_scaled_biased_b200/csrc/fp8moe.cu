@@ -1087,6 +1087,8 @@ int mla_decode_fwd(const uint16_t* q, const uint16_t* kv_buffer, uint16_t* o, co
     return fail(FP8MOE_EINVAL, "mla_decode_fwd: q, o and kv_buffer must be 16-byte aligned");
   if (static_cast<long long>(num_pages) * page_size * kMlaDk >= (1ll << 40))
     return fail(FP8MOE_EUNSUPPORTED, "mla_decode_fwd: KV buffer too large");
+  if (static_cast<long long>(num_indices) * page_size >= (1ll << 31))   // token positions are int32 in the kernel
+    return fail(FP8MOE_EUNSUPPORTED, "mla_decode_fwd: num_indices x page_size must stay below 2^31");
   const int splits = num_kv_splits > 0 ? num_kv_splits : mla_decode_num_splits(batch, num_heads);
   const size_t need = mla_decode_workspace(batch, num_heads, splits);
   if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))

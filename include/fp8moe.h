@@ -591,8 +591,8 @@ int moe_combine_pairs(const uint16_t* rows, const void* flag_region, int T, int 
  *                (0 when there is one split), 16-byte aligned
  * The score of token j is s_j = sm_scale * <q, key_j> over the 576 entries, and
  * o = sum_j softmax(s)_j value_j. A sequence with no page gets o = 0 and lse =
- * -inf. num_heads must be a multiple of 16 up to 128 (FP8MOE_EUNSUPPORTED
- * otherwise). Scores and sums are fp32; the softmax weights are rounded to bf16
+ * -inf. num_heads must be a multiple of 16 up to 128, batch at most 65535 and
+ * num_indices * page_size below 2^31 (FP8MOE_EUNSUPPORTED otherwise). Scores and sums are fp32; the softmax weights are rounded to bf16
  * before they multiply the values (their running sum adds the rounded weights).
  * A page-table entry out of range (an index outside [0, num_pages), kv_indptr not
  * non-decreasing within [0, num_indices], a last-page length outside [1,

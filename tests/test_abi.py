@@ -237,4 +237,6 @@ def test_mla_decode_rejects_bad_arguments_and_sizes_its_workspace(lib):
     assert call(q=odd) == 1 and call(kv=odd) == 1
     assert call(splits=2) == 3                                             # partials need a workspace
     assert call(splits=2, ws=p, wsb=lib.mla_decode_workspace(2, 16, 2) - 1) == 3
+    assert call(ni=1 << 20, ps=4096) == 2                                  # token positions past int32
+    assert call(B=70000) == 2
     assert call(B=0) == 0                                                  # nothing to do
