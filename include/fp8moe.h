@@ -9,7 +9,8 @@
  * the MI300X "fnuz" variant. The tensor- and expert-parallel entry points at the
  * end follow the same page's TP8 run and custom all-reduce ("Performance
  * Reproduction for AITER-Optimized in SGLang", "Other Operators") and asm_moe's
- * expert_mask.
+ * expert_mask. The MLA decode entry point at the very end follows the same page's
+ * section "Attention Mechanisms" ("MLA For Decode").
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller; the library never
@@ -54,7 +55,7 @@ enum fp8moe_status {
 
 /* Device error word bits reported by fp8moe_device_status(). */
 enum fp8moe_device_error {
-  FP8MOE_DEVERR_TIMEOUT = 1u,     /* a bounded wait inside a GEMM kernel expired  */
+  FP8MOE_DEVERR_TIMEOUT = 1u,     /* a bounded wait inside a kernel expired       */
   FP8MOE_DEVERR_EXPERT_ID = 2u,   /* an expert id outside [0, E) was met          */
   FP8MOE_DEVERR_PAIR_ID = 4u,     /* a sorted pair id outside [0, T*topk] was met */
   FP8MOE_DEVERR_NUM_VALID = 8u,   /* num_valid_ids above capacity or not a multiple of block_m */
