@@ -162,3 +162,24 @@ def test_ep_emulate_option_is_checked():
                 ["--workload", "prefill_ep", "--ep-emulate", "3"]):
         r = subprocess.run([sys.executable, "bench.py", *bad], cwd=ROOT, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0 and "--ep-emulate" in r.stderr, bad
+
+
+def test_mla_work_counts_by_hand():
+    """MLA decode's algorithmic bytes: KV rows once, q, o, lse and the page table."""
+    nbytes, flops = bench.mla_work(I.MLA_DECODE)
+    rows = 64 * 544
+    assert nbytes == rows * 1152 + 64 * 16 * (1152 + 1024 + 4) + rows * 4 + (2 * 64 + 1) * 4 == 42_480_132
+    assert flops == 2 * rows * 16 * (576 + 512)
+    cfg = I.MlaConfig("t", B=3, Hq=32, L=(0, 5, 17), page_size=4)
+    nbytes, _ = bench.mla_work(cfg)
+    assert nbytes == 22 * 1152 + 3 * 32 * 2180 + (0 + 2 + 5) * 4 + 7 * 4
+
+
+def test_reference_arm_mla_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "mla_decode",
+                        "--steps", "2", "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "sequences/s" and line["value"] > 0
+    assert line["config"]["workload"] == I.MLA_DECODE.name
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
